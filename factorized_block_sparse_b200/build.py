@@ -1,0 +1,53 @@
+"""Builds the in-tree shared library ``libsparse_attn.so`` for sm_100a.
+
+One nvcc invocation compiles the CUDA translation unit (kernels and C ABI)
+and the host layout builder.  The CUDA runtime is linked statically and the
+driver is reached through ``cudaGetDriverEntryPoint``, so the library loads
+on a host without a GPU (for the CPU tests of the layout builder and the
+exported symbols) and needs only the NVIDIA driver on a GPU host.
+"""
+
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB = os.path.join(HERE, "libsparse_attn.so")
+SOURCES = [os.path.join(HERE, "csrc", "sa_api.cu"), os.path.join(HERE, "csrc", "sa_layout.cpp")]
+HEADERS = [os.path.join(ROOT, "include", "sparse_attn.h")] + [
+    os.path.join(HERE, "csrc", f) for f in ("sa_internal.h", "sa_device.cuh", "sa_fwd.cuh", "sa_bwd.cuh")]
+
+
+def nvcc_path():
+    cand = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    return cand if os.path.exists(cand) else "nvcc"
+
+
+def command(out=LIB, extra=()):
+    return [nvcc_path(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+            "-lineinfo", "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static",
+            "-I", os.path.join(ROOT, "include"), "-o", out, *extra, *SOURCES]
+
+
+def up_to_date(out=LIB):
+    if not os.path.exists(out):
+        return False
+    t = os.path.getmtime(out)
+    return all(os.path.getmtime(p) <= t for p in SOURCES + HEADERS)
+
+
+def build(force=False, verbose=False, extra=()):
+    """Compile the library if any source is newer than it; return its path."""
+    if not force and up_to_date():
+        return LIB
+    cmd = command(extra=list(extra))
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv, verbose=True,
+          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])

@@ -1,0 +1,577 @@
+// C ABI of the factorized sparse attention library (declared in
+// include/sparse_attn.h): argument checks, TMA tensor maps, per-device
+// copies of the layout tables, kernel launches, the device status word and
+// launch instrumentation.  All device code is in this translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "sa_bwd.cuh"
+#include "sa_device.cuh"
+#include "sa_fwd.cuh"
+#include "sa_internal.h"
+#include "sparse_attn.h"
+
+namespace sa {
+namespace {
+
+// ------------------------------------------------------------ instrumentation
+enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_FINAL, K_NUM };
+const char* const kKindNames[K_NUM] = {"sa_fwd_column_view", "sa_fwd_natural_view",
+                                       "sa_bwd_preprocess",  "sa_bwd_secondary_view",
+                                       "sa_bwd_natural_view", "sa_bwd_finalize_dq"};
+
+struct Pending {
+  int kind;
+  cudaEvent_t e0, e1;
+};
+
+struct Timing {
+  std::mutex mu;
+  bool on = false;
+  std::vector<Pending> pending;
+  std::vector<cudaEvent_t> pool;
+  double total_ms[K_NUM] = {};
+  long long count[K_NUM] = {};
+};
+Timing g_timing;
+std::atomic<long long> g_launches{0};
+
+cudaEvent_t take_event() {
+  if (!g_timing.pool.empty()) {
+    cudaEvent_t e = g_timing.pool.back();
+    g_timing.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+void drain_timing_locked() {
+  for (auto& p : g_timing.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(p.e1) == cudaSuccess && cudaEventElapsedTime(&ms, p.e0, p.e1) == cudaSuccess) {
+      g_timing.total_ms[p.kind] += ms;
+      g_timing.count[p.kind] += 1;
+    }
+    g_timing.pool.push_back(p.e0);
+    g_timing.pool.push_back(p.e1);
+  }
+  g_timing.pending.clear();
+}
+
+template <class F>
+int launch(int kind, cudaStream_t s, F&& f) {
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  bool timed = false;
+  {
+    std::lock_guard<std::mutex> g(g_timing.mu);
+    if (g_timing.on) {
+      e0 = take_event();
+      e1 = take_event();
+      timed = (e0 && e1);
+    }
+  }
+  if (timed) cudaEventRecord(e0, s);
+  f();
+  const cudaError_t err = cudaGetLastError();
+  g_launches.fetch_add(1);
+  if (timed) {
+    cudaEventRecord(e1, s);
+    std::lock_guard<std::mutex> g(g_timing.mu);
+    g_timing.pending.push_back({kind, e0, e1});
+  }
+  return err == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool have_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+struct Geo {
+  int BH, N, D, l, c, R;
+  int boxw;
+  CUtensorMapSwizzle swz;
+};
+
+// Natural order: {D, N, BH}, box {boxw, rows, 1}.
+int map_nat(CUtensorMap* m, const void* base, const Geo& g, int rows) {
+  const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.N * g.D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)g.boxw, (cuuint32_t)rows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                        es, CU_TENSOR_MAP_INTERLEAVE_NONE, g.swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SA_OK : SA_ERR_CUDA;
+}
+
+// The sequence as a 2-D array with rows of length l: {D, l, R, BH}.
+// Column view box {boxw, 1, min(R, rows), 1}; summary box
+// {boxw, min(c, rows), max(1, rows / c), 1}.
+int map_grid(CUtensorMap* m, const void* base, const Geo& g, uint32_t b1, uint32_t b2) {
+  const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
+  const cuuint64_t strides[3] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.l * g.D * 2, (cuuint64_t)g.N * g.D * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)g.boxw, b1, b2, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                        es, CU_TENSOR_MAP_INTERLEAVE_NONE, g.swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SA_OK : SA_ERR_CUDA;
+}
+
+struct MapSet {
+  CUtensorMap nat, col, sum;
+};
+
+int make_maps(MapSet* ms, const void* base, const Geo& g, int pattern, int rows) {
+  std::memset(ms, 0, sizeof(*ms));
+  int st = map_nat(&ms->nat, base, g, rows);
+  if (st) return st;
+  if (pattern == SA_STRIDED) {
+    st = map_grid(&ms->col, base, g, 1, (uint32_t)std::min(g.R, rows));
+    if (st) return st;
+  }
+  if (pattern == SA_FIXED) {
+    st = map_grid(&ms->sum, base, g, (uint32_t)std::min(g.c, rows), (uint32_t)std::max(1, rows / g.c));
+    if (st) return st;
+  }
+  return SA_OK;
+}
+
+// ------------------------------------------------------------ device tables
+int to_device(const sa_layout* L, DeviceCopy* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+  std::lock_guard<std::mutex> g(L->mu);
+  for (auto& d : L->dev)
+    if (d.device == dev) {
+      *out = d;
+      return SA_OK;
+    }
+  const TileTable* tabs[4] = {&L->fwd_main, &L->fwd_col, &L->bwd_main, &L->bwd_sec};
+  std::vector<int32_t> blob;
+  size_t offs[4][3];
+  for (int t = 0; t < 4; ++t) {
+    const TileTable& tt = *tabs[t];
+    offs[t][0] = blob.size();
+    blob.insert(blob.end(), tt.row_ptr.begin(), tt.row_ptr.end());
+    offs[t][1] = blob.size();
+    blob.insert(blob.end(), tt.ent.begin(), tt.ent.end());
+    offs[t][2] = blob.size();
+    blob.insert(blob.end(), tt.order.begin(), tt.order.end());
+    while (blob.size() % 4) blob.push_back(0);
+  }
+  if (blob.empty()) blob.push_back(0);
+  void* dptr = nullptr;
+  if (cudaMalloc(&dptr, blob.size() * sizeof(int32_t)) != cudaSuccess) return SA_ERR_CUDA;
+  if (cudaMemcpy(dptr, blob.data(), blob.size() * sizeof(int32_t), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(dptr);
+    return SA_ERR_CUDA;
+  }
+  DeviceCopy d;
+  d.device = dev;
+  d.blob = dptr;
+  DevTable* dts[4] = {&d.fwd_main, &d.fwd_col, &d.bwd_main, &d.bwd_sec};
+  const int32_t* base = static_cast<const int32_t*>(dptr);
+  for (int t = 0; t < 4; ++t) {
+    dts[t]->row_ptr = base + offs[t][0];
+    dts[t]->ent = base + offs[t][1];
+    dts[t]->order = base + offs[t][2];
+    dts[t]->n_rows = tabs[t]->n_rows;
+    dts[t]->nnz = static_cast<int>(tabs[t]->ent.size());
+  }
+  L->dev.push_back(d);
+  *out = d;
+  return SA_OK;
+}
+
+// ------------------------------------------------------------ checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_call(int B, int H, int N, int D, const sa_layout* L) {
+  if (!L || B < 1 || H < 1 || N < 1) return SA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return SA_ERR_INVALID_ARG;
+  if (L->N != N) return SA_ERR_LUT;
+  if (D != 32 && D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+  if (L->pattern == SA_STRIDED) {
+    const int R = L->R;
+    if (R % 8 != 0 || !(R % 128 == 0 || 128 % R == 0)) return SA_ERR_UNSUPPORTED;
+  }
+  if (L->pattern == SA_FIXED) {
+    const int c = L->c;
+    if (!(64 % c == 0 || c % 128 == 0)) return SA_ERR_UNSUPPORTED;
+  }
+  if (!have_encode()) return SA_ERR_CUDA;
+  return SA_OK;
+}
+
+Geo make_geo(int B, int H, int N, int D, const sa_layout* L) {
+  Geo g;
+  g.BH = B * H;
+  g.N = N;
+  g.D = D;
+  g.l = (L->pattern == SA_ALL) ? 1 : L->l;
+  g.c = L->c > 0 ? L->c : 1;
+  g.R = (L->pattern == SA_STRIDED || L->pattern == SA_FIXED) ? L->R : 1;
+  g.boxw = D >= 64 ? 64 : D;
+  g.swz = D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return g;
+}
+
+template <class K>
+int set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+             ? SA_OK
+             : SA_ERR_CUDA;
+}
+
+template <int D>
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+             const sa_layout* L, cudaStream_t s) {
+  const Geo g = make_geo(B, H, N, D, L);
+  MapSet mq, mk, mv;
+  int st;
+  if ((st = make_maps(&mq, q, g, L->pattern, FwdCfg<D>::TQ))) return st;
+  if ((st = make_maps(&mk, k, g, L->pattern, FwdCfg<D>::TK))) return st;
+  if ((st = make_maps(&mv, v, g, L->pattern, FwdCfg<D>::TK))) return st;
+  DeviceCopy dc;
+  if ((st = to_device(L, &dc))) return st;
+  auto kern = sa_fwd_kernel<D>;
+  if ((st = set_smem(kern, FwdCfg<D>::SMEM))) return st;
+  FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.N = N;
+  a.l = g.l;
+  a.c = g.c;
+  a.R = g.R;
+  a.pattern = L->pattern;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  const bool two_pass = (L->pattern == SA_STRIDED);
+  if (two_pass && dc.fwd_col.n_rows > 0) {
+    a.row_ptr = dc.fwd_col.row_ptr;
+    a.ent = dc.fwd_col.ent;
+    a.order = dc.fwd_col.order;
+    a.q_col = 1;
+    a.merge = 0;
+    dim3 grid(g.BH, dc.fwd_col.n_rows);
+    st = launch(K_FWD_COL, s, [&] {
+      kern<<<grid, 192, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
+    });
+    if (st) return st;
+  }
+  a.row_ptr = dc.fwd_main.row_ptr;
+  a.ent = dc.fwd_main.ent;
+  a.order = dc.fwd_main.order;
+  a.q_col = 0;
+  a.merge = (two_pass && dc.fwd_col.n_rows > 0) ? 1 : 0;
+  dim3 grid(g.BH, dc.fwd_main.n_rows);
+  return launch(K_FWD_MAIN, s, [&] {
+    kern<<<grid, 192, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
+  });
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t delta, dq, dk, dv, total;
+};
+
+WsLayout ws_layout(int B, int H, int N, int D, const sa_layout* L) {
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  WsLayout w;
+  w.delta = 0;
+  w.dq = align256(rows * 4);
+  w.dk = w.dq + align256(rows * D * 4);
+  const bool sec = L->pattern == SA_STRIDED || L->pattern == SA_FIXED;
+  w.dv = w.dk + (sec ? align256(rows * D * 4) : 0);
+  w.total = w.dv + (sec ? align256(rows * D * 4) : 0);
+  return w;
+}
+
+int grid_for(long long work_items, int per_block) {
+  long long b = (work_items + per_block - 1) / per_block;
+  if (b < 1) b = 1;
+  if (b > 148 * 16) b = 148 * 16;
+  return static_cast<int>(b);
+}
+
+template <int D>
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+             void* dq, void* dk, void* dv, int B, int H, int N, const sa_layout* L, void* ws, cudaStream_t s) {
+  const Geo g = make_geo(B, H, N, D, L);
+  MapSet mq, mdo, mk, mv;
+  int st;
+  if ((st = make_maps(&mq, q, g, L->pattern, 128))) return st;
+  if ((st = make_maps(&mdo, dO, g, L->pattern, 128))) return st;
+  if ((st = make_maps(&mk, k, g, L->pattern, 128))) return st;
+  if ((st = make_maps(&mv, v, g, L->pattern, 128))) return st;
+  DeviceCopy dc;
+  if ((st = to_device(L, &dc))) return st;
+  auto kern = sa_bwd_kernel<D>;
+  if ((st = set_smem(kern, BwdCfg<D>::SMEM))) return st;
+  const WsLayout w = ws_layout(B, H, N, D, L);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* delta = reinterpret_cast<float*>(wsb + w.delta);
+  float* dq_acc = reinterpret_cast<float*>(wsb + w.dq);
+  float* dk_part = reinterpret_cast<float*>(wsb + w.dk);
+  float* dv_part = reinterpret_cast<float*>(wsb + w.dv);
+  const long long rows = static_cast<long long>(g.BH) * N;
+
+  st = launch(K_BWD_PRE, s, [&] {
+    sa_bwd_pre_kernel<D><<<grid_for(rows * (D / 8), 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows);
+  });
+  if (st) return st;
+
+  BwdArgs a;
+  a.lse = lse;
+  a.delta = delta;
+  a.dq_acc = dq_acc;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dk_part = dk_part;
+  a.dv_part = dv_part;
+  a.N = N;
+  a.l = g.l;
+  a.c = g.c;
+  a.R = g.R;
+  a.pattern = L->pattern;
+  a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  const bool sec = (L->pattern == SA_STRIDED || L->pattern == SA_FIXED) && dc.bwd_sec.n_rows > 0;
+  if (sec) {
+    a.row_ptr = dc.bwd_sec.row_ptr;
+    a.ent = dc.bwd_sec.ent;
+    a.order = dc.bwd_sec.order;
+    a.key_view = (L->pattern == SA_STRIDED) ? SRC_T : SRC_S;
+    a.add_part = 0;
+    dim3 grid(g.BH, dc.bwd_sec.n_rows);
+    st = launch(K_BWD_SEC, s, [&] {
+      kern<<<grid, 192, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
+                                               mv.col, mv.sum, a);
+    });
+    if (st) return st;
+  }
+  a.row_ptr = dc.bwd_main.row_ptr;
+  a.ent = dc.bwd_main.ent;
+  a.order = dc.bwd_main.order;
+  a.key_view = SRC_N;
+  a.add_part = sec ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
+  {
+    dim3 grid(g.BH, dc.bwd_main.n_rows);
+    st = launch(K_BWD_MAIN, s, [&] {
+      kern<<<grid, 192, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
+                                               mv.col, mv.sum, a);
+    });
+    if (st) return st;
+  }
+  const long long n8 = rows * D / 8;
+  return launch(K_BWD_FINAL, s, [&] {
+    sa_bwd_final_kernel<<<grid_for(n8, 256), 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  });
+}
+
+}  // namespace
+}  // namespace sa
+
+// ==================================================================== C ABI
+using namespace sa;
+
+extern "C" {
+
+int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** out) {
+  if (!out) return SA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (pattern < SA_ALL || pattern > SA_FIXED || N < 1 || block < 1) return SA_ERR_INVALID_ARG;
+  if (pattern != SA_ALL && l < 1) return SA_ERR_INVALID_ARG;
+  if (pattern == SA_FIXED && (c < 1 || c > l)) return SA_ERR_INVALID_ARG;
+  if (N % block != 0) return SA_ERR_UNSUPPORTED;
+  if ((pattern == SA_STRIDED || pattern == SA_FIXED) && N % l != 0) return SA_ERR_UNSUPPORTED;
+  sa_layout* L = new (std::nothrow) sa_layout();
+  if (!L) return SA_ERR_INVALID_ARG;
+  L->pattern = pattern;
+  L->N = N;
+  L->l = (pattern == SA_ALL) ? 1 : l;
+  L->c = (pattern == SA_FIXED) ? c : 0;
+  L->block = block;
+  L->R = (pattern == SA_STRIDED || pattern == SA_FIXED) ? N / l : 1;
+  const int st = build_layout(L);
+  if (st != SA_OK) {
+    delete L;
+    return st;
+  }
+  *out = L;
+  return SA_OK;
+}
+
+int sparse_attn_layout_export(const sa_layout* L, int view, int32_t* row_ptr, int32_t* col_idx, uint8_t* kind,
+                              int* n_rows, int* nnzb) {
+  if (!L || !n_rows || !nnzb) return SA_ERR_INVALID_ARG;
+  const int v = view & 3;
+  const bool tr = (view & SA_VIEW_TRANSPOSED) != 0;
+  if (v > SA_VIEW_SUMMARY || (view & ~(3 | SA_VIEW_TRANSPOSED))) return SA_ERR_INVALID_ARG;
+  if (!L->has[v]) {
+    *n_rows = 0;
+    *nnzb = 0;
+    if (row_ptr) row_ptr[0] = 0;
+    return SA_OK;
+  }
+  const Csr& t = tr ? L->viewT[v] : L->view[v];
+  *n_rows = t.n_rows;
+  *nnzb = static_cast<int>(t.col_idx.size());
+  if (row_ptr) std::memcpy(row_ptr, t.row_ptr.data(), t.row_ptr.size() * sizeof(int32_t));
+  if (col_idx && !t.col_idx.empty()) std::memcpy(col_idx, t.col_idx.data(), t.col_idx.size() * sizeof(int32_t));
+  if (kind && !t.kind.empty()) std::memcpy(kind, t.kind.data(), t.kind.size());
+  return SA_OK;
+}
+
+int sparse_attn_layout_info(const sa_layout* L, int* pattern, int* N, int* l, int* c, int* block) {
+  if (!L) return SA_ERR_INVALID_ARG;
+  if (pattern) *pattern = L->pattern;
+  if (N) *N = L->N;
+  if (l) *l = L->l;
+  if (c) *c = L->c;
+  if (block) *block = L->block;
+  return SA_OK;
+}
+
+int sparse_attn_layout_upload(const sa_layout* L, void* stream) {
+  (void)stream;
+  if (!L) return SA_ERR_INVALID_ARG;
+  DeviceCopy dc;
+  return to_device(L, &dc);
+}
+
+void sparse_attn_layout_free(sa_layout* L) {
+  if (!L) return;
+  int cur = -1;
+  const bool have = cudaGetDevice(&cur) == cudaSuccess;
+  for (auto& d : L->dev) {
+    if (cudaSetDevice(d.device) == cudaSuccess) {
+      cudaDeviceSynchronize();
+      cudaFree(d.blob);
+    }
+  }
+  if (have && !L->dev.empty()) cudaSetDevice(cur);
+  delete L;
+}
+
+int sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
+                    const sa_layout* L, void* stream) {
+  if (!q || !k || !v || !o || !lse) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return SA_ERR_INVALID_ARG;
+  int st = check_call(B, H, N, D, L);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (D) {
+    case 32: return fwd_impl<32>(q, k, v, o, lse, B, H, N, L, s);
+    case 64: return fwd_impl<64>(q, k, v, o, lse, B, H, N, L, s);
+    default: return fwd_impl<128>(q, k, v, o, lse, B, H, N, L, s);
+  }
+}
+
+size_t sparse_attn_bwd_workspace_size(int B, int H, int N, int D, const sa_layout* L) {
+  if (!L || B < 1 || H < 1 || N < 1 || D < 1) return 0;
+  return ws_layout(B, H, N, D, L).total;
+}
+
+int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, int B, int H, int N, int D, const sa_layout* L, void* workspace,
+                    size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return SA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SA_ERR_INVALID_ARG;
+  int st = check_call(B, H, N, D, L);
+  if (st) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+      ws_bytes < sparse_attn_bwd_workspace_size(B, H, N, D, L))
+    return SA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (D) {
+    case 32: return bwd_impl<32>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, L, workspace, s);
+    case 64: return bwd_impl<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, L, workspace, s);
+    default: return bwd_impl<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, L, workspace, s);
+  }
+}
+
+int sparse_attn_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+    return v;
+  }
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+const char* sparse_attn_strerror(int status) {
+  switch (status) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case SA_ERR_CUDA: return "CUDA error";
+    case SA_ERR_LUT: return "layout does not match the call";
+    case SA_ERR_TIMEOUT: return "device-side wait timed out";
+    case SA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int sparse_attn_kernel_kinds(void) { return K_NUM; }
+
+int sparse_attn_timing_enable(int on) {
+  std::lock_guard<std::mutex> g(g_timing.mu);
+  g_timing.on = (on != 0);
+  return SA_OK;
+}
+
+int sparse_attn_timing_reset(void) {
+  std::lock_guard<std::mutex> g(g_timing.mu);
+  drain_timing_locked();
+  for (int i = 0; i < K_NUM; ++i) {
+    g_timing.total_ms[i] = 0;
+    g_timing.count[i] = 0;
+  }
+  return SA_OK;
+}
+
+int sparse_attn_timing_read(int kind, const char** name, double* total_ms, long long* launches) {
+  if (kind < 0 || kind >= K_NUM) return SA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> g(g_timing.mu);
+  drain_timing_locked();
+  if (name) *name = kKindNames[kind];
+  if (total_ms) *total_ms = g_timing.total_ms[kind];
+  if (launches) *launches = g_timing.count[kind];
+  return SA_OK;
+}
+
+long long sparse_attn_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

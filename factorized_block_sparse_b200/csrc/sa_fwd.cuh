@@ -1,0 +1,419 @@
+// Forward kernel: fused online-softmax block-sparse attention on tcgen05.
+//
+// One CTA = one 128-row query tile of one (batch, head), in the view order
+// of its table (natural, or column-major for the strided column view).  It
+// walks the tile's list of 64-key tiles.  Per key tile:
+//   S = Q K^T            tcgen05.mma, bf16 in smem -> fp32 in TMEM
+//   mask (PARTIAL only), running max, P = exp2(S*scale*log2e - m) -> bf16
+//   O += P V             tcgen05.mma, P staged in 128B-swizzled smem
+// This is masked softmax attention restricted to the nonzero blocks of the
+// layout ("OpenAI Sparse Transformer", "Sparse Attention and Algorithmic
+// Complexity" and "Implementation and Limitations").
+//
+// Roles (192 threads):
+//   warp 0 lane 0 : TMA producer (Q once, K/V through a STAGES-deep ring)
+//   warp 1        : allocates TMEM; lane 0 issues every tcgen05.mma
+//   warps 2..5    : softmax; thread t of warp w owns query row
+//                   32*(w%4)+t, which is TMEM lane 32*(w%4)+t.
+// TMEM columns: S double buffer [0,64) and [64,128); O accumulator [128,128+D).
+//
+// The running max is only moved when it grows by more than 2^8 (in the
+// exp2 domain), so O is rescaled rarely; the final normalisation uses the
+// same max, so the result is exact up to rounding.
+#pragma once
+
+#include "sa_device.cuh"
+
+namespace sa {
+
+struct FwdArgs {
+  const int32_t* row_ptr;
+  const int32_t* ent;
+  const int32_t* order;
+  __nv_bfloat16* o;
+  float* lse;
+  int N, l, c, R;
+  int pattern;  // sa_pattern
+  int q_col;    // 1: query tiles are in column-major (T) order
+  int merge;    // 1: combine with the partial (o, lse) already stored
+  float scale_log2;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int TQ = 128, TK = 64;
+  static constexpr int STAGES = (D >= 128) ? 2 : 3;
+  static constexpr int ROWB = (D >= 64) ? 128 : 64;     // bytes per row per panel
+  static constexpr int PANELS = (D >= 64) ? D / 64 : 1;
+  static constexpr int BOXW = (D >= 64) ? 64 : D;       // TMA box inner width (elements)
+  static constexpr uint64_t SWZ = (D >= 64) ? kSwizzle128 : kSwizzle64;
+  static constexpr int SBO = 8 * ROWB;
+  static constexpr int Q_BYTES = TQ * D * 2;
+  static constexpr int KV_BYTES = TK * D * 2;
+  static constexpr int P_BYTES = TQ * TK * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int N_BARS = 1 + 3 * STAGES + 8;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int TMEM_COLS = 256;
+  static constexpr int COL_O = 128;
+};
+
+// Loads a tile of `rows` positions starting at view position `pos0` into
+// `dst` (PANELS panels of rows x ROWB bytes).
+//   src N: natural order, 3-D map {D, N, BH}, box {BOXW, rows, 1}
+//   src T: column-major order, 4-D map {D, l, R, BH}, box {BOXW, 1, RB, 1}
+//          with RB = min(R, rows): one load per column segment
+//   src S: summary order, 4-D map {D, l, R, BH}, box {BOXW, CB, GB, 1} with
+//          CB = min(c, rows), GB = max(1, rows / c)
+template <int D>
+__device__ __forceinline__ void load_rows(uint8_t* dst, int src, int pos0, int rows, int bh,
+                                          const CUtensorMap* m_nat, const CUtensorMap* m_col,
+                                          const CUtensorMap* m_sum, uint64_t* bar, int R, int l,
+                                          int c) {
+  using C = FwdCfg<D>;
+  const int panel_bytes = rows * C::ROWB;
+#pragma unroll
+  for (int p = 0; p < C::PANELS; ++p) {
+    uint8_t* d = dst + p * panel_bytes;
+    const int x = p * 64;
+    if (src == SRC_N) {
+      tma_load_3d(d, m_nat, bar, x, pos0, bh);
+    } else if (src == SRC_T) {
+      const int rb = R < rows ? R : rows;
+      for (int s = 0; s < rows; s += rb) {
+        const int t = pos0 + s;
+        tma_load_4d(d + s * C::ROWB, m_col, bar, x, t / R, t % R, bh);
+      }
+    } else {
+      if (c >= rows) {
+        tma_load_4d(d, m_sum, bar, x, l - c + (pos0 % c), pos0 / c, bh);
+      } else {
+        tma_load_4d(d, m_sum, bar, x, l - c, pos0 / c, bh);
+      }
+    }
+  }
+}
+
+// K-major operand descriptor for k-step kk (16 elements of K) of a tile with
+// PANELS panels of `rows` rows.
+template <int D>
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int rows, int kk) {
+  using C = FwdCfg<D>;
+  constexpr int steps_per_panel = C::ROWB / 32;
+  const int panel = kk / steps_per_panel;
+  const int within = (kk % steps_per_panel) * 32;
+  return make_desc(base + panel * rows * C::ROWB + within, 16, C::SBO, C::SWZ);
+}
+
+// MN-major operand descriptor (N = D contiguous in panels of rows x ROWB),
+// for k-step kk = 16 rows of K.
+template <int D>
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int rows, int kk) {
+  using C = FwdCfg<D>;
+  return make_desc(base + kk * 16 * C::ROWB, rows * C::ROWB, C::SBO, C::SWZ);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    sa_fwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
+                  const __grid_constant__ CUtensorMap mk_nat, const __grid_constant__ CUtensorMap mk_col,
+                  const __grid_constant__ CUtensorMap mk_sum, const __grid_constant__ CUtensorMap mv_nat,
+                  const __grid_constant__ CUtensorMap mv_col, const __grid_constant__ CUtensorMap mv_sum,
+                  const FwdArgs a) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sP = smem + C::OFF_P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_k_full = bars + 1;
+  uint64_t* bar_v_full = bar_k_full + C::STAGES;
+  uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
+  uint64_t* bar_s_full = bar_kv_empty + C::STAGES;  // [2]
+  uint64_t* bar_s_empty = bar_s_full + 2;           // [2]
+  uint64_t* bar_p_full = bar_s_empty + 2;           // [2]
+  uint64_t* bar_pv_done = bar_p_full + 2;           // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+
+  const int bh = blockIdx.x;
+  const int qt = a.order[blockIdx.y];
+  const int e0 = a.row_ptr[qt];
+  const int n = a.row_ptr[qt + 1] - e0;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar_k_full + s, 1);
+      mbar_init(bar_v_full + s, 1);
+      mbar_init(bar_kv_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_s_full + s, 1);
+      mbar_init(bar_s_empty + s, 128);
+      mbar_init(bar_p_full + s, 128);
+      mbar_init(bar_pv_done + s, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc<C::TMEM_COLS>(tmem_slot);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && n > 0) {
+      // ------------------------------------------------------------ producer
+      const CUtensorMap* mq = a.q_col ? &mq_col : &mq_nat;
+      mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+      load_rows<D>(sQ, a.q_col ? SRC_T : SRC_N, qt * C::TQ, C::TQ, bh, mq, mq, mq, bar_q, a.R,
+                   a.l, a.c);
+      for (int j = 0; j < n; ++j) {
+        const int st = j % C::STAGES;
+        if (j >= C::STAGES && !mbar_wait(bar_kv_empty + st, ((j / C::STAGES) - 1) & 1, abort_flag))
+          break;
+        const int e = a.ent[e0 + j];
+        const int src = (e >> 1) & 3;
+        const int kpos = (e >> 3) * C::TK;
+        mbar_arrive_expect_tx(bar_k_full + st, C::KV_BYTES);
+        load_rows<D>(sK + st * C::KV_BYTES, src, kpos, C::TK, bh, &mk_nat, &mk_col, &mk_sum,
+                     bar_k_full + st, a.R, a.l, a.c);
+        mbar_arrive_expect_tx(bar_v_full + st, C::KV_BYTES);
+        load_rows<D>(sV + st * C::KV_BYTES, src, kpos, C::TK, bh, &mv_nat, &mv_col, &mv_sum,
+                     bar_v_full + st, a.R, a.l, a.c);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && n > 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc_qk = make_idesc_bf16(128, C::TK, false, false);
+      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, false, true);
+      const uint32_t q_base = smem_u32(sQ);
+      bool ok = mbar_wait(bar_q, 0, abort_flag);
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % C::STAGES;
+          const int sb = j & 1;
+          ok = mbar_wait(bar_k_full + st, (j / C::STAGES) & 1, abort_flag);
+          if (ok && j >= 2) ok = mbar_wait(bar_s_empty + sb, ((j >> 1) - 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(sK + st * C::KV_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + sb * C::TK, kmajor_desc<D>(q_base, C::TQ, kk),
+                        kmajor_desc<D>(k_base, C::TK, kk), idesc_qk, kk > 0);
+          mma_commit(bar_s_full + sb);
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int st = jj % C::STAGES;
+          const int pb = jj & 1;
+          ok = mbar_wait(bar_p_full + pb, (jj >> 1) & 1, abort_flag) &&
+               mbar_wait(bar_v_full + st, (jj / C::STAGES) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t p_base = smem_u32(sP + pb * C::P_BYTES);
+          const uint32_t v_base = smem_u32(sV + st * C::KV_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < C::TK / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_O, make_desc(p_base + kk * 32, 16, 1024, kSwizzle128),
+                        mnmajor_desc<D>(v_base, C::TK, kk), idesc_pv, (jj > 0 || kk > 0));
+          mma_commit(bar_pv_done + pb);
+          mma_commit(bar_kv_empty + st);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const int x = qt * C::TQ + row;  // view position of this query
+    const bool valid = x < a.N;
+    const int nat = a.q_col ? (x % a.R) * a.l + x / a.R : x;
+    // key intervals by source view (inclusive)
+    int lo_n, hi_n;
+    if (a.pattern == SA_ALL) {
+      lo_n = 0;
+    } else if (a.pattern == SA_FIXED) {
+      lo_n = (nat / a.l) * a.l;
+    } else {
+      lo_n = max(0, nat - a.l + 1);
+    }
+    hi_n = nat;
+    const int lo_t = (x / a.R) * a.R, hi_t = x - 1;
+    const int lo_s = 0, hi_s = (nat / a.l) * a.c - 1;
+
+    float m_used = -INFINITY;
+    float l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int sb = j & 1;
+      ok = ok && mbar_wait(bar_s_full + sb, (j >> 1) & 1, abort_flag);
+      tc_fence_after();
+      float s[C::TK];
+#pragma unroll
+      for (int i = 0; i < C::TK / 16; ++i) tmem_ld16(tmem + lane_base + sb * C::TK + i * 16, s + i * 16);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_s_empty + sb);
+
+      const int e = a.ent[e0 + j];
+      if (e & 1) {
+        const int src = (e >> 1) & 3;
+        const int k0 = (e >> 3) * C::TK;
+        const int lo = src == SRC_N ? lo_n : (src == SRC_T ? lo_t : lo_s);
+        const int hi = src == SRC_N ? hi_n : (src == SRC_T ? hi_t : hi_s);
+#pragma unroll
+        for (int i = 0; i < C::TK; ++i) {
+          const int key = k0 + i;
+          if (key < lo || key > hi) s[i] = -INFINITY;
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < C::TK; ++i) mx = fmaxf(mx, s[i]);
+      const float m_tile = mx * a.scale_log2;
+      float factor = 1.f;
+      if (m_tile > m_used + 8.f) {
+        factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_tile);
+        m_used = m_tile;
+      }
+      // Rescale the O accumulator (only after the first tile, only if needed).
+      if (j > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
+        const int jp = j - 1;
+        ok = ok && mbar_wait(bar_pv_done + (jp & 1), (jp >> 1) & 1, abort_flag);
+        tc_fence_after();
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+          float ov[16];
+          tmem_ld16(tmem + lane_base + C::COL_O + i * 16, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 16; ++u) ov[u] *= factor;
+          tmem_st16(tmem + lane_base + C::COL_O + i * 16, ov);
+        }
+        tmem_wait_st();
+      }
+      // P buffer j&1 is free once PV of tile j-2 has completed.
+      if (j >= 2) ok = ok && mbar_wait(bar_pv_done + sb, ((j >> 1) - 1) & 1, abort_flag);
+      const float neg = (m_used == -INFINITY) ? 0.f : -m_used;
+      float rsum = 0.f;
+      uint8_t* pbuf = sP + sb * C::P_BYTES;
+#pragma unroll
+      for (int ch = 0; ch < C::TK / 8; ++ch) {
+        float p[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          p[u] = ex2(fmaf(s[ch * 8 + u], a.scale_log2, neg));
+          rsum += p[u];
+        }
+        uint4 w;
+        w.x = pack_bf16(p[0], p[1]);
+        w.y = pack_bf16(p[2], p[3]);
+        w.z = pack_bf16(p[4], p[5]);
+        w.w = pack_bf16(p[6], p[7]);
+        *reinterpret_cast<uint4*>(pbuf + sw128_offset(row, ch)) = w;
+      }
+      l_sum = l_sum * factor + rsum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_p_full + sb);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    float inv = 0.f, lse_row = -INFINITY;
+    if (l_sum > 0.f) {
+      inv = 1.f / l_sum;
+      lse_row = (m_used + lg2(l_sum)) * 0.6931471805599453f;
+    }
+    if (n > 0) {
+      const int jl = n - 1;
+      ok = ok && mbar_wait(bar_pv_done + (jl & 1), (jl >> 1) & 1, abort_flag);
+      tc_fence_after();
+    }
+    float w_new = 1.f, w_old = 0.f, lse_out = lse_row;
+    const size_t row_off = (static_cast<size_t>(bh) * a.N + (valid ? nat : 0)) * D;
+    if (a.merge && valid) {
+      const float lse_old = a.lse[static_cast<size_t>(bh) * a.N + nat];
+      const float mm = fmaxf(lse_row, lse_old);
+      if (mm == -INFINITY) {
+        w_new = 0.f;
+        w_old = 0.f;
+      } else {
+        const float en = ex2((lse_row - mm) * 1.4426950408889634f);
+        const float eo = ex2((lse_old - mm) * 1.4426950408889634f);
+        const float tot = en + eo;
+        w_new = en / tot;
+        w_old = eo / tot;
+        lse_out = mm + lg2(tot) * 0.6931471805599453f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+      float ov[16];
+      if (n > 0) {
+        tmem_ld16(tmem + lane_base + C::COL_O + i * 16, ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) ov[u] = 0.f;
+      }
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(a.o + row_off + i * 16);
+        float old[16];
+        if (a.merge) {
+          const uint4 o0 = dst[0], o1 = dst[1];
+          const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&o0);
+          const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&o1);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 f0 = __bfloat1622float2(h0[u]);
+            const float2 f1 = __bfloat1622float2(h1[u]);
+            old[2 * u] = f0.x;
+            old[2 * u + 1] = f0.y;
+            old[8 + 2 * u] = f1.x;
+            old[8 + 2 * u + 1] = f1.y;
+          }
+        }
+        float r[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) r[u] = a.merge ? (w_new * ov[u] * inv + w_old * old[u]) : ov[u] * inv;
+        uint4 w0, w1;
+        w0.x = pack_bf16(r[0], r[1]);
+        w0.y = pack_bf16(r[2], r[3]);
+        w0.z = pack_bf16(r[4], r[5]);
+        w0.w = pack_bf16(r[6], r[7]);
+        w1.x = pack_bf16(r[8], r[9]);
+        w1.y = pack_bf16(r[10], r[11]);
+        w1.z = pack_bf16(r[12], r[13]);
+        w1.w = pack_bf16(r[14], r[15]);
+        dst[0] = w0;
+        dst[1] = w1;
+      }
+    }
+    if (valid) a.lse[static_cast<size_t>(bh) * a.N + nat] = lse_out;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<C::TMEM_COLS>(tmem);
+  }
+}
+
+}  // namespace sa

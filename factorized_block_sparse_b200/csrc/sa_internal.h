@@ -1,0 +1,77 @@
+// Internal declarations shared by the layout builder, the C ABI and the
+// kernels.  Not part of the public interface (include/sparse_attn.h is).
+#pragma once
+
+#include <cstdint>
+#include <mutex>
+#include <vector>
+
+#include "sparse_attn.h"
+
+namespace sa {
+
+// Kernel tile sizes.  The public block tables are at the caller's `block`
+// granularity; the kernels run on coarser tiles whose tables are derived
+// from them (a tile is present when any block overlapping it is, FULL when
+// every overlapping block is FULL and the tile lies inside the view).
+constexpr int kFwdTQ = 128;  // forward: query rows per CTA (tcgen05 M)
+constexpr int kFwdTK = 64;   // forward: keys per step (tcgen05 N of Q K^T)
+constexpr int kBwdTK = 128;  // backward: keys per CTA (tcgen05 M of K Q^T)
+constexpr int kBwdTQ = 128;  // backward: queries per step
+
+enum Src : int { SRC_N = 0, SRC_T = 1, SRC_S = 2 };
+
+// Entry of a kernel tile table: (tile << 3) | (src << 1) | partial.
+inline int32_t pack_entry(int tile, int src, int partial) {
+  return (tile << 3) | (src << 1) | (partial & 1);
+}
+
+struct Csr {
+  std::vector<int32_t> row_ptr, col_idx;
+  std::vector<uint8_t> kind;
+  int n_rows = 0, n_cols = 0;
+};
+
+struct TileTable {
+  std::vector<int32_t> row_ptr;  // n_rows + 1
+  std::vector<int32_t> ent;      // packed entries, ascending tile per source
+  std::vector<int32_t> order;    // rows by descending entry count (launch order)
+  int n_rows = 0;
+};
+
+struct DevTable {
+  const int32_t* row_ptr = nullptr;
+  const int32_t* ent = nullptr;
+  const int32_t* order = nullptr;
+  int n_rows = 0;
+  int nnz = 0;
+};
+
+struct DeviceCopy {
+  int device = -1;
+  void* blob = nullptr;
+  DevTable fwd_main, fwd_col, bwd_main, bwd_sec;
+};
+
+}  // namespace sa
+
+struct sa_layout {
+  int pattern = 0, N = 0, l = 1, c = 0, block = 1, R = 1;
+  bool has[3] = {false, false, false};
+  sa::Csr view[3];   // public tables, query-block major
+  sa::Csr viewT[3];  // public tables, key-block major
+  // Kernel tables.
+  sa::TileTable fwd_main;  // natural query tiles: N-view keys (+ S-view keys for fixed)
+  sa::TileTable fwd_col;   // column-order query tiles: T-view keys (strided)
+  sa::TileTable bwd_main;  // natural key tiles: N-view query tiles
+  sa::TileTable bwd_sec;   // T-order (strided) or summary-order (fixed) key tiles
+  mutable std::mutex mu;
+  mutable std::vector<sa::DeviceCopy> dev;
+};
+
+namespace sa {
+// Builds every table of a layout (host only).  Returns an sa_status.
+int build_layout(sa_layout* L);
+// Number of key positions of a view (summary view: R * c).
+int view_keys(const sa_layout* L, int view);
+}  // namespace sa

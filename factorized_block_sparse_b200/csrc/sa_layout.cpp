@@ -1,0 +1,247 @@
+// Layout builder: block look-up tables of the factorized patterns.
+//
+// The block-sparse kernels of the Sparse Transformer slice queries and keys
+// into blocks and visit only the blocks that hold part of the mask ("OpenAI
+// Sparse Transformer", "Implementation and Limitations"; pcnews translation,
+// "Релиз кода").  A factorized pattern is block-dense only after the column
+// step is relabelled: attention along a column of the 2-D array is attention
+// along a row of the transposed array (pcnews translation, "Разреженное
+// внимание").  So each pattern is split into views that are dense in their
+// own order (natural; column-major for the strided column part; consecutive
+// summary keys for the fixed pattern's summary part).
+//
+// In every view the keys a query position x may see form one interval
+// [lo(x), hi(x)] of view key positions (possibly empty), with lo and hi
+// non-decreasing in x.  The builder classifies each (query block, key block)
+// pair from these intervals, row by row; it never forms the element mask.
+#include <algorithm>
+#include <cstring>
+#include <numeric>
+
+#include "sa_internal.h"
+
+namespace sa {
+
+namespace {
+
+struct Interval {
+  long long lo, hi;  // inclusive; empty when lo > hi
+};
+
+// Key interval of view position x.
+Interval key_interval(const sa_layout* L, int view, long long x) {
+  const long long l = L->l, c = L->c, R = L->R;
+  if (view == SA_VIEW_NATURAL) {
+    switch (L->pattern) {
+      case SA_ALL:
+        return {0, x};
+      case SA_LOCAL:
+      case SA_STRIDED:
+        return {std::max(0LL, x - l + 1), x};
+      default:  // SA_FIXED: own l-block, causal
+        return {(x / l) * l, x};
+    }
+  }
+  if (view == SA_VIEW_COLUMN) {  // strict, inside the column run of length R
+    return {(x / R) * R, x - 1};
+  }
+  // SA_VIEW_SUMMARY: summary keys of strictly earlier blocks
+  return {0, (x / l) * c - 1};
+}
+
+Csr build_public(const sa_layout* L, int view) {
+  Csr t;
+  const int b = L->block;
+  const long long nq = L->N;
+  const long long nk = view_keys(L, view);
+  t.n_rows = static_cast<int>(nq / b);
+  t.n_cols = static_cast<int>((nk + b - 1) / b);
+  t.row_ptr.assign(1, 0);
+  std::vector<Interval> iv(b);
+  for (int r = 0; r < t.n_rows; ++r) {
+    long long lo_min = nk, hi_max = -1;
+    for (int u = 0; u < b; ++u) {
+      iv[u] = key_interval(L, view, static_cast<long long>(r) * b + u);
+      if (iv[u].lo <= iv[u].hi) {
+        lo_min = std::min(lo_min, iv[u].lo);
+        hi_max = std::max(hi_max, iv[u].hi);
+      }
+    }
+    if (hi_max >= 0) {
+      for (long long cb = lo_min / b; cb <= hi_max / b && cb < t.n_cols; ++cb) {
+        const long long y0 = cb * b, y1 = cb * b + b - 1;
+        bool any = false, all = (y1 < nk);
+        for (int u = 0; u < b; ++u) {
+          const long long lo = iv[u].lo, hi = iv[u].hi;
+          if (std::max(lo, y0) <= std::min(hi, y1)) any = true;
+          if (!(lo <= y0 && hi >= y1)) all = false;
+        }
+        if (any) {
+          t.col_idx.push_back(static_cast<int32_t>(cb));
+          t.kind.push_back(all ? SA_BLOCK_FULL : SA_BLOCK_PARTIAL);
+        }
+      }
+    }
+    t.row_ptr.push_back(static_cast<int32_t>(t.col_idx.size()));
+  }
+  return t;
+}
+
+Csr transpose(const Csr& a) {
+  Csr t;
+  t.n_rows = a.n_cols;
+  t.n_cols = a.n_rows;
+  std::vector<int32_t> cnt(a.n_cols + 1, 0);
+  for (int32_t cidx : a.col_idx) cnt[cidx + 1]++;
+  for (int i = 0; i < a.n_cols; ++i) cnt[i + 1] += cnt[i];
+  t.row_ptr = cnt;
+  t.col_idx.resize(a.col_idx.size());
+  t.kind.resize(a.kind.size());
+  std::vector<int32_t> fill(cnt.begin(), cnt.end() - 1);
+  for (int r = 0; r < a.n_rows; ++r) {  // ascending r keeps each output row sorted
+    for (int e = a.row_ptr[r]; e < a.row_ptr[r + 1]; ++e) {
+      const int32_t dst = fill[a.col_idx[e]]++;
+      t.col_idx[dst] = r;
+      t.kind[dst] = a.kind[e];
+    }
+  }
+  return t;
+}
+
+// Coarsens a public table (rows = major blocks, cols = minor blocks, both of
+// `b` positions) to tiles of TM major x Tm minor positions.  n_major and
+// n_minor are the view's extents in positions.  Appends entries to `out`.
+struct CoarseRow {
+  std::vector<std::pair<int, int>> ent;  // (minor tile, partial)
+};
+
+std::vector<CoarseRow> coarsen(const Csr& a, int b, int TM, int Tm, long long n_major,
+                               long long n_minor) {
+  const int n_tiles = static_cast<int>((n_major + TM - 1) / TM);
+  std::vector<CoarseRow> rows(n_tiles);
+  std::vector<int> full_cnt, touched;
+  const int n_minor_tiles = static_cast<int>((n_minor + Tm - 1) / Tm);
+  full_cnt.assign(n_minor_tiles, 0);
+  std::vector<char> present(n_minor_tiles, 0);
+  for (int r = 0; r < n_tiles; ++r) {
+    const long long p0 = static_cast<long long>(r) * TM;
+    const long long p1 = std::min(p0 + TM, n_major) - 1;
+    const int rb0 = static_cast<int>(p0 / b), rb1 = static_cast<int>(p1 / b);
+    const int n_rb = rb1 - rb0 + 1;
+    touched.clear();
+    for (int rb = rb0; rb <= rb1 && rb < a.n_rows; ++rb) {
+      for (int e = a.row_ptr[rb]; e < a.row_ptr[rb + 1]; ++e) {
+        const long long y0 = static_cast<long long>(a.col_idx[e]) * b;
+        const long long y1 = std::min(y0 + b, n_minor) - 1;
+        for (long long t = y0 / Tm; t <= y1 / Tm; ++t) {
+          if (!present[t]) {
+            present[t] = 1;
+            touched.push_back(static_cast<int>(t));
+          }
+          if (a.kind[e] == SA_BLOCK_FULL) full_cnt[t]++;
+        }
+      }
+    }
+    std::sort(touched.begin(), touched.end());
+    const bool major_whole = (p0 + TM <= n_major) && (p1 == p0 + TM - 1);
+    for (int t : touched) {
+      const long long q0 = static_cast<long long>(t) * Tm;
+      const long long q1 = q0 + Tm - 1;
+      const int cb0 = static_cast<int>(q0 / b);
+      const int cb1 = static_cast<int>(std::min(q1, n_minor - 1) / b);
+      const int need = n_rb * (cb1 - cb0 + 1);
+      const bool full = major_whole && (q1 < n_minor) && full_cnt[t] == need;
+      rows[r].ent.push_back({t, full ? 0 : 1});
+      present[t] = 0;
+      full_cnt[t] = 0;
+    }
+  }
+  return rows;
+}
+
+void finish_table(TileTable& tt, const std::vector<std::vector<int32_t>>& rows) {
+  tt.n_rows = static_cast<int>(rows.size());
+  tt.row_ptr.assign(1, 0);
+  tt.ent.clear();
+  for (const auto& r : rows) {
+    tt.ent.insert(tt.ent.end(), r.begin(), r.end());
+    tt.row_ptr.push_back(static_cast<int32_t>(tt.ent.size()));
+  }
+  tt.order.resize(tt.n_rows);
+  std::iota(tt.order.begin(), tt.order.end(), 0);
+  // Longest rows first; among equals, later rows first.
+  std::stable_sort(tt.order.begin(), tt.order.end(), [&](int x, int y) {
+    const int lx = tt.row_ptr[x + 1] - tt.row_ptr[x], ly = tt.row_ptr[y + 1] - tt.row_ptr[y];
+    if (lx != ly) return lx > ly;
+    return x > y;
+  });
+}
+
+}  // namespace
+
+int view_keys(const sa_layout* L, int view) {
+  if (view == SA_VIEW_SUMMARY) return L->R * L->c;
+  return L->N;
+}
+
+int build_layout(sa_layout* L) {
+  const int p = L->pattern;
+  L->has[SA_VIEW_NATURAL] = true;
+  L->has[SA_VIEW_COLUMN] = (p == SA_STRIDED);
+  L->has[SA_VIEW_SUMMARY] = (p == SA_FIXED);
+  for (int v = 0; v < 3; ++v) {
+    if (!L->has[v]) continue;
+    L->view[v] = build_public(L, v);
+    L->viewT[v] = transpose(L->view[v]);
+  }
+  const long long N = L->N;
+  const int b = L->block;
+
+  // Forward, natural query tiles: summary entries first (fixed), then natural.
+  {
+    auto nat = coarsen(L->view[SA_VIEW_NATURAL], b, kFwdTQ, kFwdTK, N, N);
+    std::vector<CoarseRow> sum;
+    if (L->has[SA_VIEW_SUMMARY])
+      sum = coarsen(L->view[SA_VIEW_SUMMARY], b, kFwdTQ, kFwdTK, N, view_keys(L, SA_VIEW_SUMMARY));
+    std::vector<std::vector<int32_t>> rows(nat.size());
+    for (size_t r = 0; r < nat.size(); ++r) {
+      if (!sum.empty())
+        for (auto& e : sum[r].ent) rows[r].push_back(pack_entry(e.first, SRC_S, e.second));
+      for (auto& e : nat[r].ent) rows[r].push_back(pack_entry(e.first, SRC_N, e.second));
+    }
+    finish_table(L->fwd_main, rows);
+  }
+  // Forward, column-order query tiles (strided).
+  if (L->has[SA_VIEW_COLUMN]) {
+    auto col = coarsen(L->view[SA_VIEW_COLUMN], b, kFwdTQ, kFwdTK, N, N);
+    std::vector<std::vector<int32_t>> rows(col.size());
+    for (size_t r = 0; r < col.size(); ++r)
+      for (auto& e : col[r].ent) rows[r].push_back(pack_entry(e.first, SRC_T, e.second));
+    finish_table(L->fwd_col, rows);
+  } else {
+    finish_table(L->fwd_col, {});
+  }
+  // Backward, natural key tiles -> natural query tiles.
+  {
+    auto kt = coarsen(L->viewT[SA_VIEW_NATURAL], b, kBwdTK, kBwdTQ, N, N);
+    std::vector<std::vector<int32_t>> rows(kt.size());
+    for (size_t r = 0; r < kt.size(); ++r)
+      for (auto& e : kt[r].ent) rows[r].push_back(pack_entry(e.first, SRC_N, e.second));
+    finish_table(L->bwd_main, rows);
+  }
+  // Backward, secondary view key tiles (T order or summary order).
+  if (L->has[SA_VIEW_COLUMN] || L->has[SA_VIEW_SUMMARY]) {
+    const int v = L->has[SA_VIEW_COLUMN] ? SA_VIEW_COLUMN : SA_VIEW_SUMMARY;
+    const int src = (v == SA_VIEW_COLUMN) ? SRC_T : SRC_S;
+    auto kt = coarsen(L->viewT[v], b, kBwdTK, kBwdTQ, view_keys(L, v), N);
+    std::vector<std::vector<int32_t>> rows(kt.size());
+    for (size_t r = 0; r < kt.size(); ++r)
+      for (auto& e : kt[r].ent) rows[r].push_back(pack_entry(e.first, src, e.second));
+    finish_table(L->bwd_sec, rows);
+  } else {
+    finish_table(L->bwd_sec, {});
+  }
+  return SA_OK;
+}
+
+}  // namespace sa

@@ -1,0 +1,233 @@
+"""Thin Python binding of the C ABI in ``include/sparse_attn.h``.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libsparse_attn.so``.  Tensors are ``torch.Tensor`` objects on a
+CUDA device (bf16 ``[B, H, N, D]`` contiguous; lse fp32 ``[B, H, N]``); the
+stream is torch's current stream unless one is given.  There is no CPU
+fallback: if the library is missing, loading this module raises.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
+
+PATTERNS = {"all": 0, "local": 1, "strided": 2, "fixed": 3}
+VIEWS = {"N": 0, "T": 1, "S": 2}
+VIEW_TRANSPOSED = 4
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_LUT, SA_ERR_TIMEOUT, SA_ERR_WORKSPACE = range(7)
+
+# Every entry point declared in include/sparse_attn.h.
+EXPORTS = (
+    "sparse_attn_layout", "sparse_attn_layout_export", "sparse_attn_layout_info",
+    "sparse_attn_layout_upload", "sparse_attn_layout_free", "sparse_attn_fwd",
+    "sparse_attn_bwd_workspace_size", "sparse_attn_bwd", "sparse_attn_status",
+    "sparse_attn_strerror", "sparse_attn_kernel_kinds", "sparse_attn_timing_enable",
+    "sparse_attn_timing_reset", "sparse_attn_timing_read", "sparse_attn_launch_count",
+)
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {strerror(status)} (status {status})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m factorized_block_sparse_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, VP = ctypes.POINTER, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+    lib.sparse_attn_layout.argtypes = [I, I, I, I, I, P(VP)]
+    lib.sparse_attn_layout.restype = I
+    lib.sparse_attn_layout_export.argtypes = [VP, I, VP, VP, VP, P(I), P(I)]
+    lib.sparse_attn_layout_export.restype = I
+    lib.sparse_attn_layout_info.argtypes = [VP, P(I), P(I), P(I), P(I), P(I)]
+    lib.sparse_attn_layout_info.restype = I
+    lib.sparse_attn_layout_upload.argtypes = [VP, VP]
+    lib.sparse_attn_layout_upload.restype = I
+    lib.sparse_attn_layout_free.argtypes = [VP]
+    lib.sparse_attn_layout_free.restype = None
+    lib.sparse_attn_fwd.argtypes = [VP, VP, VP, VP, VP, I, I, I, I, VP, VP]
+    lib.sparse_attn_fwd.restype = I
+    lib.sparse_attn_bwd_workspace_size.argtypes = [I, I, I, I, VP]
+    lib.sparse_attn_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.sparse_attn_bwd.argtypes = [VP] * 9 + [I, I, I, I, VP, VP, ctypes.c_size_t, VP]
+    lib.sparse_attn_bwd.restype = I
+    lib.sparse_attn_status.argtypes = [VP]
+    lib.sparse_attn_status.restype = I
+    lib.sparse_attn_strerror.argtypes = [I]
+    lib.sparse_attn_strerror.restype = ctypes.c_char_p
+    lib.sparse_attn_kernel_kinds.argtypes = []
+    lib.sparse_attn_kernel_kinds.restype = I
+    lib.sparse_attn_timing_enable.argtypes = [I]
+    lib.sparse_attn_timing_enable.restype = I
+    lib.sparse_attn_timing_reset.argtypes = []
+    lib.sparse_attn_timing_reset.restype = I
+    lib.sparse_attn_timing_read.argtypes = [I, P(ctypes.c_char_p), P(ctypes.c_double), P(ctypes.c_longlong)]
+    lib.sparse_attn_timing_read.restype = I
+    lib.sparse_attn_launch_count.argtypes = []
+    lib.sparse_attn_launch_count.restype = ctypes.c_longlong
+    del F
+    return lib
+
+
+lib = _load()
+
+
+def strerror(status):
+    return lib.sparse_attn_strerror(int(status)).decode()
+
+
+def _check(status, what):
+    if status != SA_OK:
+        raise SparseAttnError(status, what)
+
+
+class Layout:
+    """Owns an ``sa_layout*`` built by ``sparse_attn_layout``."""
+
+    def __init__(self, pattern, N, l=1, c=0, block=64):
+        self.pattern = pattern
+        self.N, self.l, self.c, self.block = int(N), int(l), int(c), int(block)
+        h = ctypes.c_void_p()
+        _check(lib.sparse_attn_layout(PATTERNS[pattern], self.N, self.l, self.c, self.block,
+                                      ctypes.byref(h)), "sparse_attn_layout")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def export(self, view, transposed=False):
+        """Host copy of one view's block table: dict(row_ptr, col_idx, kind, n_rows)."""
+        vid = VIEWS[view] | (VIEW_TRANSPOSED if transposed else 0)
+        n_rows, nnz = ctypes.c_int(), ctypes.c_int()
+        _check(lib.sparse_attn_layout_export(self._h, vid, None, None, None,
+                                             ctypes.byref(n_rows), ctypes.byref(nnz)), "export")
+        rp = np.zeros(n_rows.value + 1, np.int32)
+        ci = np.zeros(max(nnz.value, 1), np.int32)
+        kd = np.zeros(max(nnz.value, 1), np.uint8)
+        _check(lib.sparse_attn_layout_export(self._h, vid, rp.ctypes.data, ci.ctypes.data, kd.ctypes.data,
+                                             ctypes.byref(n_rows), ctypes.byref(nnz)), "export")
+        return dict(row_ptr=rp, col_idx=ci[:nnz.value], kind=kd[:nnz.value], n_rows=n_rows.value)
+
+    def upload(self, stream=None):
+        _check(lib.sparse_attn_layout_upload(self._h, _stream_ptr(stream)), "sparse_attn_layout_upload")
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib.sparse_attn_layout_free(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def sparse_attn_layout(pattern, N, l=1, c=0, block=64):
+    return Layout(pattern, N, l, c, block)
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        import torch
+
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, D]")
+    return tuple(int(x) for x in q.shape)
+
+
+def sparse_attn_fwd(q, k, v, o, lse, layout, stream=None):
+    """Writes ``o`` and ``lse`` in place (C ABI call)."""
+    B, H, N, D = _shape(q)
+    _check(lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, D,
+                               layout.handle, _stream_ptr(stream)), "sparse_attn_fwd")
+
+
+def sparse_attn_bwd_workspace_size(B, H, N, D, layout):
+    return int(lib.sparse_attn_bwd_workspace_size(B, H, N, D, layout.handle))
+
+
+def sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, layout, workspace, stream=None):
+    """Writes ``dq``, ``dk``, ``dv`` in place (C ABI call)."""
+    B, H, N, D = _shape(q)
+    _check(lib.sparse_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                               _ptr(dk), _ptr(dv), B, H, N, D, layout.handle, _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
+           "sparse_attn_bwd")
+
+
+def sparse_attn_status(stream=None):
+    return int(lib.sparse_attn_status(_stream_ptr(stream)))
+
+
+# ------------------------------------------------------------ conveniences
+def forward(q, k, v, layout, stream=None):
+    """Allocates ``o`` (bf16) and ``lse`` (fp32) with torch and runs the forward pass."""
+    import torch
+
+    B, H, N, D = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    sparse_attn_fwd(q, k, v, o, lse, layout, stream)
+    return o, lse
+
+
+def workspace(B, H, N, D, layout, device):
+    import torch
+
+    n = sparse_attn_bwd_workspace_size(B, H, N, D, layout)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def backward(q, k, v, o, lse, dO, layout, ws=None, stream=None):
+    """Allocates ``dq``, ``dk``, ``dv`` (and a workspace if none is given)."""
+    import torch
+
+    B, H, N, D = _shape(q)
+    if ws is None:
+        ws = workspace(B, H, N, D, layout, q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, layout, ws, stream)
+    return dq, dk, dv
+
+
+def kernel_times():
+    """{kernel name: (total ms, launches)} recorded while timing is enabled."""
+    out = {}
+    for i in range(lib.sparse_attn_kernel_kinds()):
+        name, ms, cnt = ctypes.c_char_p(), ctypes.c_double(), ctypes.c_longlong()
+        _check(lib.sparse_attn_timing_read(i, ctypes.byref(name), ctypes.byref(ms), ctypes.byref(cnt)),
+               "timing_read")
+        out[name.value.decode()] = (ms.value, cnt.value)
+    return out
+
+
+def timing_enable(on=True):
+    lib.sparse_attn_timing_enable(1 if on else 0)
+
+
+def timing_reset():
+    lib.sparse_attn_timing_reset()
+
+
+def launch_count():
+    return int(lib.sparse_attn_launch_count())

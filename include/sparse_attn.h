@@ -1,0 +1,201 @@
+/*
+ * sparse_attn.h - C ABI of the B200 (sm_100a) causal factorized sparse
+ * self-attention library (Sparse Transformer attention, forward and
+ * backward).
+ *
+ * What is computed.  For one (batch b, head h) slice with queries, keys and
+ * values q, k, v of shape [N, D]:
+ *     S_ij = <q_i, k_j> / sqrt(D)          for (i, j) in the pattern's mask
+ *     lse_i = log sum_j exp S_ij,  P = exp(S - lse),  O = P V
+ * and, in the backward pass, the gradients dQ, dK, dV of sum(O * dO).
+ * This is ordinary masked softmax attention ("Insights: 희소 어텐션
+ * (Sparse Attention)", the attention_impl / blocksparse_attention_impl
+ * paragraph), restricted to a sparse factorized mask ("OpenAI Sparse
+ * Transformer", sections "Sparse Attention and Algorithmic Complexity" and
+ * "Factorized Attention Patterns"; pcnews translation "Генеративное
+ * моделирование с разреженными трансформерами", section "Разреженное
+ * внимание").
+ *
+ * Masks (every mode is causal and includes j == i):
+ *   SA_ALL      j <= i                                    (dense causal)
+ *   SA_LOCAL    0 <= i - j < l                            (window of l)
+ *   SA_STRIDED  0 <= i - j < l  or  (i - j) mod l == 0    (row + column)
+ *   SA_FIXED    j <= i and ( j / l == i / l  or  j mod l >= l - c )
+ *               (own l-block + the last c "summary" offsets of each block)
+ *
+ * The backward pass recomputes P from the saved lse and never stores an
+ * N x N matrix, the memory-saving recomputation of "Generating Long
+ * Sequences with Sparse Transformers" (ABSTRACT, item b) and of the pcnews
+ * translation, section "Глубокое внимание".
+ *
+ * Tensor conventions (all calls):
+ *   q, k, v, o, dO, dq, dk, dv : bfloat16, [B, H, N, D] contiguous (row
+ *       major, D fastest), device pointers, 16-byte aligned, owned by the
+ *       caller.  bfloat16 values are passed as raw 16-bit patterns.
+ *   lse : float32 [B, H, N], natural logarithm, device pointer.
+ *   D   : 32, 64 or 128.  Scale is fixed at 1/sqrt(D).
+ *   stream : a cudaStream_t passed as void*; NULL means the legacy default
+ *       stream.  Every compute call only enqueues work on that stream and
+ *       returns; none synchronises except sparse_attn_status().
+ * Errors: every int-returning call returns SA_OK (0) or one of the
+ * sa_status codes below; sparse_attn_strerror() names them.  Argument
+ * errors are detected on the host before anything is enqueued.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sa_layout sa_layout; /* opaque, owned by the library */
+
+enum sa_pattern { SA_ALL = 0, SA_LOCAL = 1, SA_STRIDED = 2, SA_FIXED = 3 };
+
+/* Views of a pattern.  Each view is dense in its own relabelled order:
+ *   SA_VIEW_NATURAL : natural order, queries and keys (every pattern).
+ *   SA_VIEW_COLUMN  : strided only.  Positions relabelled column-major,
+ *       t(p) = (p mod l) * R + p / l with R = N / l; holds the strictly
+ *       earlier positions of the same column (attending along a column is
+ *       attending along a row of the transposed 2-D array: pcnews
+ *       translation, "Разреженное внимание").
+ *   SA_VIEW_SUMMARY : fixed only.  Queries natural; keys are the summary
+ *       positions j mod l >= l - c numbered consecutively,
+ *       sigma(j) = (j / l) * c + (j mod l - (l - c)); holds the summary keys
+ *       of strictly earlier blocks.
+ * OR SA_VIEW_TRANSPOSED into a view id to export the key-block-major table
+ * of that view (used by the backward pass). */
+enum sa_view {
+  SA_VIEW_NATURAL = 0,
+  SA_VIEW_COLUMN = 1,
+  SA_VIEW_SUMMARY = 2,
+  SA_VIEW_TRANSPOSED = 4
+};
+
+enum sa_status {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad enum   */
+  SA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (D, divisibility) */
+  SA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed           */
+  SA_ERR_LUT = 4,          /* layout does not match the call's shape      */
+  SA_ERR_TIMEOUT = 5,      /* a device-side wait gave up (status word)    */
+  SA_ERR_WORKSPACE = 6     /* workspace missing or too small              */
+};
+
+/* Block look-up table kinds. */
+enum sa_block_kind { SA_BLOCK_FULL = 0, SA_BLOCK_PARTIAL = 1 };
+
+/*
+ * sparse_attn_layout - build the block layout of a pattern.
+ *
+ * The block-sparse kernels of the pages slice queries and keys into blocks
+ * ("OpenAI Sparse Transformer", "Implementation and Limitations"; pcnews
+ * translation, "Релиз кода"; the SparseAttention class of the "Insights"
+ * page reshapes its inputs to the block size).  For every view of the
+ * pattern this builds, on the host, a CSR table over query blocks of
+ * `block` positions listing the key blocks that hold part of the mask, in
+ * ascending order, each marked FULL (every element in the mask) or PARTIAL,
+ * plus its key-block-major transpose, and the coarser tile tables the
+ * kernels run on.  Device copies are made on the first compute call on each
+ * device (or by sparse_attn_layout_upload).
+ *
+ * Arguments: pattern (sa_pattern); N >= 1 sequence length; l >= 1 row
+ * length / window (ignored for SA_ALL); c summary columns, 1 <= c <= l
+ * (SA_FIXED only, ignored otherwise); block >= 1 with N % block == 0.
+ * SA_STRIDED and SA_FIXED need N % l == 0.  *out receives a layout the
+ * caller releases with sparse_attn_layout_free.
+ * Errors: SA_ERR_INVALID_ARG (bad pattern, sizes, null out),
+ * SA_ERR_UNSUPPORTED (N % block or N % l not zero).
+ */
+int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** out);
+
+/*
+ * sparse_attn_layout_export - host copy of one view's block table.
+ * view: an sa_view id, optionally OR SA_VIEW_TRANSPOSED.  Any of row_ptr
+ * (n_rows + 1 entries), col_idx, kind (nnzb entries each) may be NULL; the
+ * sizes are always written to *n_rows and *nnzb (both required).
+ * A view the pattern does not have exports as zero rows.
+ * Errors: SA_ERR_INVALID_ARG.
+ */
+int sparse_attn_layout_export(const sa_layout* layout, int view, int32_t* row_ptr,
+                              int32_t* col_idx, uint8_t* kind, int* n_rows, int* nnzb);
+
+/* Pattern parameters stored in a layout (any output pointer may be NULL). */
+int sparse_attn_layout_info(const sa_layout* layout, int* pattern, int* N, int* l, int* c,
+                            int* block);
+
+/* Copy the layout's tables to the current device now, on `stream`
+ * (otherwise the first compute call does it).  Call before any stream
+ * capture.  Errors: SA_ERR_INVALID_ARG, SA_ERR_CUDA. */
+int sparse_attn_layout_upload(const sa_layout* layout, void* stream);
+
+/* Release a layout and its device copies (synchronises the device). */
+void sparse_attn_layout_free(sa_layout* layout);
+
+/*
+ * sparse_attn_fwd - forward pass.  Writes o [B,H,N,D] (bf16) and lse
+ * [B,H,N] (fp32, natural log).  For SA_STRIDED the column view runs first
+ * and its partial result is merged exactly (log-sum-exp) into the natural
+ * view's.  layout must have been built for this N.
+ * Errors: SA_ERR_INVALID_ARG (null pointer, B/H < 1), SA_ERR_LUT (layout N
+ * differs), SA_ERR_UNSUPPORTED (D not 32/64/128, column geometry the
+ * kernels do not tile: R = N/l must be a multiple of 8 and divide or be
+ * divisible by 128), SA_ERR_CUDA.
+ */
+int sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int N, int D, const sa_layout* layout, void* stream);
+
+/* Bytes of device workspace sparse_attn_bwd needs for this shape. */
+size_t sparse_attn_bwd_workspace_size(int B, int H, int N, int D, const sa_layout* layout);
+
+/*
+ * sparse_attn_bwd - backward pass with recomputation.  Inputs q, k, v, o,
+ * lse (as written by sparse_attn_fwd) and dO; outputs dq, dk, dv (bf16).
+ * workspace: caller-owned device memory of at least
+ * sparse_attn_bwd_workspace_size() bytes, 256-byte aligned; its contents on
+ * entry do not matter and on exit are unspecified.  dq accumulates in
+ * float32 with atomic adds, so its last bits may vary from run to run; dk
+ * and dv are deterministic.
+ * Errors: as sparse_attn_fwd, plus SA_ERR_WORKSPACE.
+ */
+int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                    const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int H,
+                    int N, int D, const sa_layout* layout, void* workspace, size_t ws_bytes,
+                    void* stream);
+
+/*
+ * sparse_attn_status - synchronise `stream`, then read and clear the
+ * current device's status word.  Kernels never trap: a device-side wait
+ * that gives up (about two seconds without progress) records
+ * SA_ERR_TIMEOUT there and the kernel drains and returns.  Returns SA_OK,
+ * SA_ERR_TIMEOUT or SA_ERR_CUDA (a pending CUDA error).
+ */
+int sparse_attn_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* sparse_attn_strerror(int status);
+
+/*
+ * Instrumentation for benchmarks (off by default; no effect on results).
+ * sparse_attn_timing_enable(1) brackets every kernel launch with CUDA
+ * events on its stream; sparse_attn_timing_read(i, ...) returns, for kernel
+ * kind i in [0, sparse_attn_kernel_kinds()), its name, the summed elapsed
+ * milliseconds of completed launches and their count (it synchronises the
+ * events).  sparse_attn_timing_reset() clears the sums.
+ * sparse_attn_launch_count() counts every kernel this library has launched
+ * since load (timing on or off).
+ */
+int sparse_attn_kernel_kinds(void);
+int sparse_attn_timing_enable(int on);
+int sparse_attn_timing_reset(void);
+int sparse_attn_timing_read(int kind, const char** name, double* total_ms, long long* launches);
+long long sparse_attn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */
