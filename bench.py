@@ -1,0 +1,503 @@
+#!/usr/bin/env python
+"""Benchmark: forward + backward of causal factorized sparse attention.
+
+One step = sparse_attn_fwd + sparse_attn_bwd (through the C ABI) on every
+workload of the step.  The default step holds both N = 12288 workloads, so
+it runs every kernel of the hot path (natural, column and summary views):
+  text-fixed      fixed pattern,   B=2 H=8  N=12288 D=64 l=128 c=32 block=64
+  image64-strided strided pattern, B=1 H=16 N=12288 D=64 l=192      block=64
+Metric: nonzero-block TFLOP/s, counted on the public block tables
+(4 b^2 D per nonzero block forward, 10 b^2 D backward, per batch and head),
+and tokens/s = B*N per workload / step time.  Inputs are seeded N(0,1)
+bf16 tensors (synthetic; no dataset).
+
+Timing: W untimed warm-up steps, then exactly K steps, each bracketed by
+CUDA events on the launching stream, with a 256 MiB write between steps to
+flush L2; barrier + synchronize around the timed loop; max over ranks.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from factorized_block_sparse_b200 import synth  # noqa: E402
+
+METRIC = "fwd+bwd nonzero-block TFLOP/s (% of B200 BF16 peak) and tokens/s at N=12288"
+STEPS = {
+    "n12288": ["text-fixed", "image64-strided"],
+}
+for _n in synth.WORKLOADS:
+    STEPS[_n] = [_n]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"], hbm=p["hbm_gbs"],
+                    source="measured")
+    return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ----------------------------------------------------------------- flop counts
+def block_counts(w, sa=None):
+    """Nonzero public blocks per view of a workload (from the library's table)."""
+    if sa is not None:
+        lay = sa.Layout(w["mode"], w["N"], w["l"], w["c"], w["block"])
+        views = {"strided": ("N", "T"), "fixed": ("N", "S")}.get(w["mode"], ("N",))
+        return {v: len(lay.export(v)["col_idx"]) for v in views}, lay
+    raise ValueError("library needed")
+
+
+def flops(w, counts):
+    per = w["block"] ** 2 * w["D"] * w["B"] * w["H"]
+    nnz = sum(counts.values())
+    return 4 * per * nnz, 10 * per * nnz
+
+
+def kernel_units(w, counts):
+    """Algorithmic work per launch of each kernel of a workload (flops or bytes)."""
+    per = w["block"] ** 2 * w["D"] * w["B"] * w["H"]
+    rows = w["B"] * w["H"] * w["N"]
+    D = w["D"]
+    m = w["mode"]
+    sec = counts.get("T", 0) + counts.get("S", 0)
+    fwd_main = counts["N"] + (counts.get("S", 0) if m == "fixed" else 0)
+    out = {
+        f"sa_fwd_natural_view.{m}": ("tensor", 4 * per * fwd_main),
+        f"sa_bwd_natural_view.{m}": ("tensor", 10 * per * counts["N"]),
+        f"sa_bwd_preprocess.{m}": ("hbm", rows * (2 * D * 2 + 4)),
+        f"sa_bwd_finalize_dq.{m}": ("hbm", rows * D * (4 + 2)),
+    }
+    if m == "strided":
+        out[f"sa_fwd_column_view.{m}"] = ("tensor", 4 * per * counts["T"])
+    if sec:
+        out[f"sa_bwd_secondary_view.{m}"] = ("tensor", 10 * per * sec)
+    return out
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons, power = [], None, set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(value, world, device):
+    """Max of a float over ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_nnz(w):
+    """Nonzero public blocks per (batch, head) of a workload, from the oracle's tables."""
+    from oracle import views as oviews
+
+    return sum(oviews.block_nonzeros(w["mode"], w["N"], w["l"], w["c"], w["block"]).values())
+
+
+def oracle_inputs(names):
+    out = []
+    for n in names:
+        w = synth.WORKLOADS[n]
+        # a [1, 1, N, D] draw equals slice (b=0, h=0) of the full workload's draw
+        out.append((w, synth.inputs(1, 1, w["N"], w["D"]), oracle_nnz(w)))
+    return out
+
+
+def oracle_sample_step(ws, step_idx, rows_per=512):
+    """Bounded oracle sample: query rows [r0, r0+rows_per) of slice (0, 0) of
+    each workload; forward rows (O, lse) and dQ rows with the float64 oracle
+    as it stands.  Returns (seconds, credited flops).  Credit: 10 b^2 D
+    (QK^T, PV, the recomputed QK^T, dO V^T, dS K) per nonzero public block,
+    times rows_per / N of the head's blocks (the chunk start rotates over the
+    sequence from step to step)."""
+    from oracle import attention
+
+    total_s, total_f = 0.0, 0.0
+    for w, x, nnz in ws:
+        N, b, D = w["N"], w["block"], w["D"]
+        n_chunks = N // rows_per
+        r0 = (step_idx % n_chunks) * rows_per
+        rows = list(range(r0, r0 + rows_per))
+        q, k, v, dO = (synth.to_f64(x[n]) for n in ("q", "k", "v", "dO"))
+        t0 = time.perf_counter()
+        attention.forward_rows(q, k, v, w["mode"], w["l"], w["c"], rows)
+        attention.dq_rows(q, k, v, dO, w["mode"], w["l"], w["c"], rows)
+        total_s += time.perf_counter() - t0
+        total_f += 10 * b * b * D * nnz * rows_per / N
+    return total_s, total_f
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        return int(n[0]) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(names, seconds_budget=15.0):
+    ws = oracle_inputs(names)
+    oracle_sample_step(ws, 0, 128)  # first touch
+    spent, fl, steps = 0.0, 0, 0
+    while spent < seconds_budget and steps < 48:
+        s, f = oracle_sample_step(ws, steps)
+        spent += s
+        fl += f
+        steps += 1
+    return {"value": fl / spent / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "seconds": round(spent, 2),
+            "sample": f"{steps} chunks of 512 query rows of slice (b=0,h=0) of each of {names}: float64 "
+                      "oracle forward rows + dQ rows; credited 10 b^2 D per nonzero block, pro rata of rows"}
+
+
+def run_reference(args, names):
+    world, rank, _ = dist_setup_cpu_only()
+    if rank != 0:
+        return 0
+    ws = oracle_inputs(names)
+    for i in range(args.warmup):
+        oracle_sample_step(ws, i, 256)
+    spent, fl = 0.0, 0
+    for i in range(args.steps):
+        s, f = oracle_sample_step(ws, i, 256)
+        spent += s
+        fl += f
+    value = fl / spent / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * spent / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(names, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"per step: 256 query rows of slice (b=0,h=0) of each of {names}; float64 "
+                                   "oracle forward rows + dQ rows; credited 10 b^2 D per nonzero block, pro rata of rows"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def dist_setup_cpu_only():
+    return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+
+
+def config_dict(names, args):
+    ws = [synth.WORKLOADS[n] for n in names]
+    return {
+        "workload": " + ".join(
+            f"{n}({w['mode']}, B={w['B']}, H={w['H']}, N={w['N']}, D={w['D']}, l={w['l']}"
+            + (f", c={w['c']}" if w["mode"] == "fixed" else "") + f", block={w['block']})"
+            for n, w in zip(names, ws)) + ", fwd+bwd",
+        "global_batch": sum(w["B"] for w in ws) * max(1, args.gpus),
+        "seq_len": ws[0]["N"],
+        "parallelism": f"replicas x{max(1, args.gpus)} (independent (batch, head) work per GPU, no collective)",
+        "l2": "flushed between timed steps (256 MiB write outside the events)",
+    }
+
+
+# ----------------------------------------------------------------- main arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="n12288", choices=sorted(STEPS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    names = STEPS[args.workload]
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args, names)
+
+    import torch
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from factorized_block_sparse_b200 import sparse_attn as sa
+
+    pk = peaks()
+    # inputs resident in HBM
+    state = []
+    fl_fwd = fl_bwd = 0
+    units = {}
+    for n in names:
+        w = synth.WORKLOADS[n]
+        counts, lay = block_counts(w, sa)
+        f0, f1 = flops(w, counts)
+        fl_fwd += f0
+        fl_bwd += f1
+        units.update(kernel_units(w, counts))
+        x = synth.inputs(w["B"], w["H"], w["N"], w["D"], seed_offset=rank)
+        q, k, v, dO = (x[t].to(dev) for t in ("q", "k", "v", "dO"))
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = sa.workspace(w["B"], w["H"], w["N"], w["D"], lay, dev)
+        lay.upload()
+        state.append(dict(w=w, lay=lay, x=x, q=q, k=k, v=v, dO=dO, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws))
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+
+    def step():
+        for s in state:
+            sa.sparse_attn_fwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["lay"], sptr)
+            sa.sparse_attn_bwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["dO"], s["dq"], s["dk"], s["dv"],
+                               s["lay"], s["ws"], sptr)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = sa.sparse_attn_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {sa.strerror(st)}")
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sa.timing_reset()
+    sa.timing_enable(True)
+    launches0 = sa.launch_count()
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    launches = sa.launch_count() - launches0
+    sa.timing_enable(False)
+    ktimes = sa.kernel_times()
+    st = sa.sparse_attn_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {sa.strerror(st)}")
+    local_ms = sum(a.elapsed_time(b) for a, b in evs)
+    total_ms = max_over_ranks(local_ms, world, dev)
+    ms_step = total_ms / args.steps
+    step_flops = fl_fwd + fl_bwd
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    tokens = world * sum(s["w"]["B"] * s["w"]["N"] for s in state)
+
+    # dominant kernel of the timed region
+    dom, dom_ms = None, -1.0
+    for name, (ms, cnt) in ktimes.items():
+        if cnt and ms > dom_ms:
+            dom, dom_ms = name, ms
+    cnt = ktimes[dom][1]
+    bound, per_launch = units.get(dom, ("tensor", None))
+    avg_ms = dom_ms / cnt
+    if bound == "tensor":
+        achieved = per_launch / (avg_ms * 1e-3) / 1e12
+        peak, unit = pk["bf16"], "TFLOP/s"
+    else:
+        achieved = per_launch / (avg_ms * 1e-3) / 1e9
+        peak, unit = pk["hbm"], "GB/s"
+    traffic = read_traffic(dom)
+    kernels = {n: {"ms_per_launch": round(ms / c, 4), "launches": c,
+                   **({"achieved": round(units[n][1] / (ms / c * 1e-3) / (1e12 if units[n][0] == "tensor" else 1e9), 2),
+                       "unit": "TFLOP/s" if units[n][0] == "tensor" else "GB/s"} if n in units else {})}
+               for n, (ms, c) in ktimes.items() if c}
+
+    # end to end through the C ABI with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = measure_e2e(sa, state, stream, args.e2e_steps, step_flops, world, dev)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded iid N(0,1), rounded to bf16)",
+        "config": config_dict(names, args),
+        "tokens_per_s": round(tokens / (ms_step * 1e-3), 1),
+        "pct_of_bf16_peak": round(100 * value / (world * pk["bf16"]), 2),
+        "pct_of_bf16_sustained": round(100 * value / (world * pk["bf16_sustained"]), 2),
+        "peak_source": pk["source"],
+        "flops_per_step": {"fwd": fl_fwd, "bwd": fl_bwd},
+        "roofline": {"kernel": dom, "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": "burst (of measured)" if pk["source"] == "measured" else "fallback"},
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(names, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_e2e(sa, state, stream, steps, step_flops, world, dev):
+    import torch
+
+    host = []
+    h2d = d2h = 0
+    for s in state:
+        hin = {t: s["x"][t].pin_memory() for t in ("q", "k", "v", "dO")}
+        hout = {t: torch.empty(s[t].shape, dtype=s[t].dtype, pin_memory=True) for t in ("o", "lse", "dq", "dk", "dv")}
+        h2d += sum(t.numel() * t.element_size() for t in hin.values())
+        d2h += sum(t.numel() * t.element_size() for t in hout.values())
+        host.append((hin, hout))
+    sptr = stream.cuda_stream
+
+    def one():
+        for s, (hin, hout) in zip(state, host):
+            for t in ("q", "k", "v", "dO"):
+                s[t].copy_(hin[t], non_blocking=True)
+            sa.sparse_attn_fwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["lay"], sptr)
+            sa.sparse_attn_bwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["dO"], s["dq"], s["dk"], s["dv"],
+                               s["lay"], s["ws"], sptr)
+            for t in ("o", "lse", "dq", "dk", "dv"):
+                hout[t].copy_(s[t], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    return {"value": round(world * step_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def read_traffic(kernel):
+    """Per-launch DRAM bytes of `kernel` from profiles/dram_traffic.txt, if the
+    recorded kernel source hash still matches the current sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = source_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel and parts[1] == cur:
+            return float(parts[2])
+    return None
+
+
+def source_hash():
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "factorized_block_sparse_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -24,10 +25,23 @@ namespace sa {
 namespace {
 
 // ------------------------------------------------------------ instrumentation
-enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_FINAL, K_NUM };
-const char* const kKindNames[K_NUM] = {"sa_fwd_column_view", "sa_fwd_natural_view",
-                                       "sa_bwd_preprocess",  "sa_bwd_secondary_view",
-                                       "sa_bwd_natural_view", "sa_bwd_finalize_dq"};
+enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_FINAL, K_KERNELS };
+const char* const kKernelNames[K_KERNELS] = {"sa_fwd_column_view", "sa_fwd_natural_view",
+                                             "sa_bwd_preprocess",  "sa_bwd_secondary_view",
+                                             "sa_bwd_natural_view", "sa_bwd_finalize_dq"};
+const char* const kPatternNames[4] = {"all", "local", "strided", "fixed"};
+// Instrumentation kinds: one per (kernel, pattern), kind = kernel * 4 + pattern.
+constexpr int K_NUM = K_KERNELS * 4;
+char g_kind_names[K_NUM][48];
+std::once_flag g_names_once;
+
+const char* kind_name(int kind) {
+  std::call_once(g_names_once, [] {
+    for (int k = 0; k < K_NUM; ++k)
+      std::snprintf(g_kind_names[k], sizeof(g_kind_names[k]), "%s.%s", kKernelNames[k / 4], kPatternNames[k % 4]);
+  });
+  return g_kind_names[kind];
+}
 
 struct Pending {
   int kind;
@@ -276,7 +290,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     a.q_col = 1;
     a.merge = 0;
     dim3 grid(g.BH, dc.fwd_col.n_rows);
-    st = launch(K_FWD_COL, s, [&] {
+    st = launch(K_FWD_COL * 4 + L->pattern, s, [&] {
       kern<<<grid, 192, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
     });
     if (st) return st;
@@ -287,7 +301,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.q_col = 0;
   a.merge = (two_pass && dc.fwd_col.n_rows > 0) ? 1 : 0;
   dim3 grid(g.BH, dc.fwd_main.n_rows);
-  return launch(K_FWD_MAIN, s, [&] {
+  return launch(K_FWD_MAIN * 4 + L->pattern, s, [&] {
     kern<<<grid, 192, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
   });
 }
@@ -339,7 +353,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   float* dv_part = reinterpret_cast<float*>(wsb + w.dv);
   const long long rows = static_cast<long long>(g.BH) * N;
 
-  st = launch(K_BWD_PRE, s, [&] {
+  st = launch(K_BWD_PRE * 4 + L->pattern, s, [&] {
     sa_bwd_pre_kernel<D><<<grid_for(rows * (D / 8), 256), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows);
   });
@@ -368,7 +382,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.key_view = (L->pattern == SA_STRIDED) ? SRC_T : SRC_S;
     a.add_part = 0;
     dim3 grid(g.BH, dc.bwd_sec.n_rows);
-    st = launch(K_BWD_SEC, s, [&] {
+    st = launch(K_BWD_SEC * 4 + L->pattern, s, [&] {
       kern<<<grid, 192, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                                                mv.col, mv.sum, a);
     });
@@ -381,14 +395,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.add_part = sec ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
   {
     dim3 grid(g.BH, dc.bwd_main.n_rows);
-    st = launch(K_BWD_MAIN, s, [&] {
+    st = launch(K_BWD_MAIN * 4 + L->pattern, s, [&] {
       kern<<<grid, 192, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                                                mv.col, mv.sum, a);
     });
     if (st) return st;
   }
   const long long n8 = rows * D / 8;
-  return launch(K_BWD_FINAL, s, [&] {
+  return launch(K_BWD_FINAL * 4 + L->pattern, s, [&] {
     sa_bwd_final_kernel<<<grid_for(n8, 256), 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
   });
 }
@@ -566,7 +580,7 @@ int sparse_attn_timing_read(int kind, const char** name, double* total_ms, long 
   if (kind < 0 || kind >= K_NUM) return SA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> g(g_timing.mu);
   drain_timing_locked();
-  if (name) *name = kKindNames[kind];
+  if (name) *name = kind_name(kind);
   if (total_ms) *total_ms = g_timing.total_ms[kind];
   if (launches) *launches = g_timing.count[kind];
   return SA_OK;

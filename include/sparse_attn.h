@@ -181,10 +181,10 @@ const char* sparse_attn_strerror(int status);
 /*
  * Instrumentation for benchmarks (off by default; no effect on results).
  * sparse_attn_timing_enable(1) brackets every kernel launch with CUDA
- * events on its stream; sparse_attn_timing_read(i, ...) returns, for kernel
- * kind i in [0, sparse_attn_kernel_kinds()), its name, the summed elapsed
- * milliseconds of completed launches and their count (it synchronises the
- * events).  sparse_attn_timing_reset() clears the sums.
+ * events on its stream; sparse_attn_timing_read(i, ...) returns, for kind i
+ * in [0, sparse_attn_kernel_kinds()), its name ("<kernel>.<pattern>", one
+ * kind per kernel and pattern), the summed elapsed milliseconds of
+ * completed launches and their count (it synchronises the events).  sparse_attn_timing_reset() clears the sums.
  * sparse_attn_launch_count() counts every kernel this library has launched
  * since load (timing on or off).
  */

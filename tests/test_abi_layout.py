@@ -78,7 +78,7 @@ def test_argument_errors(sa):
     assert sa.lib.sparse_attn_fwd(fake, fake, fake, fake, fake, 0, 1, 256, 32, lay.handle, None) \
         == sa.SA_ERR_INVALID_ARG
     assert sa.strerror(sa.SA_ERR_TIMEOUT) == "device-side wait timed out"
-    assert sa.lib.sparse_attn_kernel_kinds() == 6
+    assert sa.lib.sparse_attn_kernel_kinds() == 24
 
 
 def _compare(sa, mode, N, l, c, b, rows=None):
