@@ -589,3 +589,60 @@ int sparse_attn_timing_read(int kind, const char** name, double* total_ms, long 
 long long sparse_attn_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ==================================================================== no-alloc backward
+// Scratch for sparse_attn_bwd_noalloc: a file-scope device array, so callers
+// that cannot allocate device memory can still run the backward pass.  Host
+// code must not use the symbol itself as a device address; the address is
+// looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_sa_noalloc_scratch[SA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 128;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_sa_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return SA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SA_OK;
+}
+
+// True when the layout's tables are already on the current device.
+bool layout_on_device(const sa_layout* L) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> g(L->mu);
+  for (const auto& d : L->dev)
+    if (d.device == dev) return true;
+  return false;
+}
+}  // namespace
+
+extern "C" int sparse_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                       const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                                       int H, int N, int D, const sa_layout* L, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return SA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SA_ERR_INVALID_ARG;
+  int st = check_call(B, H, N, D, L);
+  if (st) return st;
+  const size_t need = sparse_attn_bwd_workspace_size(B, H, N, D, L);
+  if (need == 0 || need > SA_NOALLOC_SCRATCH_BYTES) return SA_ERR_WORKSPACE;
+  if (!layout_on_device(L)) return SA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch))) return st;
+  return sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, D, L, scratch, SA_NOALLOC_SCRATCH_BYTES,
+                         stream);
+}

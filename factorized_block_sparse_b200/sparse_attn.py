@@ -24,7 +24,7 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_LUT, SA_ERR_T
 EXPORTS = (
     "sparse_attn_layout", "sparse_attn_layout_export", "sparse_attn_layout_info",
     "sparse_attn_layout_upload", "sparse_attn_layout_free", "sparse_attn_fwd",
-    "sparse_attn_bwd_workspace_size", "sparse_attn_bwd", "sparse_attn_status",
+    "sparse_attn_bwd_workspace_size", "sparse_attn_bwd", "sparse_attn_bwd_noalloc", "sparse_attn_status",
     "sparse_attn_strerror", "sparse_attn_kernel_kinds", "sparse_attn_timing_enable",
     "sparse_attn_timing_reset", "sparse_attn_timing_read", "sparse_attn_launch_count",
 )
@@ -58,6 +58,8 @@ def _load():
     lib.sparse_attn_bwd_workspace_size.restype = ctypes.c_size_t
     lib.sparse_attn_bwd.argtypes = [VP] * 9 + [I, I, I, I, VP, VP, ctypes.c_size_t, VP]
     lib.sparse_attn_bwd.restype = I
+    lib.sparse_attn_bwd_noalloc.argtypes = [VP] * 9 + [I, I, I, I, VP, VP]
+    lib.sparse_attn_bwd_noalloc.restype = I
     lib.sparse_attn_status.argtypes = [VP]
     lib.sparse_attn_status.restype = I
     lib.sparse_attn_strerror.argtypes = [I]
@@ -173,6 +175,21 @@ def sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, layout, workspace, stream=N
                                _ptr(dk), _ptr(dv), B, H, N, D, layout.handle, _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
            "sparse_attn_bwd")
+
+
+def sparse_attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, layout, stream=None):
+    """Backward pass that allocates nothing: it runs in the library's built-in
+    scratch array (SA_NOALLOC_SCRATCH_BYTES per device) instead of a caller
+    workspace.  For callers that may not allocate device memory.  The layout
+    must already be on the device (``layout.upload()``); calls that overlap on
+    the GPU share the scratch array and race."""
+    B, H, N, D = _shape(q)
+    _check(lib.sparse_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                                       _ptr(dk), _ptr(dv), B, H, N, D, layout.handle, _stream_ptr(stream)),
+           "sparse_attn_bwd_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 def sparse_attn_status(stream=None):

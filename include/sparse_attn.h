@@ -167,6 +167,43 @@ int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                     void* stream);
 
 /*
+ * sparse_attn_bwd_noalloc - the backward pass for callers that cannot
+ * allocate device memory.  (Library-specific; the pages have no counterpart.)
+ *
+ * Some callers may not call cudaMalloc at all: for example a host framework
+ * that has handed every byte of device memory to its own pool and forbids
+ * outside allocations, or an application with a rule against device
+ * allocation after start-up.  They cannot supply the workspace that
+ * sparse_attn_bwd needs.  This entry point takes the same arguments minus the
+ * workspace and uses instead a scratch array compiled into the library: a
+ * file-scope __device__ array of SA_NOALLOC_SCRATCH_BYTES bytes, which every
+ * GPU that loads the library holds until the process exits.
+ *
+ * Limits and behaviour:
+ *  - shapes whose sparse_attn_bwd_workspace_size() exceeds
+ *    SA_NOALLOC_SCRATCH_BYTES are rejected with SA_ERR_WORKSPACE;
+ *  - it calls no cudaMalloc, cudaFree or other allocating routine, so the
+ *    layout's tables must already be on the current device (call
+ *    sparse_attn_layout_upload, or any other compute call with this layout,
+ *    on this device first); otherwise it returns SA_ERR_INVALID_ARG;
+ *  - the first call on a device looks up the device address of the scratch
+ *    array (cudaGetSymbolAddress) once for that device; make that first call
+ *    before any stream capture;
+ *  - every call on a device shares the one array, which keeps whatever the
+ *    last call left in it.  The kernels set everything they read from it
+ *    (the dQ accumulator is cleared by the preprocess kernel), so no clearing
+ *    is needed between calls, but calls whose GPU work overlaps (different
+ *    streams, or different host threads) race on the array and give wrong
+ *    results: order them on one stream or with events.
+ * Results equal those of sparse_attn_bwd (dq up to the run-to-run rounding of
+ * its atomic accumulation).  Errors: as sparse_attn_bwd.
+ */
+#define SA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int sparse_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            int B, int H, int N, int D, const sa_layout* layout, void* stream);
+
+/*
  * sparse_attn_status - synchronise `stream`, then read and clear the
  * current device's status word.  Kernels never trap: a device-side wait
  * that gives up (about two seconds without progress) records
