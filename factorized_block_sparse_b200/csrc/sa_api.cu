@@ -337,10 +337,10 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   const Geo g = make_geo(B, H, N, D, L);
   MapSet mq, mdo, mk, mv;
   int st;
-  if ((st = make_maps(&mq, q, g, L->pattern, 128))) return st;
-  if ((st = make_maps(&mdo, dO, g, L->pattern, 128))) return st;
-  if ((st = make_maps(&mk, k, g, L->pattern, 128))) return st;
-  if ((st = make_maps(&mv, v, g, L->pattern, 128))) return st;
+  if ((st = make_maps(&mq, q, g, L->pattern, BwdCfg<D>::TQ))) return st;
+  if ((st = make_maps(&mdo, dO, g, L->pattern, BwdCfg<D>::TQ))) return st;
+  if ((st = make_maps(&mk, k, g, L->pattern, BwdCfg<D>::TK))) return st;
+  if ((st = make_maps(&mv, v, g, L->pattern, BwdCfg<D>::TK))) return st;
   DeviceCopy dc;
   if ((st = to_device(L, &dc))) return st;
   auto kern = sa_bwd_kernel<D>;
@@ -383,7 +383,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.add_part = 0;
     dim3 grid(g.BH, dc.bwd_sec.n_rows);
     st = launch(K_BWD_SEC * 4 + L->pattern, s, [&] {
-      kern<<<grid, 192, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
+      kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                                                mv.col, mv.sum, a);
     });
     if (st) return st;
@@ -396,7 +396,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   {
     dim3 grid(g.BH, dc.bwd_main.n_rows);
     st = launch(K_BWD_MAIN * 4 + L->pattern, s, [&] {
-      kern<<<grid, 192, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
+      kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                                                mv.col, mv.sum, a);
     });
     if (st) return st;

@@ -8,16 +8,23 @@
 //   dK = s dS^T Q, dQ = s dS K.
 //
 // sa_bwd_kernel: one CTA = one 128-key tile of one (batch, head), in the
-// view order of its table; it walks the 128-query tiles that see it.
-//   ST  = K Q^T      (keys on TMEM lanes)          -> P^T   (bf16, smem)
-//   dPT = V dO^T                                    -> dS^T  (bf16, smem)
-//   dV += P^T dO,  dK += dS^T Q   (TMEM accumulators for the whole CTA)
-//   dQ  = dS K       (queries on TMEM lanes, reusing the ST columns), then
-//                    added to an fp32 workspace with vector reductions.
-// Roles: warp 0 lane 0 TMA producer; warp 1 TMEM allocation and lane 0 MMA
-// issue; warps 2..5 elementwise work, thread t of warp w owns TMEM lane
-// 32*(w%4)+t (a key row for ST/dPT/dV/dK, a query row for dQ).
-// TMEM columns: ST/dQ [0,128), dPT [128,256), dV [256,256+D), dK [256+D,256+2D).
+// view order of its table; it walks the 64-query steps that see it.  Per
+// step j:
+//   ST_j  = K Q_j^T, dPT_j = V dO_j^T  (keys on TMEM lanes, 64 columns each,
+//                                       double-buffered so step j+1's products
+//                                       overlap step j's elementwise work)
+//   P^T_j (bf16, smem), dS^T_j (bf16, smem) by the elementwise warps
+//   dV += P^T_j dO_j,  dK += dS^T_j Q_j   (TMEM accumulators for the CTA)
+//   every second step: dQ = dS_pair K for the two steps' 128 queries
+//                      (M = 128), read by the dQ warps and added to an fp32
+//                      workspace with vector reductions.
+// Roles (448 threads): warp 0 producer (TMA for K, V, Q, dO; plain loads of
+// lse and Delta), warp 1 TMEM allocation and lane 0 MMA issue, warps 2..9
+// elementwise (two warps per TMEM lane quarter, 32 query columns each),
+// warps 10..13 dQ reduction.  Warp w may only touch TMEM lanes
+// 32*(w%4)..32*(w%4)+31, so every role picks its rows by w%4.
+// TMEM columns (NBUF = 2 for D <= 64, 1 for D = 128):
+//   ST[b] = b*64, dPT[b] = NBUF*64 + b*64, dV = 2*NBUF*64, dK = dV + D, dQ = dK + D.
 #pragma once
 
 #include "sa_device.cuh"
@@ -46,55 +53,66 @@ struct BwdArgs {
 
 template <int D>
 struct BwdCfg {
-  static constexpr int TK = 128, TQ = 128;
-  static constexpr int STAGES = (D >= 128) ? 1 : 2;
+  static constexpr int TK = 128, TQ = 64;
+  static constexpr int NBUF = (D >= 128) ? 1 : 2;      // ST/dPT buffers in TMEM
+  // Q/dO ring.  At least 2: the MMA issuer asks for step j's Q/dO before it
+  // releases step j-1's (it issues S_j ahead of dV/dK of step j-1).
+  static constexpr int STAGES = (D >= 128) ? 2 : 3;
+  static constexpr int DST_BUFS = (D >= 128) ? 1 : 2;  // dS^T pair buffers
   static constexpr int ROWB = (D >= 64) ? 128 : 64;
-  static constexpr int PANELS = (D >= 64) ? D / 64 : 1;
   static constexpr uint64_t SWZ = (D >= 64) ? kSwizzle128 : kSwizzle64;
   static constexpr int SBO = 8 * ROWB;
-  static constexpr int T_BYTES = 128 * D * 2;   // one 128-row tile of D
-  static constexpr int PT_BYTES = 128 * 128 * 2;
+  static constexpr int KV_BYTES = TK * D * 2;          // 128-key tile
+  static constexpr int QS_BYTES = TQ * D * 2;          // 64-query tile
+  static constexpr int PT_BYTES = TK * TQ * 2;         // [128 keys][64 queries] bf16 = 16 KiB
+  static constexpr int DST_BYTES = 2 * PT_BYTES;       // a pair of steps (2 panels)
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + T_BYTES;
-  static constexpr int OFF_Q = OFF_V + T_BYTES;
-  static constexpr int OFF_DO = OFF_Q + STAGES * T_BYTES;
-  static constexpr int OFF_PT = OFF_DO + STAGES * T_BYTES;
-  static constexpr int OFF_DST = OFF_PT + PT_BYTES;
-  static constexpr int OFF_LSE = OFF_DST + PT_BYTES;        // float [2][128]
-  static constexpr int OFF_DELTA = OFF_LSE + 2 * 128 * 4;   // float [2][128]
-  static constexpr int OFF_BAR = OFF_DELTA + 2 * 128 * 4;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 8;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + STAGES * QS_BYTES;
+  static constexpr int OFF_PT = OFF_DO + STAGES * QS_BYTES;
+  static constexpr int OFF_DST = OFF_PT + 2 * PT_BYTES;
+  static constexpr int OFF_LSE = OFF_DST + DST_BUFS * DST_BYTES;  // float [STAGES][64]
+  static constexpr int OFF_DELTA = OFF_LSE + STAGES * TQ * 4;      // float [STAGES][64]
+  static constexpr int OFF_BAR = OFF_DELTA + STAGES * TQ * 4;
+  static constexpr int N_BARS = 1 + 2 * STAGES + 2 * NBUF + 2 * 2 + 2 + 2 * DST_BUFS + 3;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int COL_ST = 0, COL_DPT = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr int COL_DPT = NBUF * 64;
+  static constexpr int COL_DV = 2 * NBUF * 64;
+  static constexpr int COL_DK = COL_DV + D;
+  static constexpr int COL_DQ = COL_DK + D;
+  static constexpr int THREADS = 448;
+  static_assert(COL_DQ + D <= TMEM_COLS, "TMEM budget");
+  static_assert(STAGES >= 2, "the software-pipelined MMA loop needs two Q/dO stages");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
+// K-major operand (rows x D) for k-step kk (16 elements of D).
 template <int D>
-__device__ __forceinline__ uint64_t bwd_kdesc(uint32_t base, int kk) {  // K-major, 128 rows, K = D
+__device__ __forceinline__ uint64_t bwd_kdesc(uint32_t base, int rows, int kk) {
   using C = BwdCfg<D>;
   constexpr int spp = C::ROWB / 32;
-  return make_desc(base + (kk / spp) * 128 * C::ROWB + (kk % spp) * 32, 16, C::SBO, C::SWZ);
+  return make_desc(base + (kk / spp) * rows * C::ROWB + (kk % spp) * 32, 16, C::SBO, C::SWZ);
 }
+// MN-major operand: N = D contiguous in panels of rows x ROWB, k-step = 16 rows.
 template <int D>
-__device__ __forceinline__ uint64_t bwd_mndesc(uint32_t base, int kk) {  // MN-major, N = D, K = 128 rows
+__device__ __forceinline__ uint64_t bwd_mndesc(uint32_t base, int rows, int kk) {
   using C = BwdCfg<D>;
-  return make_desc(base + kk * 16 * C::ROWB, 128 * C::ROWB, C::SBO, C::SWZ);
+  return make_desc(base + kk * 16 * C::ROWB, rows * C::ROWB, C::SBO, C::SWZ);
 }
-// P^T / dS^T buffers: [128 rows][128 cols] bf16 as 2 panels of [128][64], 128B swizzle.
-__device__ __forceinline__ uint64_t pt_kdesc(uint32_t base, int kk) {  // K-major (K = cols)
-  return make_desc(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
+// [128 keys][64 queries] bf16 panel, 128B swizzle: K-major with K = queries.
+__device__ __forceinline__ uint64_t pt_kdesc(uint32_t base, int kk) {
+  return make_desc(base + kk * 32, 16, 1024, kSwizzle128);
 }
-__device__ __forceinline__ uint64_t pt_mndesc(uint32_t base, int kk) {  // MN-major (M = cols, K = rows)
+// A pair of panels viewed MN-major: M = 128 queries (2 panels), K = keys.
+__device__ __forceinline__ uint64_t pair_mndesc(uint32_t base, int kk) {
   return make_desc(base + kk * 2048, 16384, 1024, kSwizzle128);
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(448, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mdo_nat, const __grid_constant__ CUtensorMap mdo_col,
                   const __grid_constant__ CUtensorMap mk_nat, const __grid_constant__ CUtensorMap mk_col,
@@ -114,13 +132,15 @@ __global__ void __launch_bounds__(192, 1)
   float* sDelta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars;
-  uint64_t* bar_qdo_full = bars + 1;
-  uint64_t* bar_qdo_empty = bar_qdo_full + C::STAGES;
-  uint64_t* bar_st_full = bar_qdo_empty + C::STAGES;
-  uint64_t* bar_dpt_full = bar_st_full + 1;
-  uint64_t* bar_pt_full = bar_dpt_full + 1;
-  uint64_t* bar_dst_full = bar_pt_full + 1;
-  uint64_t* bar_dq_full = bar_dst_full + 1;
+  uint64_t* bar_qdo_full = bar_kv + 1;                 // [STAGES]
+  uint64_t* bar_qdo_empty = bar_qdo_full + C::STAGES;  // [STAGES]
+  uint64_t* bar_s_full = bar_qdo_empty + C::STAGES;    // [NBUF]  ST and dPT of a step
+  uint64_t* bar_s_free = bar_s_full + C::NBUF;         // [NBUF]  elementwise done reading them
+  uint64_t* bar_pt_full = bar_s_free + C::NBUF;        // [2]
+  uint64_t* bar_pt_free = bar_pt_full + 2;             // [2]
+  uint64_t* bar_dst_full = bar_pt_free + 2;            // [2]  per step parity
+  uint64_t* bar_dst_free = bar_dst_full + 2;           // [DST_BUFS] per pair
+  uint64_t* bar_dq_full = bar_dst_free + C::DST_BUFS;
   uint64_t* bar_dq_free = bar_dq_full + 1;
   uint64_t* bar_dkv_full = bar_dq_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -129,7 +149,7 @@ __global__ void __launch_bounds__(192, 1)
   const int bh = blockIdx.x;
   const int kt = a.order[blockIdx.y];
   const int e0 = a.row_ptr[kt];
-  const int n = a.row_ptr[kt + 1] - e0;
+  const int n = a.row_ptr[kt + 1] - e0;  // 64-query steps
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int q_src = (a.key_view == SRC_T) ? SRC_T : SRC_N;
@@ -137,13 +157,19 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(bar_qdo_full + s, 1);
+      mbar_init(bar_qdo_full + s, 2);  // TMA bytes + the producer warp's lse/Delta stores
       mbar_init(bar_qdo_empty + s, 1);
     }
-    mbar_init(bar_st_full, 1);
-    mbar_init(bar_dpt_full, 1);
-    mbar_init(bar_pt_full, 128);
-    mbar_init(bar_dst_full, 128);
+    for (int b = 0; b < C::NBUF; ++b) {
+      mbar_init(bar_s_full + b, 1);
+      mbar_init(bar_s_free + b, 256);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_pt_full + b, 256);
+      mbar_init(bar_pt_free + b, 1);
+      mbar_init(bar_dst_full + b, 256);
+    }
+    for (int b = 0; b < C::DST_BUFS; ++b) mbar_init(bar_dst_free + b, 1);
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_free, 128);
     mbar_init(bar_dkv_full, 1);
@@ -157,73 +183,114 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0 && n > 0) {
-      // ------------------------------------------------------------ producer
-      mbar_arrive_expect_tx(bar_kv, 2 * C::T_BYTES);
-      load_rows<D>(sK, a.key_view, kt * C::TK, C::TK, bh, &mk_nat, &mk_col, &mk_sum, bar_kv, a.R, a.l, a.c);
-      load_rows<D>(sV, a.key_view, kt * C::TK, C::TK, bh, &mv_nat, &mv_col, &mv_sum, bar_kv, a.R, a.l, a.c);
+    // ------------------------------------------------------------ producer
+    if (n > 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_kv, 2 * C::KV_BYTES);
+        load_rows<D>(sK, a.key_view, kt * C::TK, C::TK, bh, &mk_nat, &mk_col, &mk_sum, bar_kv, a.R, a.l, a.c);
+        load_rows<D>(sV, a.key_view, kt * C::TK, C::TK, bh, &mv_nat, &mv_col, &mv_sum, bar_kv, a.R, a.l, a.c);
+      }
       for (int j = 0; j < n; ++j) {
         const int st = j % C::STAGES;
         if (j >= C::STAGES && !mbar_wait(bar_qdo_empty + st, ((j / C::STAGES) - 1) & 1, abort_flag)) break;
         const int qpos = (a.ent[e0 + j] >> 3) * C::TQ;
-        mbar_arrive_expect_tx(bar_qdo_full + st, 2 * C::T_BYTES);
-        load_rows<D>(sQ + st * C::T_BYTES, q_src, qpos, C::TQ, bh, &mq_nat, &mq_col, &mq_col,
-                     bar_qdo_full + st, a.R, a.l, a.c);
-        load_rows<D>(sDO + st * C::T_BYTES, q_src, qpos, C::TQ, bh, &mdo_nat, &mdo_col, &mdo_col,
-                     bar_qdo_full + st, a.R, a.l, a.c);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_qdo_full + st, 2 * C::QS_BYTES);
+          load_rows<D>(sQ + st * C::QS_BYTES, q_src, qpos, C::TQ, bh, &mq_nat, &mq_col, &mq_col,
+                       bar_qdo_full + st, a.R, a.l, a.c);
+          load_rows<D>(sDO + st * C::QS_BYTES, q_src, qpos, C::TQ, bh, &mdo_nat, &mdo_col, &mdo_col,
+                       bar_qdo_full + st, a.R, a.l, a.c);
+        }
+        // lse (log2 units) and Delta of the step's 64 queries
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = h * 32 + lane;
+          const int x = qpos + i;
+          float lv = INFINITY, dv = 0.f;
+          if (x < a.N) {
+            const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
+            lv = a.lse[static_cast<size_t>(bh) * a.N + qn] * 1.4426950408889634f;
+            dv = a.delta[static_cast<size_t>(bh) * a.N + qn];
+          }
+          sLse[st * C::TQ + i] = lv;
+          sDelta[st * C::TQ + i] = dv;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_qdo_full + st);
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
-      // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t id_s = make_idesc_bf16(128, 128, false, false);  // ST, dPT
-      constexpr uint32_t id_kv = make_idesc_bf16(128, D, false, true);    // dV, dK
-      constexpr uint32_t id_q = make_idesc_bf16(128, D, true, true);      // dQ
+      constexpr uint32_t id_s = make_idesc_bf16(128, C::TQ, false, false);  // ST, dPT: N = 64 queries
+      constexpr uint32_t id_kv = make_idesc_bf16(128, D, false, true);      // dV, dK
+      constexpr uint32_t id_q = make_idesc_bf16(128, D, true, true);        // dQ (pair)
       const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
-      const uint32_t pt_base = smem_u32(sPT), dst_base = smem_u32(sDST);
       bool ok = mbar_wait(bar_kv, 0, abort_flag);
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % C::STAGES;
-        ok = mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
-        if (ok && j > 0) ok = mbar_wait(bar_dq_free, (j - 1) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ + st * C::T_BYTES);
-        const uint32_t do_base = smem_u32(sDO + st * C::T_BYTES);
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int st = j % C::STAGES;
+          const int b = j % C::NBUF;
+          ok = mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
+          if (ok && j >= C::NBUF) ok = mbar_wait(bar_s_free + b, ((j / C::NBUF) - 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
+          const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_ST, bwd_kdesc<D>(k_base, kk), bwd_kdesc<D>(q_base, kk), id_s, kk > 0);
-        mma_commit(bar_st_full);
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + b * 64, bwd_kdesc<D>(k_base, C::TK, kk), bwd_kdesc<D>(q_base, C::TQ, kk), id_s,
+                        kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_DPT, bwd_kdesc<D>(v_base, kk), bwd_kdesc<D>(do_base, kk), id_s, kk > 0);
-        mma_commit(bar_dpt_full);
-        if (!mbar_wait(bar_pt_full, j & 1, abort_flag)) break;
-        tc_fence_after();
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_DPT + b * 64, bwd_kdesc<D>(v_base, C::TK, kk),
+                        bwd_kdesc<D>(do_base, C::TQ, kk), id_s, kk > 0);
+          mma_commit(bar_s_full + b);
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int st = jj % C::STAGES;
+          const int pb = jj & 1;
+          const int pair = jj >> 1;
+          const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
+          const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
+          const uint32_t dst_pair = smem_u32(sDST + (pair % C::DST_BUFS) * C::DST_BYTES);
+          if (!mbar_wait(bar_pt_full + pb, (jj >> 1) & 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + C::COL_DV, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, kk), id_kv, (j > 0 || kk > 0));
-        if (!mbar_wait(bar_dst_full, j & 1, abort_flag)) break;
-        tc_fence_after();
+          for (int kk = 0; kk < C::TQ / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_DV, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
+                        (jj > 0 || kk > 0));
+          mma_commit(bar_pt_free + pb);
+          if (!mbar_wait(bar_dst_full + pb, (jj >> 1) & 1, abort_flag)) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + C::COL_DK, pt_kdesc(dst_base, kk), bwd_mndesc<D>(q_base, kk), id_kv, (j > 0 || kk > 0));
+          for (int kk = 0; kk < C::TQ / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_DK, pt_kdesc(dst_pair + pb * C::PT_BYTES, kk),
+                        bwd_mndesc<D>(q_base, C::TQ, kk), id_kv, (jj > 0 || kk > 0));
+          mma_commit(bar_qdo_empty + st);
+          if ((jj & 1) || jj == n - 1) {
+            if (pair >= 1 && !mbar_wait(bar_dq_free, (pair - 1) & 1, abort_flag)) break;
+            tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + C::COL_ST, pt_mndesc(dst_base, kk), bwd_mndesc<D>(k_base, kk), id_q, kk > 0);
-        mma_commit(bar_dq_full);
-        mma_commit(bar_qdo_empty + st);
+            for (int kk = 0; kk < C::TK / 16; ++kk)
+              mma_bf16_ss(tmem + C::COL_DQ, pair_mndesc(dst_pair, kk), bwd_mndesc<D>(k_base, C::TK, kk), id_q,
+                          kk > 0);
+            mma_commit(bar_dq_full);
+            mma_commit(bar_dst_free + (pair % C::DST_BUFS));
+          }
+        }
       }
       mma_commit(bar_dkv_full);
     }
-  } else {
+  } else if (warp < 10) {
     // ------------------------------------------------------------ elementwise
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // query columns [32*half, 32*half + 32) of a step
     const int row = quarter * 32 + lane;
-    const int ctid = threadIdx.x - 64;  // 0..127
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    // this thread's key: view position y, natural position
-    const int y = kt * C::TK + row;
+    const int y = kt * C::TK + row;  // this thread's key, view order
     const int nkeys = (a.key_view == SRC_S) ? a.R * a.c : a.N;
     const bool kvalid = y < nkeys;
     int knat;
@@ -250,35 +317,28 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int e = a.ent[e0 + j];
-      const int qt = e >> 3;
+      const int st = j % C::STAGES;
+      const int b = j % C::NBUF;
+      const int pb = j & 1;
+      const int pair = j >> 1;
       const bool partial = e & 1;
-      const int buf = j & 1;
-      // lse (log2 units) and Delta of this tile's queries
-      {
-        const int x = qt * C::TQ + ctid;
-        float lv = INFINITY, dv = 0.f;
-        if (x < a.N) {
-          const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
-          lv = a.lse[static_cast<size_t>(bh) * a.N + qn] * 1.4426950408889634f;
-          dv = a.delta[static_cast<size_t>(bh) * a.N + qn];
-        }
-        sLse[buf * 128 + ctid] = lv;
-        sDelta[buf * 128 + ctid] = dv;
-      }
-      named_bar_sync(1, 128);
-      const float* lse_t = sLse + buf * 128;
-      const float* del_t = sDelta + buf * 128;
-      const int x0 = qt * C::TQ;
-
-      // ---- P^T row (this key against 128 queries)
-      ok = ok && mbar_wait(bar_st_full, j & 1, abort_flag);
+      const int x0 = (e >> 3) * C::TQ + half * 32;
+      ok = ok && mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
+      ok = ok && mbar_wait(bar_s_full + b, (j / C::NBUF) & 1, abort_flag);
       tc_fence_after();
-      float p[128];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) tmem_ld16(tmem + lane_base + C::COL_ST + i * 16, p + i * 16);
+      float p[32];
+      tmem_ld16(tmem + lane_base + b * 64 + half * 32, p);
+      tmem_ld16(tmem + lane_base + b * 64 + half * 32 + 16, p + 16);
+      float dp[32];
+      tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + half * 32, dp);
+      tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + half * 32 + 16, dp + 16);
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_s_free + b);
+      const float* lse_t = sLse + st * C::TQ + half * 32;
+      const float* del_t = sDelta + st * C::TQ + half * 32;
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
+      for (int i = 0; i < 32; ++i) {
         float v = ex2(fmaf(p[i], a.scale_log2, -lse_t[i]));
         if (partial) {
           const int x = x0 + i;
@@ -286,71 +346,41 @@ __global__ void __launch_bounds__(192, 1)
         }
         p[i] = v;
       }
+      // P^T buffer pb is free once dV of step j-2 has completed
+      if (j >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((j >> 1) - 1) & 1, abort_flag);
+      uint8_t* pt = sPT + pb * C::PT_BYTES;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
+      for (int ch = 0; ch < 4; ++ch) {
         uint4 w;
         w.x = pack_bf16(p[ch * 8 + 0], p[ch * 8 + 1]);
         w.y = pack_bf16(p[ch * 8 + 2], p[ch * 8 + 3]);
         w.z = pack_bf16(p[ch * 8 + 4], p[ch * 8 + 5]);
         w.w = pack_bf16(p[ch * 8 + 6], p[ch * 8 + 7]);
-        *reinterpret_cast<uint4*>(sPT + (ch >> 3) * 16384 + sw128_offset(row, ch & 7)) = w;
+        *reinterpret_cast<uint4*>(pt + sw128_offset(row, half * 4 + ch)) = w;
       }
       fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_pt_full);
-
-      // ---- dS^T row
-      ok = ok && mbar_wait(bar_dpt_full, j & 1, abort_flag);
-      tc_fence_after();
+      mbar_arrive(bar_pt_full + pb);
+      // dS^T into panel pb of pair buffer pair % DST_BUFS (free once dQ of pair - DST_BUFS is done)
+      if (pair >= C::DST_BUFS)
+        ok = ok && mbar_wait(bar_dst_free + (pair % C::DST_BUFS), ((pair / C::DST_BUFS) - 1) & 1, abort_flag);
+      uint8_t* dst = sDST + (pair % C::DST_BUFS) * C::DST_BYTES + pb * C::PT_BYTES;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float dp[16];
-        tmem_ld16(tmem + lane_base + C::COL_DPT + i * 16, dp);
-        tmem_wait_ld();
-        float ds[16];
+      for (int ch = 0; ch < 4; ++ch) {
+        float d8[8];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) ds[u] = p[i * 16 + u] * (dp[u] - del_t[i * 16 + u]);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int ch = i * 2 + h;
-          uint4 w;
-          w.x = pack_bf16(ds[h * 8 + 0], ds[h * 8 + 1]);
-          w.y = pack_bf16(ds[h * 8 + 2], ds[h * 8 + 3]);
-          w.z = pack_bf16(ds[h * 8 + 4], ds[h * 8 + 5]);
-          w.w = pack_bf16(ds[h * 8 + 6], ds[h * 8 + 7]);
-          *reinterpret_cast<uint4*>(sDST + (ch >> 3) * 16384 + sw128_offset(row, ch & 7)) = w;
-        }
+        for (int u = 0; u < 8; ++u) d8[u] = p[ch * 8 + u] * (dp[ch * 8 + u] - del_t[ch * 8 + u]);
+        uint4 w;
+        w.x = pack_bf16(d8[0], d8[1]);
+        w.y = pack_bf16(d8[2], d8[3]);
+        w.z = pack_bf16(d8[4], d8[5]);
+        w.w = pack_bf16(d8[6], d8[7]);
+        *reinterpret_cast<uint4*>(dst + sw128_offset(row, half * 4 + ch)) = w;
       }
       fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_dst_full);
-
-      // ---- dQ rows: this thread now owns query row `row` of the tile
-      ok = ok && mbar_wait(bar_dq_full, j & 1, abort_flag);
-      tc_fence_after();
-      {
-        const int x = x0 + row;
-        const bool qvalid = x < a.N;
-        const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
-        float* dst = a.dq_acc + (static_cast<size_t>(bh) * a.N + (qvalid ? qn : 0)) * D;
-#pragma unroll
-        for (int i = 0; i < D / 16; ++i) {
-          float g[16];
-          tmem_ld16(tmem + lane_base + C::COL_ST + i * 16, g);
-          tmem_wait_ld();
-          if (qvalid) {
-#pragma unroll
-            for (int u = 0; u < 16; u += 4)
-              red_add_v4(dst + i * 16 + u, g[u] * a.scale, g[u + 1] * a.scale, g[u + 2] * a.scale,
-                         g[u + 3] * a.scale);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar_dq_free);
+      mbar_arrive(bar_dst_full + pb);
     }
 
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (dV, dK)
     if (n > 0) {
       ok = ok && mbar_wait(bar_dkv_full, 0, abort_flag);
       tc_fence_after();
@@ -359,12 +389,13 @@ __global__ void __launch_bounds__(192, 1)
     bool add = false;
     if (a.add_part == 1) add = true;
     else if (a.add_part == 2) add = (knat % a.l) >= (a.l - a.c);
+    constexpr int HC = D / 2;  // columns per half
 #pragma unroll
     for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
-      const uint32_t col = which ? C::COL_DK : C::COL_DV;
+      const uint32_t col = (which ? C::COL_DK : C::COL_DV) + half * HC;
       const float mul = which ? a.scale : 1.f;
 #pragma unroll
-      for (int i = 0; i < D / 16; ++i) {
+      for (int i = 0; i < HC / 16; ++i) {
         float g[16];
         if (n > 0) {
           tmem_ld16(tmem + lane_base + col + i * 16, g);
@@ -376,14 +407,15 @@ __global__ void __launch_bounds__(192, 1)
         if (!kvalid) continue;
 #pragma unroll
         for (int u = 0; u < 16; ++u) g[u] *= mul;
+        const size_t eo = off + half * HC + i * 16;
         if (a.key_view != SRC_N) {
-          float* dstp = (which ? a.dk_part : a.dv_part) + off + i * 16;
+          float* dstp = (which ? a.dk_part : a.dv_part) + eo;
 #pragma unroll
           for (int u = 0; u < 16; u += 4)
             *reinterpret_cast<float4*>(dstp + u) = make_float4(g[u], g[u + 1], g[u + 2], g[u + 3]);
         } else {
           if (add) {
-            const float* srcp = (which ? a.dk_part : a.dv_part) + off + i * 16;
+            const float* srcp = (which ? a.dk_part : a.dv_part) + eo;
 #pragma unroll
             for (int u = 0; u < 16; u += 4) {
               const float4 t = *reinterpret_cast<const float4*>(srcp + u);
@@ -402,11 +434,45 @@ __global__ void __launch_bounds__(192, 1)
           w1.y = pack_bf16(g[10], g[11]);
           w1.z = pack_bf16(g[12], g[13]);
           w1.w = pack_bf16(g[14], g[15]);
-          uint4* dstp = reinterpret_cast<uint4*>((which ? a.dk : a.dv) + off + i * 16);
+          uint4* dstp = reinterpret_cast<uint4*>((which ? a.dk : a.dv) + eo);
           dstp[0] = w0;
           dstp[1] = w1;
         }
       }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ reduction
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // query row of the pair: step 2p + row / 64
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const int n_pairs = (n + 1) >> 1;
+    bool ok = true;
+    for (int p = 0; p < n_pairs; ++p) {
+      ok = ok && mbar_wait(bar_dq_full, p & 1, abort_flag);
+      tc_fence_after();
+      const int s = 2 * p + (row >> 6);
+      bool qvalid = false;
+      float* dstp = a.dq_acc;
+      if (s < n) {
+        const int x = (a.ent[e0 + s] >> 3) * C::TQ + (row & 63);
+        qvalid = x < a.N;
+        const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
+        dstp = a.dq_acc + (static_cast<size_t>(bh) * a.N + (qvalid ? qn : 0)) * D;
+      }
+#pragma unroll
+      for (int i = 0; i < D / 16; ++i) {
+        float g[16];
+        tmem_ld16(tmem + lane_base + C::COL_DQ + i * 16, g);
+        tmem_wait_ld();
+        if (qvalid) {
+#pragma unroll
+          for (int u = 0; u < 16; u += 4)
+            red_add_v4(dstp + i * 16 + u, g[u] * a.scale, g[u + 1] * a.scale, g[u + 2] * a.scale,
+                       g[u + 3] * a.scale);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_dq_free);
     }
   }
 

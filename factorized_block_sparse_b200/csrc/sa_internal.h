@@ -17,7 +17,7 @@ namespace sa {
 constexpr int kFwdTQ = 128;  // forward: query rows per CTA (tcgen05 M)
 constexpr int kFwdTK = 64;   // forward: keys per step (tcgen05 N of Q K^T)
 constexpr int kBwdTK = 128;  // backward: keys per CTA (tcgen05 M of K Q^T)
-constexpr int kBwdTQ = 128;  // backward: queries per step
+constexpr int kBwdTQ = 64;   // backward: queries per step
 
 enum Src : int { SRC_N = 0, SRC_T = 1, SRC_S = 2 };
 
