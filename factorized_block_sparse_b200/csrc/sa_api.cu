@@ -291,7 +291,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     a.merge = 0;
     dim3 grid(g.BH, dc.fwd_col.n_rows);
     st = launch(K_FWD_COL * 4 + L->pattern, s, [&] {
-      kern<<<grid, 192, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
+      kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
     });
     if (st) return st;
   }
@@ -302,21 +302,30 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.merge = (two_pass && dc.fwd_col.n_rows > 0) ? 1 : 0;
   dim3 grid(g.BH, dc.fwd_main.n_rows);
   return launch(K_FWD_MAIN * 4 + L->pattern, s, [&] {
-    kern<<<grid, 192, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
+    kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
   });
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t delta, dq, dk, dv, total;
+  size_t ld_nat, ld_col, dq, dk, dv, total;
+  int n_pad;
 };
 
+// Backward workspace: packed (lse * log2 e, Delta) per query in natural order
+// (and column-major order for strided), the fp32 dQ accumulator, and for
+// strided / fixed the fp32 dK, dV partials of the secondary view.
 WsLayout ws_layout(int B, int H, int N, int D, const sa_layout* L) {
-  const size_t rows = static_cast<size_t>(B) * H * N;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t rows = BH * N;
   WsLayout w;
-  w.delta = 0;
-  w.dq = align256(rows * 4);
+  w.n_pad = (N + BwdCfg<64>::TQ - 1) / BwdCfg<64>::TQ * BwdCfg<64>::TQ;
+  const size_t ld_bytes = align256(BH * w.n_pad * 8);
+  w.ld_nat = 0;
+  w.ld_col = ld_bytes;
+  const bool col = L->pattern == SA_STRIDED;
+  w.dq = w.ld_col + (col ? ld_bytes : 0);
   w.dk = w.dq + align256(rows * D * 4);
   const bool sec = L->pattern == SA_STRIDED || L->pattern == SA_FIXED;
   w.dv = w.dk + (sec ? align256(rows * D * 4) : 0);
@@ -347,7 +356,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = set_smem(kern, BwdCfg<D>::SMEM))) return st;
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  float* delta = reinterpret_cast<float*>(wsb + w.delta);
+  float2* ld_nat = reinterpret_cast<float2*>(wsb + w.ld_nat);
+  float2* ld_col = (L->pattern == SA_STRIDED) ? reinterpret_cast<float2*>(wsb + w.ld_col) : nullptr;
   float* dq_acc = reinterpret_cast<float*>(wsb + w.dq);
   float* dk_part = reinterpret_cast<float*>(wsb + w.dk);
   float* dv_part = reinterpret_cast<float*>(wsb + w.dv);
@@ -355,13 +365,15 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
 
   st = launch(K_BWD_PRE * 4 + L->pattern, s, [&] {
     sa_bwd_pre_kernel<D><<<grid_for(rows * (D / 8), 256), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta, dq_acc, rows);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ld_nat, ld_col, dq_acc,
+        g.BH, N, w.n_pad, g.l, g.R);
   });
   if (st) return st;
 
   BwdArgs a;
-  a.lse = lse;
-  a.delta = delta;
+  a.ld_nat = ld_nat;
+  a.ld_col = ld_col ? ld_col : ld_nat;
+  a.n_pad = w.n_pad;
   a.dq_acc = dq_acc;
   a.dk = static_cast<__nv_bfloat16*>(dk);
   a.dv = static_cast<__nv_bfloat16*>(dv);

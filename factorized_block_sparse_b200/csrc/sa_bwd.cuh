@@ -18,13 +18,16 @@
 //   every second step: dQ = dS_pair K for the two steps' 128 queries
 //                      (M = 128), read by the dQ warps and added to an fp32
 //                      workspace with vector reductions.
-// Roles (448 threads): warp 0 producer (TMA for K, V, Q, dO; plain loads of
-// lse and Delta), warp 1 TMEM allocation and lane 0 MMA issue, warps 2..9
-// elementwise (two warps per TMEM lane quarter, 32 query columns each),
-// warps 10..13 dQ reduction.  Warp w may only touch TMEM lanes
+// Roles (480 threads): warp 0 producer (TMA for K, V, Q, dO; bulk copy of
+// the packed lse/Delta), warp 1 TMEM allocation and lane 0 issue of ST/dPT,
+// warps 2..9 elementwise (two groups of four, one warp per TMEM lane quarter
+// each, taking alternate steps), warps 10..13 dQ reduction, warp 14 lane 0 issue of dV/dK/dQ.  Two
+// issuing threads keep the S products of later steps flowing while dV/dK/dQ
+// of earlier steps wait on the elementwise warps.  Warp w may only touch TMEM lanes
 // 32*(w%4)..32*(w%4)+31, so every role picks its rows by w%4.
 // TMEM columns (NBUF = 2 for D <= 64, 1 for D = 128):
-//   ST[b] = b*64, dPT[b] = NBUF*64 + b*64, dV = 2*NBUF*64, dK = dV + D, dQ = dK + D.
+//   ST[b] = b*64, dPT[b] = NBUF*64 + b*64, dV = 2*NBUF*64, dK = dV + D,
+//   dQ[b] = dK + D + b*D (two dQ buffers for D <= 64, one for D = 128).
 #pragma once
 
 #include "sa_device.cuh"
@@ -36,8 +39,9 @@ struct BwdArgs {
   const int32_t* row_ptr;
   const int32_t* ent;
   const int32_t* order;
-  const float* lse;      // [BH, N] natural log
-  const float* delta;    // [BH, N]
+  const float2* ld_nat;  // [BH, n_pad] (lse * log2(e), Delta) in natural query order
+  const float2* ld_col;  // [BH, n_pad] the same in column-major order (strided)
+  int n_pad;             // N rounded up to the 64-query step, padded with (+inf, 0)
   float* dq_acc;         // [BH, N, D] fp32, scaled
   __nv_bfloat16* dk;     // final outputs (main pass)
   __nv_bfloat16* dv;
@@ -57,7 +61,7 @@ struct BwdCfg {
   static constexpr int NBUF = (D >= 128) ? 1 : 2;      // ST/dPT buffers in TMEM
   // Q/dO ring.  At least 2: the MMA issuer asks for step j's Q/dO before it
   // releases step j-1's (it issues S_j ahead of dV/dK of step j-1).
-  static constexpr int STAGES = (D >= 128) ? 2 : 3;
+  static constexpr int STAGES = (D >= 128) ? 2 : 4;
   static constexpr int DST_BUFS = (D >= 128) ? 1 : 2;  // dS^T pair buffers
   static constexpr int ROWB = (D >= 64) ? 128 : 64;
   static constexpr uint64_t SWZ = (D >= 64) ? kSwizzle128 : kSwizzle64;
@@ -72,10 +76,12 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + STAGES * QS_BYTES;
   static constexpr int OFF_PT = OFF_DO + STAGES * QS_BYTES;
   static constexpr int OFF_DST = OFF_PT + 2 * PT_BYTES;
-  static constexpr int OFF_LSE = OFF_DST + DST_BUFS * DST_BYTES;  // float [STAGES][64]
-  static constexpr int OFF_DELTA = OFF_LSE + STAGES * TQ * 4;      // float [STAGES][64]
-  static constexpr int OFF_BAR = OFF_DELTA + STAGES * TQ * 4;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 2 * NBUF + 2 * 2 + 2 + 2 * DST_BUFS + 3;
+  static constexpr int OFF_LD = OFF_DST + DST_BUFS * DST_BYTES;  // float2 [STAGES][64]
+  static constexpr int LD_BYTES = TQ * 8;
+  static constexpr int OFF_ENT = OFF_LD + STAGES * LD_BYTES;
+  static constexpr int OFF_BAR = OFF_ENT + kMaxStagedEnt * 4;
+  static constexpr int DQBUF = (D >= 128) ? 1 : 2;       // dQ TMEM buffers
+  static constexpr int N_BARS = 1 + 2 * STAGES + 2 * 2 + 2 * 2 + 2 + DST_BUFS + 2 * DQBUF + 1;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
@@ -83,8 +89,8 @@ struct BwdCfg {
   static constexpr int COL_DV = 2 * NBUF * 64;
   static constexpr int COL_DK = COL_DV + D;
   static constexpr int COL_DQ = COL_DK + D;
-  static constexpr int THREADS = 448;
-  static_assert(COL_DQ + D <= TMEM_COLS, "TMEM budget");
+  static constexpr int THREADS = 480;
+  static_assert(COL_DQ + DQBUF * D <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 2, "the software-pipelined MMA loop needs two Q/dO stages");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
@@ -112,7 +118,7 @@ __device__ __forceinline__ uint64_t pair_mndesc(uint32_t base, int kk) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(480, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mdo_nat, const __grid_constant__ CUtensorMap mdo_col,
                   const __grid_constant__ CUtensorMap mk_nat, const __grid_constant__ CUtensorMap mk_col,
@@ -128,28 +134,33 @@ __global__ void __launch_bounds__(448, 1)
   uint8_t* sDO = smem + C::OFF_DO;
   uint8_t* sPT = smem + C::OFF_PT;
   uint8_t* sDST = smem + C::OFF_DST;
-  float* sLse = reinterpret_cast<float*>(smem + C::OFF_LSE);
-  float* sDelta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
+  float2* sLD = reinterpret_cast<float2*>(smem + C::OFF_LD);
+  int32_t* sEnt = reinterpret_cast<int32_t*>(smem + C::OFF_ENT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars;
   uint64_t* bar_qdo_full = bar_kv + 1;                 // [STAGES]
   uint64_t* bar_qdo_empty = bar_qdo_full + C::STAGES;  // [STAGES]
-  uint64_t* bar_s_full = bar_qdo_empty + C::STAGES;    // [NBUF]  ST and dPT of a step
-  uint64_t* bar_s_free = bar_s_full + C::NBUF;         // [NBUF]  elementwise done reading them
-  uint64_t* bar_pt_full = bar_s_free + C::NBUF;        // [2]
+  // s_full / s_free are indexed by step parity (one per elementwise group),
+  // not by TMEM buffer: with a single buffer the two groups alternate on it,
+  // and a shared barrier could be waited on two phases ahead.
+  uint64_t* bar_s_full = bar_qdo_empty + C::STAGES;    // [2]  ST and dPT of a step
+  uint64_t* bar_s_free = bar_s_full + 2;               // [2]  elementwise done reading them
+  uint64_t* bar_pt_full = bar_s_free + 2;              // [2]
   uint64_t* bar_pt_free = bar_pt_full + 2;             // [2]
   uint64_t* bar_dst_full = bar_pt_free + 2;            // [2]  per step parity
   uint64_t* bar_dst_free = bar_dst_full + 2;           // [DST_BUFS] per pair
-  uint64_t* bar_dq_full = bar_dst_free + C::DST_BUFS;
-  uint64_t* bar_dq_free = bar_dq_full + 1;
-  uint64_t* bar_dkv_full = bar_dq_free + 1;
+  uint64_t* bar_dq_full = bar_dst_free + C::DST_BUFS;  // [DQBUF]
+  uint64_t* bar_dq_free = bar_dq_full + C::DQBUF;      // [DQBUF]
+  uint64_t* bar_dkv_full = bar_dq_free + C::DQBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x;  // all heads of the longest tiles first (longest-first balance)
   const int kt = a.order[blockIdx.y];
   const int e0 = a.row_ptr[kt];
   const int n = a.row_ptr[kt + 1] - e0;  // 64-query steps
+  const int32_t* gEnt = a.ent + e0;
+  stage_entries(sEnt, gEnt, n);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int q_src = (a.key_view == SRC_T) ? SRC_T : SRC_N;
@@ -157,21 +168,23 @@ __global__ void __launch_bounds__(448, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(bar_qdo_full + s, 2);  // TMA bytes + the producer warp's lse/Delta stores
+      mbar_init(bar_qdo_full + s, 1);
       mbar_init(bar_qdo_empty + s, 1);
     }
-    for (int b = 0; b < C::NBUF; ++b) {
+    for (int b = 0; b < 2; ++b) {
       mbar_init(bar_s_full + b, 1);
-      mbar_init(bar_s_free + b, 256);
+      mbar_init(bar_s_free + b, 128);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_pt_full + b, 256);
+      mbar_init(bar_pt_full + b, 128);
       mbar_init(bar_pt_free + b, 1);
-      mbar_init(bar_dst_full + b, 256);
+      mbar_init(bar_dst_full + b, 128);
     }
     for (int b = 0; b < C::DST_BUFS; ++b) mbar_init(bar_dst_free + b, 1);
-    mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 128);
+    for (int b = 0; b < C::DQBUF; ++b) {
+      mbar_init(bar_dq_full + b, 1);
+      mbar_init(bar_dq_free + b, 128);
+    }
     mbar_init(bar_dkv_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -190,96 +203,94 @@ __global__ void __launch_bounds__(448, 1)
         load_rows<D>(sK, a.key_view, kt * C::TK, C::TK, bh, &mk_nat, &mk_col, &mk_sum, bar_kv, a.R, a.l, a.c);
         load_rows<D>(sV, a.key_view, kt * C::TK, C::TK, bh, &mv_nat, &mv_col, &mv_sum, bar_kv, a.R, a.l, a.c);
       }
-      for (int j = 0; j < n; ++j) {
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES && !mbar_wait(bar_qdo_empty + st, ((j / C::STAGES) - 1) & 1, abort_flag)) break;
-        const int qpos = (a.ent[e0 + j] >> 3) * C::TQ;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar_qdo_full + st, 2 * C::QS_BYTES);
+      if (lane == 0) {
+        const float2* ld = (q_src == SRC_T ? a.ld_col : a.ld_nat) + static_cast<size_t>(bh) * a.n_pad;
+        for (int j = 0; j < n; ++j) {
+          const int st = j % C::STAGES;
+          if (j >= C::STAGES && !mbar_wait(bar_qdo_empty + st, ((j / C::STAGES) - 1) & 1, abort_flag)) break;
+          const int qpos = (entry_at(sEnt, gEnt, j) >> 3) * C::TQ;
+          mbar_arrive_expect_tx(bar_qdo_full + st, 2 * C::QS_BYTES + C::LD_BYTES);
           load_rows<D>(sQ + st * C::QS_BYTES, q_src, qpos, C::TQ, bh, &mq_nat, &mq_col, &mq_col,
                        bar_qdo_full + st, a.R, a.l, a.c);
           load_rows<D>(sDO + st * C::QS_BYTES, q_src, qpos, C::TQ, bh, &mdo_nat, &mdo_col, &mdo_col,
                        bar_qdo_full + st, a.R, a.l, a.c);
+          bulk_load(sLD + st * C::TQ, ld + qpos, C::LD_BYTES, bar_qdo_full + st);
         }
-        // lse (log2 units) and Delta of the step's 64 queries
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int i = h * 32 + lane;
-          const int x = qpos + i;
-          float lv = INFINITY, dv = 0.f;
-          if (x < a.N) {
-            const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
-            lv = a.lse[static_cast<size_t>(bh) * a.N + qn] * 1.4426950408889634f;
-            dv = a.delta[static_cast<size_t>(bh) * a.N + qn];
-          }
-          sLse[st * C::TQ + i] = lv;
-          sDelta[st * C::TQ + i] = dv;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_qdo_full + st);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer: ST_j, dPT_j
+    // Runs up to NBUF steps ahead of the elementwise warps; only waits for
+    // the step's Q/dO and for its TMEM buffer to be read out.
     if (lane == 0 && n > 0) {
-      constexpr uint32_t id_s = make_idesc_bf16(128, C::TQ, false, false);  // ST, dPT: N = 64 queries
-      constexpr uint32_t id_kv = make_idesc_bf16(128, D, false, true);      // dV, dK
-      constexpr uint32_t id_q = make_idesc_bf16(128, D, true, true);        // dQ (pair)
+      constexpr uint32_t id_s = make_idesc_bf16(128, C::TQ, false, false);  // N = 64 queries
       const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
       bool ok = mbar_wait(bar_kv, 0, abort_flag);
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j < n) {
-          const int st = j % C::STAGES;
-          const int b = j % C::NBUF;
-          ok = mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
-          if (ok && j >= C::NBUF) ok = mbar_wait(bar_s_free + b, ((j / C::NBUF) - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
-          const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16_ss(tmem + b * 64, bwd_kdesc<D>(k_base, C::TK, kk), bwd_kdesc<D>(q_base, C::TQ, kk), id_s,
-                        kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_DPT + b * 64, bwd_kdesc<D>(v_base, C::TK, kk),
-                        bwd_kdesc<D>(do_base, C::TQ, kk), id_s, kk > 0);
-          mma_commit(bar_s_full + b);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % C::STAGES;
+        const int b = j % C::NBUF;
+        ok = mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
+        if (ok && j >= C::NBUF) {  // buffer b was last used by step j - NBUF
+          const int jp = j - C::NBUF;
+          ok = mbar_wait(bar_s_free + (jp & 1), (jp >> 1) & 1, abort_flag);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int st = jj % C::STAGES;
-          const int pb = jj & 1;
-          const int pair = jj >> 1;
-          const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
-          const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
-          const uint32_t dst_pair = smem_u32(sDST + (pair % C::DST_BUFS) * C::DST_BYTES);
-          if (!mbar_wait(bar_pt_full + pb, (jj >> 1) & 1, abort_flag)) break;
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
+        const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem + b * 64, bwd_kdesc<D>(k_base, C::TK, kk), bwd_kdesc<D>(q_base, C::TQ, kk), id_s,
+                      kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem + C::COL_DPT + b * 64, bwd_kdesc<D>(v_base, C::TK, kk),
+                      bwd_kdesc<D>(do_base, C::TQ, kk), id_s, kk > 0);
+        mma_commit(bar_s_full + (j & 1));
+      }
+    }
+  } else if (warp == 14) {
+    // ------------------------------------------------------------ G issuer: dV, dK, dQ
+    // Its commits track only its own MMAs; the S issuer's products of a step
+    // are complete before the step's P^T exists, so releasing the Q/dO stage
+    // after dK covers both issuers.
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t id_kv = make_idesc_bf16(128, D, false, true);  // dV, dK
+      constexpr uint32_t id_q = make_idesc_bf16(128, D, true, true);    // dQ (pair)
+      const uint32_t k_base = smem_u32(sK);
+      bool ok = mbar_wait(bar_kv, 0, abort_flag);
+      for (int jj = 0; ok && jj < n; ++jj) {
+        const int st = jj % C::STAGES;
+        const int pb = jj & 1;
+        const int pair = jj >> 1;
+        const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
+        const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
+        const uint32_t dst_pair = smem_u32(sDST + (pair % C::DST_BUFS) * C::DST_BYTES);
+        if (!mbar_wait(bar_pt_full + pb, (jj >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < C::TQ / 16; ++kk)
+          mma_bf16_ss(tmem + C::COL_DV, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
+                      (jj > 0 || kk > 0));
+        mma_commit(bar_pt_free + pb);
+        if (!mbar_wait(bar_dst_full + pb, (jj >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::TQ / 16; ++kk)
+          mma_bf16_ss(tmem + C::COL_DK, pt_kdesc(dst_pair + pb * C::PT_BYTES, kk),
+                      bwd_mndesc<D>(q_base, C::TQ, kk), id_kv, (jj > 0 || kk > 0));
+        mma_commit(bar_qdo_empty + st);
+        if ((jj & 1) || jj == n - 1) {
+          const int qb = pair % C::DQBUF;
+          if (pair >= C::DQBUF && !mbar_wait(bar_dq_free + qb, ((pair / C::DQBUF) - 1) & 1, abort_flag)) break;
           tc_fence_after();
-          const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::TQ / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_DV, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
-                        (jj > 0 || kk > 0));
-          mma_commit(bar_pt_free + pb);
-          if (!mbar_wait(bar_dst_full + pb, (jj >> 1) & 1, abort_flag)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < C::TQ / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_DK, pt_kdesc(dst_pair + pb * C::PT_BYTES, kk),
-                        bwd_mndesc<D>(q_base, C::TQ, kk), id_kv, (jj > 0 || kk > 0));
-          mma_commit(bar_qdo_empty + st);
-          if ((jj & 1) || jj == n - 1) {
-            if (pair >= 1 && !mbar_wait(bar_dq_free, (pair - 1) & 1, abort_flag)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < C::TK / 16; ++kk)
-              mma_bf16_ss(tmem + C::COL_DQ, pair_mndesc(dst_pair, kk), bwd_mndesc<D>(k_base, C::TK, kk), id_q,
-                          kk > 0);
-            mma_commit(bar_dq_full);
-            mma_commit(bar_dst_free + (pair % C::DST_BUFS));
-          }
+          for (int kk = 0; kk < C::TK / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_DQ + qb * D, pair_mndesc(dst_pair, kk), bwd_mndesc<D>(k_base, C::TK, kk),
+                        id_q, kk > 0);
+          mma_commit(bar_dq_full + qb);
+          mma_commit(bar_dst_free + (pair % C::DST_BUFS));
         }
       }
       mma_commit(bar_dkv_full);
@@ -287,7 +298,7 @@ __global__ void __launch_bounds__(448, 1)
   } else if (warp < 10) {
     // ------------------------------------------------------------ elementwise
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;  // query columns [32*half, 32*half + 32) of a step
+    const int half = (warp - 2) >> 2;  // step parity of this group; dV/dK column half in the epilogue
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int y = kt * C::TK + row;  // this thread's key, view order
@@ -314,69 +325,81 @@ __global__ void __launch_bounds__(448, 1)
     if (qhi > a.N - 1) qhi = a.N - 1;
     if (!kvalid) qhi = qlo - 1;
 
+    // Group `half` takes the steps j with j % 2 == half, each thread a whole
+    // 64-query row in chunks of 16 columns; the two groups run out of phase,
+    // so one group's exp2 (MUFU) work overlaps the other's dS (ALU) work.
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int e = a.ent[e0 + j];
+    for (int j = half; j < n; j += 2) {
+      const int e = entry_at(sEnt, gEnt, j);
       const int st = j % C::STAGES;
       const int b = j % C::NBUF;
       const int pb = j & 1;
       const int pair = j >> 1;
       const bool partial = e & 1;
-      const int x0 = (e >> 3) * C::TQ + half * 32;
+      const int x0 = (e >> 3) * C::TQ;
       ok = ok && mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
-      ok = ok && mbar_wait(bar_s_full + b, (j / C::NBUF) & 1, abort_flag);
-      tc_fence_after();
-      float p[32];
-      tmem_ld16(tmem + lane_base + b * 64 + half * 32, p);
-      tmem_ld16(tmem + lane_base + b * 64 + half * 32 + 16, p + 16);
-      float dp[32];
-      tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + half * 32, dp);
-      tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + half * 32 + 16, dp + 16);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_s_free + b);
-      const float* lse_t = sLse + st * C::TQ + half * 32;
-      const float* del_t = sDelta + st * C::TQ + half * 32;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float v = ex2(fmaf(p[i], a.scale_log2, -lse_t[i]));
-        if (partial) {
-          const int x = x0 + i;
-          if (x < qlo || x > qhi) v = 0.f;
-        }
-        p[i] = v;
-      }
-      // P^T buffer pb is free once dV of step j-2 has completed
+      ok = ok && mbar_wait(bar_s_full + pb, (j >> 1) & 1, abort_flag);
+      // P^T buffer pb is free once dV of step j-2 has completed; dS^T pair
+      // buffer once dQ of pair - DST_BUFS has completed.
       if (j >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((j >> 1) - 1) & 1, abort_flag);
+      if (pair >= C::DST_BUFS)
+        ok = ok && mbar_wait(bar_dst_free + (pair % C::DST_BUFS), ((pair / C::DST_BUFS) - 1) & 1, abort_flag);
+      tc_fence_after();
+      const float4* ld_t = reinterpret_cast<const float4*>(sLD + st * C::TQ);  // (lse*log2 e, Delta) x 2
       uint8_t* pt = sPT + pb * C::PT_BYTES;
+      uint8_t* dst = sDST + (pair % C::DST_BUFS) * C::DST_BYTES + pb * C::PT_BYTES;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint4 w;
-        w.x = pack_bf16(p[ch * 8 + 0], p[ch * 8 + 1]);
-        w.y = pack_bf16(p[ch * 8 + 2], p[ch * 8 + 3]);
-        w.z = pack_bf16(p[ch * 8 + 4], p[ch * 8 + 5]);
-        w.w = pack_bf16(p[ch * 8 + 6], p[ch * 8 + 7]);
-        *reinterpret_cast<uint4*>(pt + sw128_offset(row, half * 4 + ch)) = w;
+      for (int c16 = 0; c16 < 4; ++c16) {
+        float p[16], dp[16];
+        tmem_ld16(tmem + lane_base + b * 64 + c16 * 16, p);
+        tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + c16 * 16, dp);
+        tmem_wait_ld();
+        if (c16 == 3) {  // both TMEM buffers of this step have been read
+          tc_fence_before();
+          mbar_arrive(bar_s_free + pb);
+        }
+        float lse2[16], dl[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 t = ld_t[c16 * 8 + i];
+          lse2[2 * i] = t.x;
+          dl[2 * i] = t.y;
+          lse2[2 * i + 1] = t.z;
+          dl[2 * i + 1] = t.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float v = ex2(fmaf(p[i], a.scale_log2, -lse2[i]));
+          if (partial) {
+            const int x = x0 + c16 * 16 + i;
+            if (x < qlo || x > qhi) v = 0.f;
+          }
+          p[i] = v;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint4 w;
+          w.x = pack_bf16(p[h * 8 + 0], p[h * 8 + 1]);
+          w.y = pack_bf16(p[h * 8 + 2], p[h * 8 + 3]);
+          w.z = pack_bf16(p[h * 8 + 4], p[h * 8 + 5]);
+          w.w = pack_bf16(p[h * 8 + 6], p[h * 8 + 7]);
+          *reinterpret_cast<uint4*>(pt + sw128_offset(row, c16 * 2 + h)) = w;
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float d8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) d8[u] = p[h * 8 + u] * (dp[h * 8 + u] - dl[h * 8 + u]);
+          uint4 w;
+          w.x = pack_bf16(d8[0], d8[1]);
+          w.y = pack_bf16(d8[2], d8[3]);
+          w.z = pack_bf16(d8[4], d8[5]);
+          w.w = pack_bf16(d8[6], d8[7]);
+          *reinterpret_cast<uint4*>(dst + sw128_offset(row, c16 * 2 + h)) = w;
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(bar_pt_full + pb);
-      // dS^T into panel pb of pair buffer pair % DST_BUFS (free once dQ of pair - DST_BUFS is done)
-      if (pair >= C::DST_BUFS)
-        ok = ok && mbar_wait(bar_dst_free + (pair % C::DST_BUFS), ((pair / C::DST_BUFS) - 1) & 1, abort_flag);
-      uint8_t* dst = sDST + (pair % C::DST_BUFS) * C::DST_BYTES + pb * C::PT_BYTES;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        float d8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) d8[u] = p[ch * 8 + u] * (dp[ch * 8 + u] - del_t[ch * 8 + u]);
-        uint4 w;
-        w.x = pack_bf16(d8[0], d8[1]);
-        w.y = pack_bf16(d8[2], d8[3]);
-        w.z = pack_bf16(d8[4], d8[5]);
-        w.w = pack_bf16(d8[6], d8[7]);
-        *reinterpret_cast<uint4*>(dst + sw128_offset(row, half * 4 + ch)) = w;
-      }
-      fence_proxy_async_smem();
       mbar_arrive(bar_dst_full + pb);
     }
 
@@ -440,7 +463,7 @@ __global__ void __launch_bounds__(448, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 14) {
     // ------------------------------------------------------------ dQ reduction
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // query row of the pair: step 2p + row / 64
@@ -448,13 +471,14 @@ __global__ void __launch_bounds__(448, 1)
     const int n_pairs = (n + 1) >> 1;
     bool ok = true;
     for (int p = 0; p < n_pairs; ++p) {
-      ok = ok && mbar_wait(bar_dq_full, p & 1, abort_flag);
+      const int qb = p % C::DQBUF;
+      ok = ok && mbar_wait(bar_dq_full + qb, (p / C::DQBUF) & 1, abort_flag);
       tc_fence_after();
       const int s = 2 * p + (row >> 6);
       bool qvalid = false;
       float* dstp = a.dq_acc;
       if (s < n) {
-        const int x = (a.ent[e0 + s] >> 3) * C::TQ + (row & 63);
+        const int x = (entry_at(sEnt, gEnt, s) >> 3) * C::TQ + (row & 63);
         qvalid = x < a.N;
         const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
         dstp = a.dq_acc + (static_cast<size_t>(bh) * a.N + (qvalid ? qn : 0)) * D;
@@ -462,7 +486,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
       for (int i = 0; i < D / 16; ++i) {
         float g[16];
-        tmem_ld16(tmem + lane_base + C::COL_DQ + i * 16, g);
+        tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, g);
         tmem_wait_ld();
         if (qvalid) {
 #pragma unroll
@@ -472,7 +496,7 @@ __global__ void __launch_bounds__(448, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_dq_free);
+      mbar_arrive(bar_dq_free + qb);
     }
   }
 
@@ -484,20 +508,28 @@ __global__ void __launch_bounds__(448, 1)
   }
 }
 
-// Delta[bh, i] = sum_d dO[bh, i, d] * O[bh, i, d] (fp32), and zero the fp32
-// dQ accumulator.  D/8 threads per row, 16-byte loads; the row loop is
-// warp-uniform so the shuffles always see every lane.
+// Backward preprocess, one row per D/8 threads (16-byte loads; the row loop
+// is warp-uniform so the shuffles always see every lane):
+//   Delta_i = sum_d dO_id O_id (fp32); writes (lse_i * log2 e, Delta_i) to the
+//   natural-order array and, for the strided pattern, at the row's
+//   column-major position t = (i mod l) * R + i / l; pads positions
+//   [N, n_pad) of both with (+inf, 0); zeroes the fp32 dQ accumulator.
 template <int D>
 __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
-                                                         float* __restrict__ delta,
-                                                         float* __restrict__ dq_acc, long long rows) {
+                                                         const float* __restrict__ lse,
+                                                         float2* __restrict__ ld_nat, float2* __restrict__ ld_col,
+                                                         float* __restrict__ dq_acc, int BH, int N, int n_pad,
+                                                         int l, int R) {
   constexpr int TPR = D / 8;         // threads per row
   constexpr int RPW = 32 / TPR;      // rows per warp per step
+  const long long rows = static_cast<long long>(BH) * N;
   const int lane = threadIdx.x & 31;
   const int sub = lane % TPR;
-  const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long nthr = static_cast<long long>(gridDim.x) * blockDim.x;
+  const long long warp_id = tid >> 5;
+  const long long n_warps = nthr >> 5;
   for (long long r0 = warp_id * RPW; r0 < rows; r0 += n_warps * RPW) {
     const long long r = r0 + lane / TPR;
     const bool valid = r < rows;
@@ -518,11 +550,24 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
 #pragma unroll
     for (int w = TPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w, TPR);
     if (valid) {
-      if (sub == 0) delta[r] = acc;
+      if (sub == 0) {
+        const long long bh = r / N;
+        const int i = static_cast<int>(r - bh * N);
+        const float2 v = make_float2(lse[r] * 1.4426950408889634f, acc);
+        ld_nat[bh * n_pad + i] = v;
+        if (ld_col) ld_col[bh * n_pad + (i % l) * R + i / l] = v;
+      }
       float4* z = reinterpret_cast<float4*>(dq_acc + r * D + sub * 8);
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+  }
+  const int pad = n_pad - N;
+  for (long long k = tid; k < static_cast<long long>(BH) * pad; k += nthr) {
+    const long long bh = k / pad;
+    const long long i = N + (k - bh * pad);
+    ld_nat[bh * n_pad + i] = make_float2(INFINITY, 0.f);
+    if (ld_col) ld_col[bh * n_pad + i] = make_float2(INFINITY, 0.f);
   }
 }
 

@@ -60,6 +60,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a waiting thread is parked by the
+// hardware until the phase completes or about `hint_ns` nanoseconds pass,
+// instead of spinning and taking issue slots from the working warps.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  After about 2^31 SM
 // cycles without completion (or once any CTA has already recorded a
 // timeout) it records SA_ERR_TIMEOUT in the status word, sets *abort and
@@ -69,8 +84,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* a
   if (*(volatile int*)abort) return false;
   const long long t0 = clock64();
   uint32_t spins = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if (((++spins) & 1023u) == 0) {
+  while (!mbar_try_wait_hint(bar, parity, 20000u)) {
+    if (((++spins) & 15u) == 0) {
       if (*(volatile int*)abort || *(volatile int*)&g_status == kStatusTimeout) {
         *(volatile int*)abort = 1;
         return false;
@@ -111,6 +126,30 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, uin
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
       : "memory");
+}
+
+// Untiled bulk copy global -> shared (both 16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ------------------------------------------------------- staged tile lists
+// Each CTA copies its row of the tile table into shared memory once, so no
+// role pays a global-memory round trip per step.  Longer rows (beyond
+// kMaxStagedEnt entries) read the tail from global memory.
+constexpr int kMaxStagedEnt = 1024;
+
+__device__ __forceinline__ void stage_entries(int32_t* s_ent, const int32_t* g_ent, int n) {
+  const int m = n < kMaxStagedEnt ? n : kMaxStagedEnt;
+  for (int i = threadIdx.x; i < m; i += blockDim.x) s_ent[i] = g_ent[i];
+}
+
+__device__ __forceinline__ int entry_at(const int32_t* s_ent, const int32_t* g_ent, int j) {
+  return j < kMaxStagedEnt ? s_ent[j] : g_ent[j];
 }
 
 // ---------------------------------------------------------------- tcgen05

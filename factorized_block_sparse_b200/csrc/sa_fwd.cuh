@@ -10,11 +10,13 @@
 // layout ("OpenAI Sparse Transformer", "Sparse Attention and Algorithmic
 // Complexity" and "Implementation and Limitations").
 //
-// Roles (192 threads):
+// Roles (224 threads):
 //   warp 0 lane 0 : TMA producer (Q once, K/V through a STAGES-deep ring)
-//   warp 1        : allocates TMEM; lane 0 issues every tcgen05.mma
+//   warp 1        : allocates TMEM; lane 0 issues S = Q K^T
 //   warps 2..5    : softmax; thread t of warp w owns query row
-//                   32*(w%4)+t, which is TMEM lane 32*(w%4)+t.
+//                   32*(w%4)+t, which is TMEM lane 32*(w%4)+t
+//   warp 6 lane 0 : issues O += P V (a second issuing thread, so S of the
+//                   next tiles never waits behind PV of earlier ones)
 // TMEM columns: S double buffer [0,64) and [64,128); O accumulator [128,128+D).
 //
 // The running max is only moved when it grows by more than 2^8 (in the
@@ -55,12 +57,14 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_ENT = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_BAR = OFF_ENT + kMaxStagedEnt * 4;
   static constexpr int N_BARS = 1 + 3 * STAGES + 8;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 256;
   static constexpr int COL_O = 128;
+  static constexpr int THREADS = 224;
 };
 
 // Loads a tile of `rows` positions starting at view position `pos0` into
@@ -119,7 +123,7 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int rows, int kk
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
     sa_fwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mk_nat, const __grid_constant__ CUtensorMap mk_col,
                   const __grid_constant__ CUtensorMap mk_sum, const __grid_constant__ CUtensorMap mv_nat,
@@ -143,11 +147,14 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bar_pv_done = bar_p_full + 2;           // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  int32_t* sEnt = reinterpret_cast<int32_t*>(smem + C::OFF_ENT);
 
-  const int bh = blockIdx.x;
+  const int bh = blockIdx.x;  // all heads of the longest tiles first (longest-first balance)
   const int qt = a.order[blockIdx.y];
   const int e0 = a.row_ptr[qt];
   const int n = a.row_ptr[qt + 1] - e0;
+  const int32_t* gEnt = a.ent + e0;
+  stage_entries(sEnt, gEnt, n);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -184,7 +191,7 @@ __global__ void __launch_bounds__(192, 1)
         const int st = j % C::STAGES;
         if (j >= C::STAGES && !mbar_wait(bar_kv_empty + st, ((j / C::STAGES) - 1) & 1, abort_flag))
           break;
-        const int e = a.ent[e0 + j];
+        const int e = entry_at(sEnt, gEnt, j);
         const int src = (e >> 1) & 3;
         const int kpos = (e >> 3) * C::TK;
         mbar_arrive_expect_tx(bar_k_full + st, C::KV_BYTES);
@@ -196,44 +203,48 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ S issuer: S_j = Q K_j^T
     if (lane == 0 && n > 0) {
-      // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, C::TK, false, false);
-      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, false, true);
       const uint32_t q_base = smem_u32(sQ);
       bool ok = mbar_wait(bar_q, 0, abort_flag);
-      for (int j = 0; ok && j <= n; ++j) {
-        if (j < n) {
-          const int st = j % C::STAGES;
-          const int sb = j & 1;
-          ok = mbar_wait(bar_k_full + st, (j / C::STAGES) & 1, abort_flag);
-          if (ok && j >= 2) ok = mbar_wait(bar_s_empty + sb, ((j >> 1) - 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(sK + st * C::KV_BYTES);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % C::STAGES;
+        const int sb = j & 1;
+        ok = mbar_wait(bar_k_full + st, (j / C::STAGES) & 1, abort_flag);
+        if (ok && j >= 2) ok = mbar_wait(bar_s_empty + sb, ((j >> 1) - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(sK + st * C::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16_ss(tmem + sb * C::TK, kmajor_desc<D>(q_base, C::TQ, kk),
-                        kmajor_desc<D>(k_base, C::TK, kk), idesc_qk, kk > 0);
-          mma_commit(bar_s_full + sb);
-        }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int st = jj % C::STAGES;
-          const int pb = jj & 1;
-          ok = mbar_wait(bar_p_full + pb, (jj >> 1) & 1, abort_flag) &&
-               mbar_wait(bar_v_full + st, (jj / C::STAGES) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t p_base = smem_u32(sP + pb * C::P_BYTES);
-          const uint32_t v_base = smem_u32(sV + st * C::KV_BYTES);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem + sb * C::TK, kmajor_desc<D>(q_base, C::TQ, kk), kmajor_desc<D>(k_base, C::TK, kk),
+                      idesc_qk, kk > 0);
+        mma_commit(bar_s_full + sb);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ PV issuer: O += P_j V_j
+    // S_j has completed before P_j exists, so this thread's commit after PV_j
+    // also releases the K half of the stage.
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, false, true);
+      bool ok = true;
+      for (int jj = 0; ok && jj < n; ++jj) {
+        const int st = jj % C::STAGES;
+        const int pb = jj & 1;
+        ok = mbar_wait(bar_p_full + pb, (jj >> 1) & 1, abort_flag) &&
+             mbar_wait(bar_v_full + st, (jj / C::STAGES) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t p_base = smem_u32(sP + pb * C::P_BYTES);
+        const uint32_t v_base = smem_u32(sV + st * C::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::TK / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_O, make_desc(p_base + kk * 32, 16, 1024, kSwizzle128),
-                        mnmajor_desc<D>(v_base, C::TK, kk), idesc_pv, (jj > 0 || kk > 0));
-          mma_commit(bar_pv_done + pb);
-          mma_commit(bar_kv_empty + st);
-        }
+        for (int kk = 0; kk < C::TK / 16; ++kk)
+          mma_bf16_ss(tmem + C::COL_O, make_desc(p_base + kk * 32, 16, 1024, kSwizzle128),
+                      mnmajor_desc<D>(v_base, C::TK, kk), idesc_pv, (jj > 0 || kk > 0));
+        mma_commit(bar_pv_done + pb);
+        mma_commit(bar_kv_empty + st);
       }
     }
   } else {
@@ -271,7 +282,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(bar_s_empty + sb);
 
-      const int e = a.ent[e0 + j];
+      const int e = entry_at(sEnt, gEnt, j);
       if (e & 1) {
         const int src = (e >> 1) & 3;
         const int k0 = (e >> 3) * C::TK;
@@ -283,9 +294,16 @@ __global__ void __launch_bounds__(192, 1)
           if (key < lo || key > hi) s[i] = -INFINITY;
         }
       }
-      float mx = -INFINITY;
+      // row max as a tree (short dependency chains)
+      float mx8[8];
 #pragma unroll
-      for (int i = 0; i < C::TK; ++i) mx = fmaxf(mx, s[i]);
+      for (int u = 0; u < 8; ++u) mx8[u] = s[u];
+#pragma unroll
+      for (int i = 8; i < C::TK; i += 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], s[i + u]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * a.scale_log2;
       float factor = 1.f;
       if (m_tile > m_used + 8.f) {
@@ -311,7 +329,7 @@ __global__ void __launch_bounds__(192, 1)
       // P buffer j&1 is free once PV of tile j-2 has completed.
       if (j >= 2) ok = ok && mbar_wait(bar_pv_done + sb, ((j >> 1) - 1) & 1, abort_flag);
       const float neg = (m_used == -INFINITY) ? 0.f : -m_used;
-      float rsum = 0.f;
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // partial row sums
       uint8_t* pbuf = sP + sb * C::P_BYTES;
 #pragma unroll
       for (int ch = 0; ch < C::TK / 8; ++ch) {
@@ -319,7 +337,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           p[u] = ex2(fmaf(s[ch * 8 + u], a.scale_log2, neg));
-          rsum += p[u];
+          rs8[u] += p[u];
         }
         uint4 w;
         w.x = pack_bf16(p[0], p[1]);
@@ -328,6 +346,7 @@ __global__ void __launch_bounds__(192, 1)
         w.w = pack_bf16(p[6], p[7]);
         *reinterpret_cast<uint4*>(pbuf + sw128_offset(row, ch)) = w;
       }
+      const float rsum = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l_sum = l_sum * factor + rsum;
       fence_proxy_async_smem();
       tc_fence_before();
