@@ -185,13 +185,17 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
     }
   const TileTable* tabs[4] = {&L->fwd_main, &L->fwd_col, &L->bwd_main, &L->bwd_sec};
   std::vector<int32_t> blob;
-  size_t offs[4][3];
+  size_t offs[4][4];
   for (int t = 0; t < 4; ++t) {
     const TileTable& tt = *tabs[t];
+    offs[t][3] = blob.size();  // 16-byte aligned: every section is padded to 4 ints
+    blob.insert(blob.end(), tt.sched.begin(), tt.sched.end());
     offs[t][0] = blob.size();
     blob.insert(blob.end(), tt.row_ptr.begin(), tt.row_ptr.end());
+    while (blob.size() % 4) blob.push_back(0);
     offs[t][1] = blob.size();
     blob.insert(blob.end(), tt.ent.begin(), tt.ent.end());
+    while (blob.size() % 4) blob.push_back(0);
     offs[t][2] = blob.size();
     blob.insert(blob.end(), tt.order.begin(), tt.order.end());
     while (blob.size() % 4) blob.push_back(0);
@@ -212,6 +216,7 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
     dts[t]->row_ptr = base + offs[t][0];
     dts[t]->ent = base + offs[t][1];
     dts[t]->order = base + offs[t][2];
+    dts[t]->sched = base + offs[t][3];
     dts[t]->n_rows = tabs[t]->n_rows;
     dts[t]->nnz = static_cast<int>(tabs[t]->ent.size());
   }
@@ -308,6 +313,12 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 struct WsLayout {
   size_t ld_nat, ld_col, dq, dk, dv, total;
   int n_pad;
@@ -321,7 +332,7 @@ WsLayout ws_layout(int B, int H, int N, int D, const sa_layout* L) {
   const size_t rows = BH * N;
   WsLayout w;
   w.n_pad = (N + BwdCfg<64>::TQ - 1) / BwdCfg<64>::TQ * BwdCfg<64>::TQ;
-  const size_t ld_bytes = align256(BH * w.n_pad * 8);
+  const size_t ld_bytes = align256(BH * w.n_pad * 8);  // two floats per query position
   w.ld_nat = 0;
   w.ld_col = ld_bytes;
   const bool col = L->pattern == SA_STRIDED;
@@ -356,8 +367,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = set_smem(kern, BwdCfg<D>::SMEM))) return st;
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  float2* ld_nat = reinterpret_cast<float2*>(wsb + w.ld_nat);
-  float2* ld_col = (L->pattern == SA_STRIDED) ? reinterpret_cast<float2*>(wsb + w.ld_col) : nullptr;
+  float* ld_nat = reinterpret_cast<float*>(wsb + w.ld_nat);
+  float* ld_col = (L->pattern == SA_STRIDED) ? reinterpret_cast<float*>(wsb + w.ld_col) : nullptr;
   float* dq_acc = reinterpret_cast<float*>(wsb + w.dq);
   float* dk_part = reinterpret_cast<float*>(wsb + w.dk);
   float* dv_part = reinterpret_cast<float*>(wsb + w.dv);
@@ -387,26 +398,30 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   const bool sec = (L->pattern == SA_STRIDED || L->pattern == SA_FIXED) && dc.bwd_sec.n_rows > 0;
+  a.BH = g.BH;
+  const int n_sm = sm_count();
   if (sec) {
-    a.row_ptr = dc.bwd_sec.row_ptr;
+    a.sched = dc.bwd_sec.sched;
     a.ent = dc.bwd_sec.ent;
-    a.order = dc.bwd_sec.order;
+    a.n_slots = dc.bwd_sec.n_rows;
     a.key_view = (L->pattern == SA_STRIDED) ? SRC_T : SRC_S;
     a.add_part = 0;
-    dim3 grid(g.BH, dc.bwd_sec.n_rows);
+    const long long items = static_cast<long long>(a.n_slots) * g.BH;
+    dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
     st = launch(K_BWD_SEC * 4 + L->pattern, s, [&] {
       kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                                                mv.col, mv.sum, a);
     });
     if (st) return st;
   }
-  a.row_ptr = dc.bwd_main.row_ptr;
+  a.sched = dc.bwd_main.sched;
   a.ent = dc.bwd_main.ent;
-  a.order = dc.bwd_main.order;
+  a.n_slots = dc.bwd_main.n_rows;
   a.key_view = SRC_N;
   a.add_part = sec ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
   {
-    dim3 grid(g.BH, dc.bwd_main.n_rows);
+    const long long items = static_cast<long long>(a.n_slots) * g.BH;
+    dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
     st = launch(K_BWD_MAIN * 4 + L->pattern, s, [&] {
       kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                                                mv.col, mv.sum, a);

@@ -7,24 +7,25 @@
 //   P = exp(S - lse), dV = P^T dO, dP = dO V^T, dS = P (dP - Delta),
 //   dK = s dS^T Q, dQ = s dS K.
 //
-// sa_bwd_kernel: one CTA = one 128-key tile of one (batch, head), in the
-// view order of its table; it walks the 64-query steps that see it.  Per
-// step j:
-//   ST_j  = K Q_j^T, dPT_j = V dO_j^T  (keys on TMEM lanes, 64 columns each,
-//                                       double-buffered so step j+1's products
-//                                       overlap step j's elementwise work)
-//   P^T_j (bf16, smem), dS^T_j (bf16, smem) by the elementwise warps
-//   dV += P^T_j dO_j,  dK += dS^T_j Q_j   (TMEM accumulators for the CTA)
-//   every second step: dQ = dS_pair K for the two steps' 128 queries
-//                      (M = 128), read by the dQ warps and added to an fp32
-//                      workspace with vector reductions.
+// sa_bwd_kernel is persistent: one CTA per SM walks a fixed zig-zag share of
+// the (key tile, batch*head) items of its table (longest tiles first), each
+// item a 128-key tile in the view order of the table and the 64-query steps
+// that see it.  Per step (global step counter g, continued across items):
+//   ST_g  = K Q^T, dPT_g = V dO^T  (keys on TMEM lanes, 64 columns each,
+//                                   double-buffered)
+//   P^T_g, dS^T_g in bf16 smem     (elementwise warps)
+//   dV += P^T dO, dK += dS^T Q     (TMEM accumulators of the item)
+//   dQ = dS K for the 128 queries of the global step pair (g even, g odd),
+//   restricted to the item's own steps, then reduced into an fp32 workspace.
+// K/V are double-buffered so the next item's tiles load during this one, and
+// the dV/dK epilogue of an item runs in the dQ warps while the next item's
+// steps proceed.
 // Roles (480 threads): warp 0 producer (TMA for K, V, Q, dO; bulk copy of
 // the packed lse/Delta), warp 1 TMEM allocation and lane 0 issue of ST/dPT,
-// warps 2..9 elementwise (two groups of four, one warp per TMEM lane quarter
-// each, taking alternate steps), warps 10..13 dQ reduction, warp 14 lane 0 issue of dV/dK/dQ.  Two
-// issuing threads keep the S products of later steps flowing while dV/dK/dQ
-// of earlier steps wait on the elementwise warps.  Warp w may only touch TMEM lanes
-// 32*(w%4)..32*(w%4)+31, so every role picks its rows by w%4.
+// warps 2..9 elementwise (two groups of four taking alternate global steps,
+// one warp per TMEM lane quarter each), warps 10..13 dQ reduction and the
+// dV/dK epilogue, warp 14 lane 0 issue of dV/dK/dQ.  Warp w may only touch
+// TMEM lanes 32*(w%4)..32*(w%4)+31, so every role picks its rows by w%4.
 // TMEM columns (NBUF = 2 for D <= 64, 1 for D = 128):
 //   ST[b] = b*64, dPT[b] = NBUF*64 + b*64, dV = 2*NBUF*64, dK = dV + D,
 //   dQ[b] = dK + D + b*D (two dQ buffers for D <= 64, one for D = 128).
@@ -36,12 +37,15 @@
 namespace sa {
 
 struct BwdArgs {
-  const int32_t* row_ptr;
+  const int32_t* sched;  // per launch slot: {tile, first entry, count, 0}
   const int32_t* ent;
-  const int32_t* order;
-  const float2* ld_nat;  // [BH, n_pad] (lse * log2(e), Delta) in natural query order
-  const float2* ld_col;  // [BH, n_pad] the same in column-major order (strided)
+  // Per 64-query step of view positions: 64 floats -lse*log2(e), then 64
+  // floats -Delta ([BH][n_pad/64][2][64]), natural query order / column-major
+  // order (strided).  Padding positions hold (-inf, 0).
+  const float* ld_nat;
+  const float* ld_col;
   int n_pad;             // N rounded up to the 64-query step, padded with (+inf, 0)
+  int n_slots, BH;       // items = n_slots * BH, slot-major (all heads of a slot together)
   float* dq_acc;         // [BH, N, D] fp32, scaled
   __nv_bfloat16* dk;     // final outputs (main pass)
   __nv_bfloat16* dv;
@@ -59,10 +63,13 @@ template <int D>
 struct BwdCfg {
   static constexpr int TK = 128, TQ = 64;
   static constexpr int NBUF = (D >= 128) ? 1 : 2;      // ST/dPT buffers in TMEM
-  // Q/dO ring.  At least 2: the MMA issuer asks for step j's Q/dO before it
-  // releases step j-1's (it issues S_j ahead of dV/dK of step j-1).
-  static constexpr int STAGES = (D >= 128) ? 2 : 4;
+  // Q/dO ring (>= 2: see the S issuer).  A stage is held from its load
+  // until dK of its step is done, which trails the S products by about two
+  // steps, so the ring must be deep for the loads to run ahead.
+  static constexpr int STAGES = (D >= 128) ? 2 : 3;
+  static constexpr int KVB = (D >= 128) ? 1 : 2;       // K/V buffers (next item's tiles load early)
   static constexpr int DST_BUFS = (D >= 128) ? 1 : 2;  // dS^T pair buffers
+  static constexpr int DQBUF = (D >= 128) ? 1 : 2;     // dQ TMEM buffers
   static constexpr int ROWB = (D >= 64) ? 128 : 64;
   static constexpr uint64_t SWZ = (D >= 64) ? kSwizzle128 : kSwizzle64;
   static constexpr int SBO = 8 * ROWB;
@@ -70,18 +77,16 @@ struct BwdCfg {
   static constexpr int QS_BYTES = TQ * D * 2;          // 64-query tile
   static constexpr int PT_BYTES = TK * TQ * 2;         // [128 keys][64 queries] bf16 = 16 KiB
   static constexpr int DST_BYTES = 2 * PT_BYTES;       // a pair of steps (2 panels)
+  static constexpr int LD_BYTES = TQ * 8;
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_Q = OFF_V + KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KVB * KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KVB * KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + STAGES * QS_BYTES;
   static constexpr int OFF_PT = OFF_DO + STAGES * QS_BYTES;
   static constexpr int OFF_DST = OFF_PT + 2 * PT_BYTES;
-  static constexpr int OFF_LD = OFF_DST + DST_BUFS * DST_BYTES;  // float2 [STAGES][64]
-  static constexpr int LD_BYTES = TQ * 8;
-  static constexpr int OFF_ENT = OFF_LD + STAGES * LD_BYTES;
-  static constexpr int OFF_BAR = OFF_ENT + kMaxStagedEnt * 4;
-  static constexpr int DQBUF = (D >= 128) ? 1 : 2;       // dQ TMEM buffers
-  static constexpr int N_BARS = 1 + 2 * STAGES + 2 * 2 + 2 * 2 + 2 + DST_BUFS + 2 * DQBUF + 1;
+  static constexpr int OFF_LD = OFF_DST + DST_BUFS * DST_BYTES;  // float [STAGES][2][64]
+  static constexpr int OFF_BAR = OFF_LD + STAGES * LD_BYTES;
+  static constexpr int N_BARS = 2 * KVB + 2 * STAGES + 2 * 5 + DST_BUFS + 2 * DQBUF + 2;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
@@ -91,7 +96,7 @@ struct BwdCfg {
   static constexpr int COL_DQ = COL_DK + D;
   static constexpr int THREADS = 480;
   static_assert(COL_DQ + DQBUF * D <= TMEM_COLS, "TMEM budget");
-  static_assert(STAGES >= 2, "the software-pipelined MMA loop needs two Q/dO stages");
+  static_assert(STAGES >= 2, "the S issuer needs step j's Q/dO while step j-1's is still in use");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -117,6 +122,90 @@ __device__ __forceinline__ uint64_t pair_mndesc(uint32_t base, int kk) {
   return make_desc(base + kk * 2048, 16384, 1024, kSwizzle128);
 }
 
+// Item k of this CTA in the zig-zag share: rounds alternate direction so
+// that long and short tiles pair up (the slots are sorted longest first).
+__device__ __forceinline__ int zigzag_item(int k, int cta, int n_ctas) {
+  return k * n_ctas + ((k & 1) ? (n_ctas - 1 - cta) : cta);
+}
+
+struct BwdItem {
+  int bh, kt, e0, n;
+};
+
+__device__ __forceinline__ BwdItem bwd_item(const BwdArgs& a, int item) {
+  const int slot = item / a.BH;
+  const int4 sc = *reinterpret_cast<const int4*>(a.sched + 4 * slot);
+  return BwdItem{item - slot * a.BH, sc.x, sc.y, sc.z};
+}
+
+// Key-row facts of an elementwise / epilogue thread for key tile kt.
+struct KeyRow {
+  int y, knat, qlo, qhi;
+  bool kvalid;
+};
+
+template <int D>
+__device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
+  KeyRow k;
+  k.y = kt * BwdCfg<D>::TK + row;
+  const int nkeys = (a.key_view == SRC_S) ? a.R * a.c : a.N;
+  k.kvalid = k.y < nkeys;
+  if (a.key_view == SRC_T) k.knat = (k.y % a.R) * a.l + k.y / a.R;
+  else if (a.key_view == SRC_S) k.knat = (k.y / a.c) * a.l + (a.l - a.c) + k.y % a.c;
+  else k.knat = k.y;
+  if (a.key_view == SRC_T) {
+    k.qlo = k.y + 1;
+    k.qhi = (k.y / a.R) * a.R + a.R - 1;
+  } else if (a.key_view == SRC_S) {
+    k.qlo = (k.y / a.c + 1) * a.l;
+    k.qhi = a.N - 1;
+  } else {
+    k.qlo = k.y;
+    if (a.pattern == SA_ALL) k.qhi = a.N - 1;
+    else if (a.pattern == SA_FIXED) k.qhi = (k.y / a.l) * a.l + a.l - 1;
+    else k.qhi = k.y + a.l - 1;
+  }
+  if (k.qhi > a.N - 1) k.qhi = a.N - 1;
+  if (!k.kvalid) k.qhi = k.qlo - 1;
+  return k;
+}
+
+// dV / dK rows of one key for columns [c0, c0 + NC): add the secondary
+// partial (natural pass) and store bf16, or store the fp32 partial
+// (secondary pass).  g holds NC fp32 values, already scaled.
+template <int D, int NC>
+__device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size_t off, int c0, float* g,
+                                               bool add) {
+  if (a.key_view != SRC_N) {
+    float* dstp = (which ? a.dk_part : a.dv_part) + off + c0;
+#pragma unroll
+    for (int u = 0; u < NC; u += 4)
+      *reinterpret_cast<float4*>(dstp + u) = make_float4(g[u], g[u + 1], g[u + 2], g[u + 3]);
+    return;
+  }
+  if (add) {
+    const float* srcp = (which ? a.dk_part : a.dv_part) + off + c0;
+#pragma unroll
+    for (int u = 0; u < NC; u += 4) {
+      const float4 t = *reinterpret_cast<const float4*>(srcp + u);
+      g[u] += t.x;
+      g[u + 1] += t.y;
+      g[u + 2] += t.z;
+      g[u + 3] += t.w;
+    }
+  }
+  uint4* dstp = reinterpret_cast<uint4*>((which ? a.dk : a.dv) + off + c0);
+#pragma unroll
+  for (int u = 0; u < NC; u += 8) {
+    uint4 w;
+    w.x = pack_bf16(g[u], g[u + 1]);
+    w.y = pack_bf16(g[u + 2], g[u + 3]);
+    w.z = pack_bf16(g[u + 4], g[u + 5]);
+    w.w = pack_bf16(g[u + 6], g[u + 7]);
+    dstp[u / 8] = w;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(480, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
@@ -134,39 +223,38 @@ __global__ void __launch_bounds__(480, 1)
   uint8_t* sDO = smem + C::OFF_DO;
   uint8_t* sPT = smem + C::OFF_PT;
   uint8_t* sDST = smem + C::OFF_DST;
-  float2* sLD = reinterpret_cast<float2*>(smem + C::OFF_LD);
-  int32_t* sEnt = reinterpret_cast<int32_t*>(smem + C::OFF_ENT);
+  float* sLD = reinterpret_cast<float*>(smem + C::OFF_LD);  // [STAGES][2][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* bar_kv = bars;
-  uint64_t* bar_qdo_full = bar_kv + 1;                 // [STAGES]
-  uint64_t* bar_qdo_empty = bar_qdo_full + C::STAGES;  // [STAGES]
-  // s_full / s_free are indexed by step parity (one per elementwise group),
-  // not by TMEM buffer: with a single buffer the two groups alternate on it,
-  // and a shared barrier could be waited on two phases ahead.
-  uint64_t* bar_s_full = bar_qdo_empty + C::STAGES;    // [2]  ST and dPT of a step
-  uint64_t* bar_s_free = bar_s_full + 2;               // [2]  elementwise done reading them
-  uint64_t* bar_pt_full = bar_s_free + 2;              // [2]
-  uint64_t* bar_pt_free = bar_pt_full + 2;             // [2]
-  uint64_t* bar_dst_full = bar_pt_free + 2;            // [2]  per step parity
-  uint64_t* bar_dst_free = bar_dst_full + 2;           // [DST_BUFS] per pair
-  uint64_t* bar_dq_full = bar_dst_free + C::DST_BUFS;  // [DQBUF]
-  uint64_t* bar_dq_free = bar_dq_full + C::DQBUF;      // [DQBUF]
-  uint64_t* bar_dkv_full = bar_dq_free + C::DQBUF;
+  uint64_t* bar_kv_full = bars;                          // [KVB]
+  uint64_t* bar_kv_empty = bar_kv_full + C::KVB;         // [KVB]
+  uint64_t* bar_qdo_full = bar_kv_empty + C::KVB;        // [STAGES]
+  uint64_t* bar_qdo_empty = bar_qdo_full + C::STAGES;    // [STAGES]
+  // Per global-step-parity barriers (one per elementwise group), so that a
+  // barrier is never waited on two phases ahead.
+  uint64_t* bar_s_full = bar_qdo_empty + C::STAGES;      // [2]  ST and dPT of a step
+  uint64_t* bar_s_free = bar_s_full + 2;                 // [2]  elementwise done reading them
+  uint64_t* bar_pt_full = bar_s_free + 2;                // [2]
+  uint64_t* bar_pt_free = bar_pt_full + 2;               // [2]
+  uint64_t* bar_dst_full = bar_pt_free + 2;              // [2]
+  uint64_t* bar_dst_free = bar_dst_full + 2;             // [DST_BUFS] per global pair
+  uint64_t* bar_dq_full = bar_dst_free + C::DST_BUFS;    // [DQBUF] per dQ product
+  uint64_t* bar_dq_free = bar_dq_full + C::DQBUF;        // [DQBUF]
+  uint64_t* bar_dkv_full = bar_dq_free + C::DQBUF;       // per non-empty item
+  uint64_t* bar_dkv_free = bar_dkv_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
-  const int bh = blockIdx.x;  // all heads of the longest tiles first (longest-first balance)
-  const int kt = a.order[blockIdx.y];
-  const int e0 = a.row_ptr[kt];
-  const int n = a.row_ptr[kt + 1] - e0;  // 64-query steps
-  const int32_t* gEnt = a.ent + e0;
-  stage_entries(sEnt, gEnt, n);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int q_src = (a.key_view == SRC_T) ? SRC_T : SRC_N;
+  const int n_items = a.n_slots * a.BH;
+  const int cta = blockIdx.x, n_ctas = gridDim.x;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_kv, 1);
+    for (int b = 0; b < C::KVB; ++b) {
+      mbar_init(bar_kv_full + b, 1);
+      mbar_init(bar_kv_empty + b, 1);
+    }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(bar_qdo_full + s, 1);
       mbar_init(bar_qdo_empty + s, 1);
@@ -174,8 +262,6 @@ __global__ void __launch_bounds__(480, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_s_full + b, 1);
       mbar_init(bar_s_free + b, 128);
-    }
-    for (int b = 0; b < 2; ++b) {
       mbar_init(bar_pt_full + b, 128);
       mbar_init(bar_pt_free + b, 1);
       mbar_init(bar_dst_full + b, 128);
@@ -186,6 +272,7 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(bar_dq_free + b, 128);
     }
     mbar_init(bar_dkv_full, 1);
+    mbar_init(bar_dkv_free, 128);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -197,306 +284,342 @@ __global__ void __launch_bounds__(480, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (n > 0) {
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar_kv, 2 * C::KV_BYTES);
-        load_rows<D>(sK, a.key_view, kt * C::TK, C::TK, bh, &mk_nat, &mk_col, &mk_sum, bar_kv, a.R, a.l, a.c);
-        load_rows<D>(sV, a.key_view, kt * C::TK, C::TK, bh, &mv_nat, &mv_col, &mv_sum, bar_kv, a.R, a.l, a.c);
-      }
-      if (lane == 0) {
-        const float2* ld = (q_src == SRC_T ? a.ld_col : a.ld_nat) + static_cast<size_t>(bh) * a.n_pad;
-        for (int j = 0; j < n; ++j) {
-          const int st = j % C::STAGES;
-          if (j >= C::STAGES && !mbar_wait(bar_qdo_empty + st, ((j / C::STAGES) - 1) & 1, abort_flag)) break;
-          const int qpos = (entry_at(sEnt, gEnt, j) >> 3) * C::TQ;
+    if (lane == 0) {
+      bool ok = true;
+      int gs = 0, ne = 0;
+      BwdItem nxt = (cta < n_items) ? bwd_item(a, cta) : BwdItem{0, 0, 0, 0};
+      for (int k = 0, item = cta; ok && item < n_items;) {
+        const BwdItem it = nxt;
+        item = zigzag_item(++k, cta, n_ctas);
+        if (item < n_items) nxt = bwd_item(a, item);
+        if (it.n == 0) continue;
+        const int kb = ne % C::KVB;
+        if (ne >= C::KVB && !mbar_wait(bar_kv_empty + kb, ((ne / C::KVB) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar_kv_full + kb, 2 * C::KV_BYTES);
+        load_rows<D>(sK + kb * C::KV_BYTES, a.key_view, it.kt * C::TK, C::TK, it.bh, &mk_nat, &mk_col, &mk_sum,
+                     bar_kv_full + kb, a.R, a.l, a.c);
+        load_rows<D>(sV + kb * C::KV_BYTES, a.key_view, it.kt * C::TK, C::TK, it.bh, &mv_nat, &mv_col, &mv_sum,
+                     bar_kv_full + kb, a.R, a.l, a.c);
+        const float* ld = (q_src == SRC_T ? a.ld_col : a.ld_nat) + static_cast<size_t>(it.bh) * a.n_pad * 2;
+        int e_next = a.ent[it.e0];
+        for (int j = 0; j < it.n; ++j) {
+          const int g = gs + j;
+          const int st = g % C::STAGES;
+          const int e = e_next;
+          if (j + 1 < it.n) e_next = a.ent[it.e0 + j + 1];
+          if (g >= C::STAGES && !mbar_wait(bar_qdo_empty + st, ((g / C::STAGES) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int qpos = (e >> 3) * C::TQ;
           mbar_arrive_expect_tx(bar_qdo_full + st, 2 * C::QS_BYTES + C::LD_BYTES);
-          load_rows<D>(sQ + st * C::QS_BYTES, q_src, qpos, C::TQ, bh, &mq_nat, &mq_col, &mq_col,
+          load_rows<D>(sQ + st * C::QS_BYTES, q_src, qpos, C::TQ, it.bh, &mq_nat, &mq_col, &mq_col,
                        bar_qdo_full + st, a.R, a.l, a.c);
-          load_rows<D>(sDO + st * C::QS_BYTES, q_src, qpos, C::TQ, bh, &mdo_nat, &mdo_col, &mdo_col,
+          load_rows<D>(sDO + st * C::QS_BYTES, q_src, qpos, C::TQ, it.bh, &mdo_nat, &mdo_col, &mdo_col,
                        bar_qdo_full + st, a.R, a.l, a.c);
-          bulk_load(sLD + st * C::TQ, ld + qpos, C::LD_BYTES, bar_qdo_full + st);
+          bulk_load(sLD + st * 2 * C::TQ, ld + 2 * qpos, C::LD_BYTES, bar_qdo_full + st);
         }
+        gs += it.n;
+        ++ne;
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ S issuer: ST_j, dPT_j
-    // Runs up to NBUF steps ahead of the elementwise warps; only waits for
-    // the step's Q/dO and for its TMEM buffer to be read out.
-    if (lane == 0 && n > 0) {
+    // ------------------------------------------------------------ S issuer: ST_g, dPT_g
+    // Runs up to NBUF steps ahead of the elementwise warps; waits only for a
+    // step's Q/dO and for its TMEM buffer to have been read out.
+    if (lane == 0) {
       constexpr uint32_t id_s = make_idesc_bf16(128, C::TQ, false, false);  // N = 64 queries
-      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
-      bool ok = mbar_wait(bar_kv, 0, abort_flag);
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % C::STAGES;
-        const int b = j % C::NBUF;
-        ok = mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
-        if (ok && j >= C::NBUF) {  // buffer b was last used by step j - NBUF
-          const int jp = j - C::NBUF;
-          ok = mbar_wait(bar_s_free + (jp & 1), (jp >> 1) & 1, abort_flag);
+      bool ok = true;
+      int gs = 0, ne = 0;
+      BwdItem nxt = (cta < n_items) ? bwd_item(a, cta) : BwdItem{0, 0, 0, 0};
+      for (int k = 0, item = cta; ok && item < n_items;) {
+        const BwdItem it = nxt;  // the next item's schedule entry is fetched one item ahead
+        item = zigzag_item(++k, cta, n_ctas);
+        if (item < n_items) nxt = bwd_item(a, item);
+        if (it.n == 0) continue;
+        const int kb = ne % C::KVB;
+        ok = mbar_wait(bar_kv_full + kb, (ne / C::KVB) & 1, abort_flag);
+        const uint32_t k_base = smem_u32(sK + kb * C::KV_BYTES), v_base = smem_u32(sV + kb * C::KV_BYTES);
+        for (int j = 0; ok && j < it.n; ++j) {
+          const int g = gs + j;
+          const int st = g % C::STAGES;
+          const int b = g % C::NBUF;
+          ok = mbar_wait(bar_qdo_full + st, (g / C::STAGES) & 1, abort_flag);
+          if (ok && g >= C::NBUF) {  // TMEM buffer b was last used by step g - NBUF
+            const int gp = g - C::NBUF;
+            ok = mbar_wait(bar_s_free + (gp & 1), (gp >> 1) & 1, abort_flag);
+          }
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
+          const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + b * 64, bwd_kdesc<D>(k_base, C::TK, kk), bwd_kdesc<D>(q_base, C::TQ, kk), id_s,
+                        kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_DPT + b * 64, bwd_kdesc<D>(v_base, C::TK, kk),
+                        bwd_kdesc<D>(do_base, C::TQ, kk), id_s, kk > 0);
+          mma_commit(bar_s_full + (g & 1));
         }
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
-        const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + b * 64, bwd_kdesc<D>(k_base, C::TK, kk), bwd_kdesc<D>(q_base, C::TQ, kk), id_s,
-                      kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_DPT + b * 64, bwd_kdesc<D>(v_base, C::TK, kk),
-                      bwd_kdesc<D>(do_base, C::TQ, kk), id_s, kk > 0);
-        mma_commit(bar_s_full + (j & 1));
+        gs += it.n;
+        ++ne;
       }
     }
   } else if (warp == 14) {
     // ------------------------------------------------------------ G issuer: dV, dK, dQ
     // Its commits track only its own MMAs; the S issuer's products of a step
     // are complete before the step's P^T exists, so releasing the Q/dO stage
-    // after dK covers both issuers.
-    if (lane == 0 && n > 0) {
+    // after dK (and the K/V buffer after the item's last dQ) covers both.
+    if (lane == 0) {
       constexpr uint32_t id_kv = make_idesc_bf16(128, D, false, true);  // dV, dK
       constexpr uint32_t id_q = make_idesc_bf16(128, D, true, true);    // dQ (pair)
-      const uint32_t k_base = smem_u32(sK);
-      bool ok = mbar_wait(bar_kv, 0, abort_flag);
-      for (int jj = 0; ok && jj < n; ++jj) {
-        const int st = jj % C::STAGES;
-        const int pb = jj & 1;
-        const int pair = jj >> 1;
-        const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
-        const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
-        const uint32_t dst_pair = smem_u32(sDST + (pair % C::DST_BUFS) * C::DST_BYTES);
-        if (!mbar_wait(bar_pt_full + pb, (jj >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
+      bool ok = true;
+      int gs = 0, ne = 0, qi = 0;
+      BwdItem nxt = (cta < n_items) ? bwd_item(a, cta) : BwdItem{0, 0, 0, 0};
+      for (int k = 0, item = cta; ok && item < n_items;) {
+        const BwdItem it = nxt;  // the next item's schedule entry is fetched one item ahead
+        item = zigzag_item(++k, cta, n_ctas);
+        if (item < n_items) nxt = bwd_item(a, item);
+        if (it.n == 0) continue;
+        const int kb = ne % C::KVB;
+        ok = mbar_wait(bar_kv_full + kb, (ne / C::KVB) & 1, abort_flag);
+        // dV/dK of the previous item must have been read out by the epilogue
+        if (ok && ne >= 1) ok = mbar_wait(bar_dkv_free, (ne - 1) & 1, abort_flag);
+        const uint32_t k_base = smem_u32(sK + kb * C::KV_BYTES);
+        for (int jj = 0; ok && jj < it.n; ++jj) {
+          const int g = gs + jj;
+          const int st = g % C::STAGES;
+          const int pb = g & 1;
+          const int P = g >> 1;
+          const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
+          const uint32_t do_base = smem_u32(sDO + st * C::QS_BYTES);
+          const uint32_t dst_pair = smem_u32(sDST + (P % C::DST_BUFS) * C::DST_BYTES);
+          if (!mbar_wait(bar_pt_full + pb, (g >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < C::TQ / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_DV, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
-                      (jj > 0 || kk > 0));
-        mma_commit(bar_pt_free + pb);
-        if (!mbar_wait(bar_dst_full + pb, (jj >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::TQ / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_DK, pt_kdesc(dst_pair + pb * C::PT_BYTES, kk),
-                      bwd_mndesc<D>(q_base, C::TQ, kk), id_kv, (jj > 0 || kk > 0));
-        mma_commit(bar_qdo_empty + st);
-        if ((jj & 1) || jj == n - 1) {
-          const int qb = pair % C::DQBUF;
-          if (pair >= C::DQBUF && !mbar_wait(bar_dq_free + qb, ((pair / C::DQBUF) - 1) & 1, abort_flag)) break;
+          for (int kk = 0; kk < C::TQ / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_DV, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
+                        (jj > 0 || kk > 0));
+          mma_commit(bar_pt_free + pb);
+          if (!mbar_wait(bar_dst_full + pb, (g >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < C::TK / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_DQ + qb * D, pair_mndesc(dst_pair, kk), bwd_mndesc<D>(k_base, C::TK, kk),
-                        id_q, kk > 0);
-          mma_commit(bar_dq_full + qb);
-          mma_commit(bar_dst_free + (pair % C::DST_BUFS));
+          for (int kk = 0; kk < C::TQ / 16; ++kk)
+            mma_bf16_ss(tmem + C::COL_DK, pt_kdesc(dst_pair + pb * C::PT_BYTES, kk),
+                        bwd_mndesc<D>(q_base, C::TQ, kk), id_kv, (jj > 0 || kk > 0));
+          mma_commit(bar_qdo_empty + st);
+          if ((g & 1) || jj == it.n - 1) {
+            // dQ for the item's steps of global pair P (one or two of them)
+            const int qb = qi % C::DQBUF;
+            if (qi >= C::DQBUF && !mbar_wait(bar_dq_free + qb, ((qi / C::DQBUF) - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < C::TK / 16; ++kk)
+              mma_bf16_ss(tmem + C::COL_DQ + qb * D, pair_mndesc(dst_pair, kk), bwd_mndesc<D>(k_base, C::TK, kk),
+                          id_q, kk > 0);
+            mma_commit(bar_dq_full + qb);
+            // the pair buffer is free once the product covering its odd step is done
+            if (g & 1) mma_commit(bar_dst_free + (P % C::DST_BUFS));
+            ++qi;
+          }
         }
+        mma_commit(bar_dkv_full);
+        mma_commit(bar_kv_empty + kb);
+        gs += it.n;
+        ++ne;
       }
-      mma_commit(bar_dkv_full);
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------ elementwise
+    // Group `half` takes the global steps g with g % 2 == half, each thread a
+    // whole 64-query row in chunks of 16 columns; the two groups run out of
+    // phase, so one group's exp2 (MUFU) work overlaps the other's dS work.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;  // step parity of this group; dV/dK column half in the epilogue
+    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const int y = kt * C::TK + row;  // this thread's key, view order
-    const int nkeys = (a.key_view == SRC_S) ? a.R * a.c : a.N;
-    const bool kvalid = y < nkeys;
-    int knat;
-    if (a.key_view == SRC_T) knat = (y % a.R) * a.l + y / a.R;
-    else if (a.key_view == SRC_S) knat = (y / a.c) * a.l + (a.l - a.c) + y % a.c;
-    else knat = y;
-    // queries (view order) that see this key: [qlo, qhi]
-    int qlo, qhi;
-    if (a.key_view == SRC_T) {
-      qlo = y + 1;
-      qhi = (y / a.R) * a.R + a.R - 1;
-    } else if (a.key_view == SRC_S) {
-      qlo = (y / a.c + 1) * a.l;
-      qhi = a.N - 1;
-    } else {
-      qlo = y;
-      if (a.pattern == SA_ALL) qhi = a.N - 1;
-      else if (a.pattern == SA_FIXED) qhi = (y / a.l) * a.l + a.l - 1;
-      else qhi = y + a.l - 1;
-    }
-    if (qhi > a.N - 1) qhi = a.N - 1;
-    if (!kvalid) qhi = qlo - 1;
-
-    // Group `half` takes the steps j with j % 2 == half, each thread a whole
-    // 64-query row in chunks of 16 columns; the two groups run out of phase,
-    // so one group's exp2 (MUFU) work overlaps the other's dS (ALU) work.
     bool ok = true;
-    for (int j = half; j < n; j += 2) {
-      const int e = entry_at(sEnt, gEnt, j);
-      const int st = j % C::STAGES;
-      const int b = j % C::NBUF;
-      const int pb = j & 1;
-      const int pair = j >> 1;
-      const bool partial = e & 1;
-      const int x0 = (e >> 3) * C::TQ;
-      ok = ok && mbar_wait(bar_qdo_full + st, (j / C::STAGES) & 1, abort_flag);
-      ok = ok && mbar_wait(bar_s_full + pb, (j >> 1) & 1, abort_flag);
-      // P^T buffer pb is free once dV of step j-2 has completed; dS^T pair
-      // buffer once dQ of pair - DST_BUFS has completed.
-      if (j >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((j >> 1) - 1) & 1, abort_flag);
-      if (pair >= C::DST_BUFS)
-        ok = ok && mbar_wait(bar_dst_free + (pair % C::DST_BUFS), ((pair / C::DST_BUFS) - 1) & 1, abort_flag);
-      tc_fence_after();
-      const float4* ld_t = reinterpret_cast<const float4*>(sLD + st * C::TQ);  // (lse*log2 e, Delta) x 2
-      uint8_t* pt = sPT + pb * C::PT_BYTES;
-      uint8_t* dst = sDST + (pair % C::DST_BUFS) * C::DST_BYTES + pb * C::PT_BYTES;
+    int gs = 0;
+    BwdItem nxt = (cta < n_items) ? bwd_item(a, cta) : BwdItem{0, 0, 0, 0};
+    for (int k = 0, item = cta; ok && item < n_items;) {
+      const BwdItem it = nxt;  // the next item's schedule entry is fetched one item ahead
+      item = zigzag_item(++k, cta, n_ctas);
+      if (item < n_items) nxt = bwd_item(a, item);
+      if (it.n == 0) continue;
+      const KeyRow kr = key_row<D>(a, it.kt, row);
+      for (int j = (half - gs) & 1; j < it.n; j += 2) {
+        const int g = gs + j;
+        const int e = a.ent[it.e0 + j];
+        const int st = g % C::STAGES;
+        const int b = g % C::NBUF;
+        const int pb = g & 1;
+        const int P = g >> 1;
+        const bool partial = e & 1;
+        const int x0 = (e >> 3) * C::TQ;
+        ok = ok && mbar_wait(bar_qdo_full + st, (g / C::STAGES) & 1, abort_flag);
+        ok = ok && mbar_wait(bar_s_full + pb, (g >> 1) & 1, abort_flag);
+        // P^T buffer pb is free once dV of step g-2 has completed; the dS^T
+        // pair buffer once the product over pair P - DST_BUFS has.
+        if (g >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((g >> 1) - 1) & 1, abort_flag);
+        if (P >= C::DST_BUFS)
+          ok = ok && mbar_wait(bar_dst_free + (P % C::DST_BUFS), ((P / C::DST_BUFS) - 1) & 1, abort_flag);
+        tc_fence_after();
+        const float4* nlse4 = reinterpret_cast<const float4*>(sLD + st * 2 * C::TQ);      // -lse*log2 e
+        const float4* ndel4 = reinterpret_cast<const float4*>(sLD + st * 2 * C::TQ + C::TQ);  // -Delta
+        uint8_t* pt = sPT + pb * C::PT_BYTES;
+        uint8_t* dst = sDST + (P % C::DST_BUFS) * C::DST_BYTES + pb * C::PT_BYTES;
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+        // (1) the whole S^T row of this key: one TMEM round trip, then 64
+        //     independent exp2 back to back (keeps the MUFU pipe busy)
+        float sv[64];
 #pragma unroll
-      for (int c16 = 0; c16 < 4; ++c16) {
-        float p[16], dp[16];
-        tmem_ld16(tmem + lane_base + b * 64 + c16 * 16, p);
-        tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + c16 * 16, dp);
+        for (int c16 = 0; c16 < 4; ++c16) tmem_ld16(tmem + lane_base + b * 64 + c16 * 16, sv + c16 * 16);
         tmem_wait_ld();
-        if (c16 == 3) {  // both TMEM buffers of this step have been read
-          tc_fence_before();
-          mbar_arrive(bar_s_free + pb);
-        }
-        float lse2[16], dl[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 t = ld_t[c16 * 8 + i];
-          lse2[2 * i] = t.x;
-          dl[2 * i] = t.y;
-          lse2[2 * i + 1] = t.z;
-          dl[2 * i + 1] = t.w;
-        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float v = ex2(fmaf(p[i], a.scale_log2, -lse2[i]));
-          if (partial) {
-            const int x = x0 + c16 * 16 + i;
-            if (x < qlo || x > qhi) v = 0.f;
+          const float4 t = nlse4[i];
+          const float2 x01 = f2_unpack(f2_fma(f2_pack(sv[4 * i], sv[4 * i + 1]), sc2, f2_pack(t.x, t.y)));
+          const float2 x23 = f2_unpack(f2_fma(f2_pack(sv[4 * i + 2], sv[4 * i + 3]), sc2, f2_pack(t.z, t.w)));
+          sv[4 * i] = ex2(x01.x);
+          sv[4 * i + 1] = ex2(x01.y);
+          sv[4 * i + 2] = ex2(x23.x);
+          sv[4 * i + 3] = ex2(x23.y);
+        }
+        if (partial) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int x = x0 + i;
+            if (x < kr.qlo || x > kr.qhi) sv[i] = 0.f;
           }
-          p[i] = v;
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint4 w;
-          w.x = pack_bf16(p[h * 8 + 0], p[h * 8 + 1]);
-          w.y = pack_bf16(p[h * 8 + 2], p[h * 8 + 3]);
-          w.z = pack_bf16(p[h * 8 + 4], p[h * 8 + 5]);
-          w.w = pack_bf16(p[h * 8 + 6], p[h * 8 + 7]);
-          *reinterpret_cast<uint4*>(pt + sw128_offset(row, c16 * 2 + h)) = w;
-        }
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(pt + sw128_offset(row, ch)) =
+              make_uint4(pack_bf16(sv[8 * ch], sv[8 * ch + 1]), pack_bf16(sv[8 * ch + 2], sv[8 * ch + 3]),
+                         pack_bf16(sv[8 * ch + 4], sv[8 * ch + 5]), pack_bf16(sv[8 * ch + 6], sv[8 * ch + 7]));
+        // (2) dP^T row in two halves (both TMEM buffers of the step are
+        //     released after the second); dS = P (dP - Delta) in fp32 pairs
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float d8[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) d8[u] = p[h * 8 + u] * (dp[h * 8 + u] - dl[h * 8 + u]);
-          uint4 w;
-          w.x = pack_bf16(d8[0], d8[1]);
-          w.y = pack_bf16(d8[2], d8[3]);
-          w.z = pack_bf16(d8[4], d8[5]);
-          w.w = pack_bf16(d8[6], d8[7]);
-          *reinterpret_cast<uint4*>(dst + sw128_offset(row, c16 * 2 + h)) = w;
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar_pt_full + pb);
-      mbar_arrive(bar_dst_full + pb);
-    }
-
-    // ------------------------------------------------------------ epilogue (dV, dK)
-    if (n > 0) {
-      ok = ok && mbar_wait(bar_dkv_full, 0, abort_flag);
-      tc_fence_after();
-    }
-    const size_t off = (static_cast<size_t>(bh) * a.N + (kvalid ? knat : 0)) * D;
-    bool add = false;
-    if (a.add_part == 1) add = true;
-    else if (a.add_part == 2) add = (knat % a.l) >= (a.l - a.c);
-    constexpr int HC = D / 2;  // columns per half
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
-      const uint32_t col = (which ? C::COL_DK : C::COL_DV) + half * HC;
-      const float mul = which ? a.scale : 1.f;
-#pragma unroll
-      for (int i = 0; i < HC / 16; ++i) {
-        float g[16];
-        if (n > 0) {
-          tmem_ld16(tmem + lane_base + col + i * 16, g);
+        for (int hh = 0; hh < 2; ++hh) {
+          float dp[32];
+          tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + hh * 32, dp);
+          tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + hh * 32 + 16, dp + 16);
           tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int u = 0; u < 16; ++u) g[u] = 0.f;
-        }
-        if (!kvalid) continue;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) g[u] *= mul;
-        const size_t eo = off + half * HC + i * 16;
-        if (a.key_view != SRC_N) {
-          float* dstp = (which ? a.dk_part : a.dv_part) + eo;
-#pragma unroll
-          for (int u = 0; u < 16; u += 4)
-            *reinterpret_cast<float4*>(dstp + u) = make_float4(g[u], g[u + 1], g[u + 2], g[u + 3]);
-        } else {
-          if (add) {
-            const float* srcp = (which ? a.dk_part : a.dv_part) + eo;
-#pragma unroll
-            for (int u = 0; u < 16; u += 4) {
-              const float4 t = *reinterpret_cast<const float4*>(srcp + u);
-              g[u] += t.x;
-              g[u + 1] += t.y;
-              g[u + 2] += t.z;
-              g[u + 3] += t.w;
-            }
+          if (hh == 1) {
+            tc_fence_before();
+            mbar_arrive(bar_s_free + pb);
           }
-          uint4 w0, w1;
-          w0.x = pack_bf16(g[0], g[1]);
-          w0.y = pack_bf16(g[2], g[3]);
-          w0.z = pack_bf16(g[4], g[5]);
-          w0.w = pack_bf16(g[6], g[7]);
-          w1.x = pack_bf16(g[8], g[9]);
-          w1.y = pack_bf16(g[10], g[11]);
-          w1.z = pack_bf16(g[12], g[13]);
-          w1.w = pack_bf16(g[14], g[15]);
-          uint4* dstp = reinterpret_cast<uint4*>((which ? a.dk : a.dv) + eo);
-          dstp[0] = w0;
-          dstp[1] = w1;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c0 = hh * 32 + cc * 8;  // first of 8 columns
+            const float4 d0 = ndel4[c0 / 4], d1 = ndel4[c0 / 4 + 1];
+            const int l0 = cc * 8;
+            const float2 s01 = f2_unpack(f2_mul(f2_pack(sv[c0], sv[c0 + 1]),
+                                                f2_add(f2_pack(dp[l0], dp[l0 + 1]), f2_pack(d0.x, d0.y))));
+            const float2 s23 = f2_unpack(f2_mul(f2_pack(sv[c0 + 2], sv[c0 + 3]),
+                                                f2_add(f2_pack(dp[l0 + 2], dp[l0 + 3]), f2_pack(d0.z, d0.w))));
+            const float2 s45 = f2_unpack(f2_mul(f2_pack(sv[c0 + 4], sv[c0 + 5]),
+                                                f2_add(f2_pack(dp[l0 + 4], dp[l0 + 5]), f2_pack(d1.x, d1.y))));
+            const float2 s67 = f2_unpack(f2_mul(f2_pack(sv[c0 + 6], sv[c0 + 7]),
+                                                f2_add(f2_pack(dp[l0 + 6], dp[l0 + 7]), f2_pack(d1.z, d1.w))));
+            *reinterpret_cast<uint4*>(dst + sw128_offset(row, c0 / 8)) =
+                make_uint4(pack_bf16(s01.x, s01.y), pack_bf16(s23.x, s23.y), pack_bf16(s45.x, s45.y),
+                           pack_bf16(s67.x, s67.y));
+          }
         }
+        fence_proxy_async_smem();
+        mbar_arrive(bar_pt_full + pb);
+        mbar_arrive(bar_dst_full + pb);
       }
+      gs += it.n;
     }
   } else if (warp < 14) {
-    // ------------------------------------------------------------ dQ reduction
+    // ------------------------------------------------------------ dQ reduction + dV/dK epilogue
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // query row of the pair: step 2p + row / 64
+    const int row = quarter * 32 + lane;  // query row of a dQ product; key row of the epilogue
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const int n_pairs = (n + 1) >> 1;
     bool ok = true;
-    for (int p = 0; p < n_pairs; ++p) {
-      const int qb = p % C::DQBUF;
-      ok = ok && mbar_wait(bar_dq_full + qb, (p / C::DQBUF) & 1, abort_flag);
-      tc_fence_after();
-      const int s = 2 * p + (row >> 6);
-      bool qvalid = false;
-      float* dstp = a.dq_acc;
-      if (s < n) {
-        const int x = (entry_at(sEnt, gEnt, s) >> 3) * C::TQ + (row & 63);
-        qvalid = x < a.N;
-        const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
-        dstp = a.dq_acc + (static_cast<size_t>(bh) * a.N + (qvalid ? qn : 0)) * D;
-      }
-#pragma unroll
-      for (int i = 0; i < D / 16; ++i) {
-        float g[16];
-        tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, g);
-        tmem_wait_ld();
+    int gs = 0, ne = 0, qi = 0;
+    BwdItem nxt = (cta < n_items) ? bwd_item(a, cta) : BwdItem{0, 0, 0, 0};
+    for (int k = 0, item = cta; ok && item < n_items;) {
+      const BwdItem it = nxt;  // the next item's schedule entry is fetched one item ahead
+      item = zigzag_item(++k, cta, n_ctas);
+      if (item < n_items) nxt = bwd_item(a, item);
+      for (int jj = 0; jj < it.n; ++jj) {
+        const int g = gs + jj;
+        if (!((g & 1) || jj == it.n - 1)) continue;
+        const int qb = qi % C::DQBUF;
+        ok = ok && mbar_wait(bar_dq_full + qb, (qi / C::DQBUF) & 1, abort_flag);
+        tc_fence_after();
+        // rows 0..63 belong to global step 2*(g/2), rows 64..127 to the next one
+        const int gstep = (g & ~1) + (row >> 6);
+        const int js = gstep - gs;
+        bool qvalid = js >= 0 && js <= jj;
+        float* dstp = a.dq_acc;
         if (qvalid) {
+          const int x = (a.ent[it.e0 + js] >> 3) * C::TQ + (row & 63);
+          qvalid = x < a.N;
+          const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
+          dstp = a.dq_acc + (static_cast<size_t>(it.bh) * a.N + (qvalid ? qn : 0)) * D;
+        }
 #pragma unroll
-          for (int u = 0; u < 16; u += 4)
-            red_add_v4(dstp + i * 16 + u, g[u] * a.scale, g[u + 1] * a.scale, g[u + 2] * a.scale,
-                       g[u + 3] * a.scale);
+        for (int i = 0; i < D / 16; ++i) {
+          float gq[16];
+          tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, gq);
+          tmem_wait_ld();
+          if (qvalid) {
+#pragma unroll
+            for (int u = 0; u < 16; u += 4)
+              red_add_v4(dstp + i * 16 + u, gq[u] * a.scale, gq[u + 1] * a.scale, gq[u + 2] * a.scale,
+                         gq[u + 3] * a.scale);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_dq_free + qb);
+        ++qi;
+      }
+      // ---- dV / dK of this item (thread = key row)
+      const KeyRow kr = key_row<D>(a, it.kt, row);
+      if (it.n > 0) {
+        ok = ok && mbar_wait(bar_dkv_full, ne & 1, abort_flag);
+        tc_fence_after();
+      }
+      const size_t off = (static_cast<size_t>(it.bh) * a.N + (kr.kvalid ? kr.knat : 0)) * D;
+      bool add = false;
+      if (a.add_part == 1) add = true;
+      else if (a.add_part == 2) add = (kr.knat % a.l) >= (a.l - a.c);
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+        const uint32_t col = which ? C::COL_DK : C::COL_DV;
+        const float mul = which ? a.scale : 1.f;
+#pragma unroll
+        for (int i = 0; i < D / 16; ++i) {
+          float gv[16];
+          if (it.n > 0) {
+            tmem_ld16(tmem + lane_base + col + i * 16, gv);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) gv[u] = 0.f;
+          }
+          if (!kr.kvalid) continue;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) gv[u] *= mul;
+          store_grad_row<D, 16>(a, which, off, i * 16, gv, add);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar_dq_free + qb);
+      if (it.n > 0) {
+        tc_fence_before();
+        mbar_arrive(bar_dkv_free);
+        ++ne;
+      }
+      gs += it.n;
     }
   }
 
@@ -510,15 +633,16 @@ __global__ void __launch_bounds__(480, 1)
 
 // Backward preprocess, one row per D/8 threads (16-byte loads; the row loop
 // is warp-uniform so the shuffles always see every lane):
-//   Delta_i = sum_d dO_id O_id (fp32); writes (lse_i * log2 e, Delta_i) to the
-//   natural-order array and, for the strided pattern, at the row's
-//   column-major position t = (i mod l) * R + i / l; pads positions
-//   [N, n_pad) of both with (+inf, 0); zeroes the fp32 dQ accumulator.
+//   Delta_i = sum_d dO_id O_id (fp32); writes -lse_i * log2 e and -Delta_i
+//   (in [64-step][2][64] blocks) to the natural-order array and, for the
+//   strided pattern, at the row's column-major position
+//   t = (i mod l) * R + i / l; pads positions [N, n_pad) of both with
+//   (-inf, 0); zeroes the fp32 dQ accumulator.
 template <int D>
 __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse,
-                                                         float2* __restrict__ ld_nat, float2* __restrict__ ld_col,
+                                                         float* __restrict__ ld_nat, float* __restrict__ ld_col,
                                                          float* __restrict__ dq_acc, int BH, int N, int n_pad,
                                                          int l, int R) {
   constexpr int TPR = D / 8;         // threads per row
@@ -553,9 +677,15 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
       if (sub == 0) {
         const long long bh = r / N;
         const int i = static_cast<int>(r - bh * N);
-        const float2 v = make_float2(lse[r] * 1.4426950408889634f, acc);
-        ld_nat[bh * n_pad + i] = v;
-        if (ld_col) ld_col[bh * n_pad + (i % l) * R + i / l] = v;
+        const float nl = -lse[r] * 1.4426950408889634f;
+        const long long o = bh * n_pad * 2;
+        ld_nat[o + (i / 64) * 128 + (i % 64)] = nl;
+        ld_nat[o + (i / 64) * 128 + 64 + (i % 64)] = -acc;
+        if (ld_col) {
+          const int t = (i % l) * R + i / l;
+          ld_col[o + (t / 64) * 128 + (t % 64)] = nl;
+          ld_col[o + (t / 64) * 128 + 64 + (t % 64)] = -acc;
+        }
       }
       float4* z = reinterpret_cast<float4*>(dq_acc + r * D + sub * 8);
       z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -566,8 +696,13 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
   for (long long k = tid; k < static_cast<long long>(BH) * pad; k += nthr) {
     const long long bh = k / pad;
     const long long i = N + (k - bh * pad);
-    ld_nat[bh * n_pad + i] = make_float2(INFINITY, 0.f);
-    if (ld_col) ld_col[bh * n_pad + i] = make_float2(INFINITY, 0.f);
+    const long long o = bh * n_pad * 2 + (i / 64) * 128 + (i % 64);
+    ld_nat[o] = -INFINITY;
+    ld_nat[o + 64] = 0.f;
+    if (ld_col) {
+      ld_col[o] = -INFINITY;
+      ld_col[o + 64] = 0.f;
+    }
   }
 }
 

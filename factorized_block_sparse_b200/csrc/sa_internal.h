@@ -36,6 +36,7 @@ struct TileTable {
   std::vector<int32_t> row_ptr;  // n_rows + 1
   std::vector<int32_t> ent;      // packed entries, ascending tile per source
   std::vector<int32_t> order;    // rows by descending entry count (launch order)
+  std::vector<int32_t> sched;    // per launch slot s: {row order[s], its first entry, its count, 0}
   int n_rows = 0;
 };
 
@@ -43,6 +44,7 @@ struct DevTable {
   const int32_t* row_ptr = nullptr;
   const int32_t* ent = nullptr;
   const int32_t* order = nullptr;
+  const int32_t* sched = nullptr;  // 16-byte aligned, 4 ints per slot
   int n_rows = 0;
   int nnz = 0;
 };

@@ -175,6 +175,13 @@ void finish_table(TileTable& tt, const std::vector<std::vector<int32_t>>& rows) 
     if (lx != ly) return lx > ly;
     return x > y;
   });
+  tt.sched.assign(4 * static_cast<size_t>(tt.n_rows), 0);
+  for (int s = 0; s < tt.n_rows; ++s) {
+    const int r = tt.order[s];
+    tt.sched[4 * s + 0] = r;
+    tt.sched[4 * s + 1] = tt.row_ptr[r];
+    tt.sched[4 * s + 2] = tt.row_ptr[r + 1] - tt.row_ptr[r];
+  }
 }
 
 }  // namespace
