@@ -158,6 +158,35 @@ struct MapSet {
   CUtensorMap nat, col, sum;
 };
 
+// fp32 maps over the dQ accumulator [BH, N, D] for TMA bulk reduce-add:
+// natural {D, N, BH} box {32, 32, 1}; column-major {D, l, R, BH} box
+// {32, 1, min(R, 32), 1}; 128-byte swizzle (32 fp32 per row of a box).
+int make_dq_maps(CUtensorMap* nat, CUtensorMap* col, const float* base, const Geo& g, int pattern) {
+  std::memset(nat, 0, sizeof(*nat));
+  std::memset(col, 0, sizeof(*col));
+  if (g.D > 64) return SA_OK;  // not used for D = 128
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.N * g.D * 4};
+    const cuuint32_t box[3] = {32, 32, 1};
+    if (g_encode(nat, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SA_ERR_CUDA;
+  }
+  if (pattern == SA_STRIDED) {
+    const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
+    const cuuint64_t strides[3] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.l * g.D * 4, (cuuint64_t)g.N * g.D * 4};
+    const cuuint32_t box[4] = {32, 1, (cuuint32_t)std::min(g.R, 32), 1};
+    if (g_encode(col, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
 int make_maps(MapSet* ms, const void* base, const Geo& g, int pattern, int rows) {
   std::memset(ms, 0, sizeof(*ms));
   int st = map_nat(&ms->nat, base, g, rows);
@@ -373,6 +402,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   float* dk_part = reinterpret_cast<float*>(wsb + w.dk);
   float* dv_part = reinterpret_cast<float*>(wsb + w.dv);
   const long long rows = static_cast<long long>(g.BH) * N;
+  CUtensorMap mdq_nat, mdq_col;
+  if ((st = make_dq_maps(&mdq_nat, &mdq_col, dq_acc, g, L->pattern))) return st;
 
   st = launch(K_BWD_PRE * 4 + L->pattern, s, [&] {
     sa_bwd_pre_kernel<D><<<grid_for(rows * (D / 8), 256), 256, 0, s>>>(
@@ -410,7 +441,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
     st = launch(K_BWD_SEC * 4 + L->pattern, s, [&] {
       kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
-                                               mv.col, mv.sum, a);
+                                               mv.col, mv.sum, mdq_nat, mdq_col, a);
     });
     if (st) return st;
   }
@@ -424,7 +455,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
     st = launch(K_BWD_MAIN * 4 + L->pattern, s, [&] {
       kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
-                                               mv.col, mv.sum, a);
+                                               mv.col, mv.sum, mdq_nat, mdq_col, a);
     });
     if (st) return st;
   }

@@ -26,8 +26,10 @@
 // one warp per TMEM lane quarter each), warps 10..13 dQ reduction and the
 // dV/dK epilogue, warp 14 lane 0 issue of dV/dK/dQ.  Warp w may only touch
 // TMEM lanes 32*(w%4)..32*(w%4)+31, so every role picks its rows by w%4.
-// TMEM columns (NBUF = 2 for D <= 64, 1 for D = 128):
-//   ST[b] = b*64, dPT[b] = NBUF*64 + b*64, dV = 2*NBUF*64, dK = dV + D,
+// TMEM columns: ST = 0, dPT = 64 (one buffer each; the two elementwise
+// groups take it in turn), dV[b] = 128 + b*2D, dK[b] = dV[b] + D with b the
+// item parity (two buffers for D <= 64, so an item's dV/dK accumulate while
+// the previous item's are read out), then the dQ buffers:
 //   dQ[b] = dK + D + b*D (two dQ buffers for D <= 64, one for D = 128).
 #pragma once
 
@@ -62,12 +64,18 @@ struct BwdArgs {
 template <int D>
 struct BwdCfg {
   static constexpr int TK = 128, TQ = 64;
-  static constexpr int NBUF = (D >= 128) ? 1 : 2;      // ST/dPT buffers in TMEM
+  static constexpr int NBUF = 1;                       // ST/dPT buffers in TMEM
+  static constexpr int DKVB = (D >= 128) ? 1 : 2;      // dV/dK buffers (by item parity)
   // Q/dO ring (>= 2: see the S issuer).  A stage is held from its load
   // until dK of its step is done, which trails the S products by about two
   // steps, so the ring must be deep for the loads to run ahead.
-  static constexpr int STAGES = (D >= 128) ? 2 : 3;
+  static constexpr int STAGES = (D == 32) ? 3 : 2;
   static constexpr int KVB = (D >= 128) ? 1 : 2;       // K/V buffers (next item's tiles load early)
+  // dQ is added to the fp32 workspace by TMA bulk reduce from a per-warp
+  // staging buffer (32 query rows x D fp32, 128B-swizzled 32-column boxes);
+  // D = 128 has no shared memory left for it and uses vector reductions.
+  static constexpr bool DQ_TMA = (D <= 64);
+  static constexpr int DQS_WARP_BYTES = DQ_TMA ? 32 * D * 4 : 0;
   static constexpr int DST_BUFS = (D >= 128) ? 1 : 2;  // dS^T pair buffers
   static constexpr int DQBUF = (D >= 128) ? 1 : 2;     // dQ TMEM buffers
   static constexpr int ROWB = (D >= 64) ? 128 : 64;
@@ -85,15 +93,17 @@ struct BwdCfg {
   static constexpr int OFF_PT = OFF_DO + STAGES * QS_BYTES;
   static constexpr int OFF_DST = OFF_PT + 2 * PT_BYTES;
   static constexpr int OFF_LD = OFF_DST + DST_BUFS * DST_BYTES;  // float [STAGES][2][64]
-  static constexpr int OFF_BAR = OFF_LD + STAGES * LD_BYTES;
-  static constexpr int N_BARS = 2 * KVB + 2 * STAGES + 2 * 5 + DST_BUFS + 2 * DQBUF + 2;
+  // 4 x DQS_WARP_BYTES; 1 KiB aligned (the 128-byte swizzle pattern is address based)
+  static constexpr int OFF_DQS = (OFF_LD + STAGES * LD_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = OFF_DQS + 4 * DQS_WARP_BYTES;
+  static constexpr int N_BARS = 2 * KVB + 2 * STAGES + 2 * 7 + DST_BUFS + 2 * DQBUF + 2 * DKVB;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int COL_DPT = NBUF * 64;
-  static constexpr int COL_DV = 2 * NBUF * 64;
-  static constexpr int COL_DK = COL_DV + D;
-  static constexpr int COL_DQ = COL_DK + D;
+  static constexpr int COL_DV = 2 * NBUF * 64;        // + b * 2D
+  static constexpr int COL_DK = COL_DV + D;           // + b * 2D
+  static constexpr int COL_DQ = COL_DV + DKVB * 2 * D;
   static constexpr int THREADS = 480;
   static_assert(COL_DQ + DQBUF * D <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 2, "the S issuer needs step j's Q/dO while step j-1's is still in use");
@@ -213,6 +223,7 @@ __global__ void __launch_bounds__(480, 1)
                   const __grid_constant__ CUtensorMap mk_nat, const __grid_constant__ CUtensorMap mk_col,
                   const __grid_constant__ CUtensorMap mk_sum, const __grid_constant__ CUtensorMap mv_nat,
                   const __grid_constant__ CUtensorMap mv_col, const __grid_constant__ CUtensorMap mv_sum,
+                  const __grid_constant__ CUtensorMap mdq_nat, const __grid_constant__ CUtensorMap mdq_col,
                   const BwdArgs a) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -231,16 +242,18 @@ __global__ void __launch_bounds__(480, 1)
   uint64_t* bar_qdo_empty = bar_qdo_full + C::STAGES;    // [STAGES]
   // Per global-step-parity barriers (one per elementwise group), so that a
   // barrier is never waited on two phases ahead.
-  uint64_t* bar_s_full = bar_qdo_empty + C::STAGES;      // [2]  ST and dPT of a step
-  uint64_t* bar_s_free = bar_s_full + 2;                 // [2]  elementwise done reading them
-  uint64_t* bar_pt_full = bar_s_free + 2;                // [2]
+  uint64_t* bar_st_full = bar_qdo_empty + C::STAGES;     // [2]  ST of a step in TMEM
+  uint64_t* bar_st_free = bar_st_full + 2;               // [2]  elementwise has read it
+  uint64_t* bar_dpt_full = bar_st_free + 2;              // [2]  dPT of a step in TMEM
+  uint64_t* bar_dpt_free = bar_dpt_full + 2;             // [2]  elementwise has read it
+  uint64_t* bar_pt_full = bar_dpt_free + 2;              // [2]
   uint64_t* bar_pt_free = bar_pt_full + 2;               // [2]
   uint64_t* bar_dst_full = bar_pt_free + 2;              // [2]
   uint64_t* bar_dst_free = bar_dst_full + 2;             // [DST_BUFS] per global pair
   uint64_t* bar_dq_full = bar_dst_free + C::DST_BUFS;    // [DQBUF] per dQ product
   uint64_t* bar_dq_free = bar_dq_full + C::DQBUF;        // [DQBUF]
-  uint64_t* bar_dkv_full = bar_dq_free + C::DQBUF;       // per non-empty item
-  uint64_t* bar_dkv_free = bar_dkv_full + 1;
+  uint64_t* bar_dkv_full = bar_dq_free + C::DQBUF;       // [DKVB] per non-empty item
+  uint64_t* bar_dkv_free = bar_dkv_full + C::DKVB;       // [DKVB]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
@@ -260,8 +273,10 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(bar_qdo_empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_s_full + b, 1);
-      mbar_init(bar_s_free + b, 128);
+      mbar_init(bar_st_full + b, 1);
+      mbar_init(bar_st_free + b, 128);
+      mbar_init(bar_dpt_full + b, 1);
+      mbar_init(bar_dpt_free + b, 128);
       mbar_init(bar_pt_full + b, 128);
       mbar_init(bar_pt_free + b, 1);
       mbar_init(bar_dst_full + b, 128);
@@ -271,8 +286,10 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(bar_dq_full + b, 1);
       mbar_init(bar_dq_free + b, 128);
     }
-    mbar_init(bar_dkv_full, 1);
-    mbar_init(bar_dkv_free, 128);
+    for (int b = 0; b < C::DKVB; ++b) {
+      mbar_init(bar_dkv_full + b, 1);
+      mbar_init(bar_dkv_free + b, 128);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -345,10 +362,8 @@ __global__ void __launch_bounds__(480, 1)
           const int st = g % C::STAGES;
           const int b = g % C::NBUF;
           ok = mbar_wait(bar_qdo_full + st, (g / C::STAGES) & 1, abort_flag);
-          if (ok && g >= C::NBUF) {  // TMEM buffer b was last used by step g - NBUF
-            const int gp = g - C::NBUF;
-            ok = mbar_wait(bar_s_free + (gp & 1), (gp >> 1) & 1, abort_flag);
-          }
+          const int gp = g - C::NBUF;  // last user of TMEM buffer b
+          if (ok && gp >= 0) ok = mbar_wait(bar_st_free + (gp & 1), (gp >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
@@ -357,11 +372,17 @@ __global__ void __launch_bounds__(480, 1)
           for (int kk = 0; kk < D / 16; ++kk)
             mma_bf16_ss(tmem + b * 64, bwd_kdesc<D>(k_base, C::TK, kk), bwd_kdesc<D>(q_base, C::TQ, kk), id_s,
                         kk > 0);
+          mma_commit(bar_st_full + (g & 1));
+          if (gp >= 0 && !mbar_wait(bar_dpt_free + (gp & 1), (gp >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_bf16_ss(tmem + C::COL_DPT + b * 64, bwd_kdesc<D>(v_base, C::TK, kk),
                         bwd_kdesc<D>(do_base, C::TQ, kk), id_s, kk > 0);
-          mma_commit(bar_s_full + (g & 1));
+          mma_commit(bar_dpt_full + (g & 1));
         }
         gs += it.n;
         ++ne;
@@ -385,8 +406,10 @@ __global__ void __launch_bounds__(480, 1)
         if (it.n == 0) continue;
         const int kb = ne % C::KVB;
         ok = mbar_wait(bar_kv_full + kb, (ne / C::KVB) & 1, abort_flag);
-        // dV/dK of the previous item must have been read out by the epilogue
-        if (ok && ne >= 1) ok = mbar_wait(bar_dkv_free, (ne - 1) & 1, abort_flag);
+        // this item's dV/dK buffer must have been read out by the epilogue of
+        // the item DKVB before it
+        const int vb = ne % C::DKVB;
+        if (ok && ne >= C::DKVB) ok = mbar_wait(bar_dkv_free + vb, ((ne / C::DKVB) - 1) & 1, abort_flag);
         const uint32_t k_base = smem_u32(sK + kb * C::KV_BYTES);
         for (int jj = 0; ok && jj < it.n; ++jj) {
           const int g = gs + jj;
@@ -401,14 +424,14 @@ __global__ void __launch_bounds__(480, 1)
           const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
 #pragma unroll
           for (int kk = 0; kk < C::TQ / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_DV, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
+            mma_bf16_ss(tmem + C::COL_DV + vb * 2 * D, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
                         (jj > 0 || kk > 0));
           mma_commit(bar_pt_free + pb);
           if (!mbar_wait(bar_dst_full + pb, (g >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < C::TQ / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_DK, pt_kdesc(dst_pair + pb * C::PT_BYTES, kk),
+            mma_bf16_ss(tmem + C::COL_DK + vb * 2 * D, pt_kdesc(dst_pair + pb * C::PT_BYTES, kk),
                         bwd_mndesc<D>(q_base, C::TQ, kk), id_kv, (jj > 0 || kk > 0));
           mma_commit(bar_qdo_empty + st);
           if ((g & 1) || jj == it.n - 1) {
@@ -429,7 +452,7 @@ __global__ void __launch_bounds__(480, 1)
             ++qi;
           }
         }
-        mma_commit(bar_dkv_full);
+        mma_commit(bar_dkv_full + vb);
         mma_commit(bar_kv_empty + kb);
         gs += it.n;
         ++ne;
@@ -463,7 +486,7 @@ __global__ void __launch_bounds__(480, 1)
         const bool partial = e & 1;
         const int x0 = (e >> 3) * C::TQ;
         ok = ok && mbar_wait(bar_qdo_full + st, (g / C::STAGES) & 1, abort_flag);
-        ok = ok && mbar_wait(bar_s_full + pb, (g >> 1) & 1, abort_flag);
+        ok = ok && mbar_wait(bar_st_full + pb, (g >> 1) & 1, abort_flag);
         // P^T buffer pb is free once dV of step g-2 has completed; the dS^T
         // pair buffer once the product over pair P - DST_BUFS has.
         if (g >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((g >> 1) - 1) & 1, abort_flag);
@@ -481,6 +504,8 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
         for (int c16 = 0; c16 < 4; ++c16) tmem_ld16(tmem + lane_base + b * 64 + c16 * 16, sv + c16 * 16);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_st_free + pb);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float4 t = nlse4[i];
@@ -503,8 +528,10 @@ __global__ void __launch_bounds__(480, 1)
           *reinterpret_cast<uint4*>(pt + sw128_offset(row, ch)) =
               make_uint4(pack_bf16(sv[8 * ch], sv[8 * ch + 1]), pack_bf16(sv[8 * ch + 2], sv[8 * ch + 3]),
                          pack_bf16(sv[8 * ch + 4], sv[8 * ch + 5]), pack_bf16(sv[8 * ch + 6], sv[8 * ch + 7]));
-        // (2) dP^T row in two halves (both TMEM buffers of the step are
-        //     released after the second); dS = P (dP - Delta) in fp32 pairs
+        // (2) dP^T row in two halves (its TMEM buffer is released after the
+        //     second); dS = P (dP - Delta) in fp32 pairs
+        ok = ok && mbar_wait(bar_dpt_full + pb, (g >> 1) & 1, abort_flag);
+        tc_fence_after();
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float dp[32];
@@ -513,7 +540,7 @@ __global__ void __launch_bounds__(480, 1)
           tmem_wait_ld();
           if (hh == 1) {
             tc_fence_before();
-            mbar_arrive(bar_s_free + pb);
+            mbar_arrive(bar_dpt_free + pb);
           }
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
@@ -560,34 +587,70 @@ __global__ void __launch_bounds__(480, 1)
         // rows 0..63 belong to global step 2*(g/2), rows 64..127 to the next one
         const int gstep = (g & ~1) + (row >> 6);
         const int js = gstep - gs;
-        bool qvalid = js >= 0 && js <= jj;
-        float* dstp = a.dq_acc;
-        if (qvalid) {
-          const int x = (a.ent[it.e0 + js] >> 3) * C::TQ + (row & 63);
-          qvalid = x < a.N;
-          const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
-          dstp = a.dq_acc + (static_cast<size_t>(it.bh) * a.N + (qvalid ? qn : 0)) * D;
-        }
+        const bool svalid = js >= 0 && js <= jj;  // the step (and so this warp's 32 rows) is this item's
+        const int xw = svalid ? (a.ent[it.e0 + js] >> 3) * C::TQ + (row & 32) : 0;  // warp's first view row
+        if constexpr (C::DQ_TMA) {
+          float gq[D];
 #pragma unroll
-        for (int i = 0; i < D / 16; ++i) {
-          float gq[16];
-          tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, gq);
+          for (int i = 0; i < D / 16; ++i) tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, gq + i * 16);
           tmem_wait_ld();
-          if (qvalid) {
+          tc_fence_before();
+          mbar_arrive(bar_dq_free + qb);  // the TMEM buffer is free; the rows are in registers
+          if (svalid) {
+            uint8_t* stg = smem + C::OFF_DQS + quarter * C::DQS_WARP_BYTES;
+            if (lane == 0) bulk_wait_read_all();  // previous reduce has read the staging buffer
+            __syncwarp();
 #pragma unroll
-            for (int u = 0; u < 16; u += 4)
-              red_add_v4(dstp + i * 16 + u, gq[u] * a.scale, gq[u + 1] * a.scale, gq[u + 2] * a.scale,
-                         gq[u + 3] * a.scale);
+            for (int bx = 0; bx < D / 32; ++bx)
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<float4*>(stg + bx * 4096 + sw128_offset(lane, ch)) =
+                    make_float4(gq[bx * 32 + ch * 4] * a.scale, gq[bx * 32 + ch * 4 + 1] * a.scale,
+                                gq[bx * 32 + ch * 4 + 2] * a.scale, gq[bx * 32 + ch * 4 + 3] * a.scale);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+#pragma unroll
+              for (int bx = 0; bx < D / 32; ++bx) {
+                if (q_src == SRC_T) {
+                  const int rb = a.R < 32 ? a.R : 32;
+                  for (int s0 = 0; s0 < 32; s0 += rb) {
+                    const int t = xw + s0;
+                    tma_reduce_add_4d(&mdq_col, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
+                  }
+                } else {
+                  tma_reduce_add_3d(&mdq_nat, stg + bx * 4096, bx * 32, xw, it.bh);
+                }
+              }
+              bulk_commit_group();
+            }
           }
+        } else {
+          const int x = xw + (row & 31);
+          const bool qvalid = svalid && x < a.N;
+          const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
+          float* dstp = a.dq_acc + (static_cast<size_t>(it.bh) * a.N + (qvalid ? qn : 0)) * D;
+#pragma unroll
+          for (int i = 0; i < D / 16; ++i) {
+            float gq[16];
+            tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, gq);
+            tmem_wait_ld();
+            if (qvalid) {
+#pragma unroll
+              for (int u = 0; u < 16; u += 4)
+                red_add_v4(dstp + i * 16 + u, gq[u] * a.scale, gq[u + 1] * a.scale, gq[u + 2] * a.scale,
+                           gq[u + 3] * a.scale);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar_dq_free + qb);
         }
-        tc_fence_before();
-        mbar_arrive(bar_dq_free + qb);
         ++qi;
       }
       // ---- dV / dK of this item (thread = key row)
       const KeyRow kr = key_row<D>(a, it.kt, row);
       if (it.n > 0) {
-        ok = ok && mbar_wait(bar_dkv_full, ne & 1, abort_flag);
+        ok = ok && mbar_wait(bar_dkv_full + ne % C::DKVB, (ne / C::DKVB) & 1, abort_flag);
         tc_fence_after();
       }
       const size_t off = (static_cast<size_t>(it.bh) * a.N + (kr.kvalid ? kr.knat : 0)) * D;
@@ -596,7 +659,7 @@ __global__ void __launch_bounds__(480, 1)
       else if (a.add_part == 2) add = (kr.knat % a.l) >= (a.l - a.c);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
-        const uint32_t col = which ? C::COL_DK : C::COL_DV;
+        const uint32_t col = (which ? C::COL_DK : C::COL_DV) + (ne % C::DKVB) * 2 * D;
         const float mul = which ? a.scale : 1.f;
 #pragma unroll
         for (int i = 0; i < D / 16; ++i) {
@@ -616,11 +679,12 @@ __global__ void __launch_bounds__(480, 1)
       }
       if (it.n > 0) {
         tc_fence_before();
-        mbar_arrive(bar_dkv_free);
+        mbar_arrive(bar_dkv_free + ne % C::DKVB);
         ++ne;
       }
       gs += it.n;
     }
+    if (C::DQ_TMA && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
