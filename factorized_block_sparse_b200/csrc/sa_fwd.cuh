@@ -4,8 +4,9 @@
 // of its table (natural, or column-major for the strided column view).  It
 // walks the tile's list of 64-key tiles.  Per key tile:
 //   S = Q K^T            tcgen05.mma, bf16 in smem -> fp32 in TMEM
-//   mask (PARTIAL only), running max, P = exp2(S*scale*log2e - m) -> bf16
-//   O += P V             tcgen05.mma, P staged in 128B-swizzled smem
+//   mask (PARTIAL only), running max, P = exp2(S*scale*log2e - m) -> bf16,
+//                        written back into TMEM over its own S columns
+//   O += P V             tcgen05.mma with A = P read from TMEM
 // This is masked softmax attention restricted to the nonzero blocks of the
 // layout ("OpenAI Sparse Transformer", "Sparse Attention and Algorithmic
 // Complexity" and "Implementation and Limitations").
@@ -17,7 +18,9 @@
 //                   32*(w%4)+t, which is TMEM lane 32*(w%4)+t
 //   warp 6 lane 0 : issues O += P V (a second issuing thread, so S of the
 //                   next tiles never waits behind PV of earlier ones)
-// TMEM columns: S double buffer [0,64) and [64,128); O accumulator [128,128+D).
+// TMEM columns: S double buffer [0,64) and [64,128) (P of a tile occupies the
+// first 32 columns of its S buffer, two bf16 per column); O accumulator
+// [128,128+D).  An S buffer is reused once PV of its tile has completed.
 //
 // The running max is only moved when it grows by more than 2^8 (in the
 // exp2 domain), so O is rescaled rarely; the final normalisation uses the
@@ -44,7 +47,7 @@ struct FwdArgs {
 template <int D>
 struct FwdCfg {
   static constexpr int TQ = 128, TK = 64;
-  static constexpr int STAGES = (D >= 128) ? 2 : 3;
+  static constexpr int STAGES = (D >= 128) ? 3 : ((D == 64) ? 5 : 6);
   static constexpr int ROWB = (D >= 64) ? 128 : 64;     // bytes per row per panel
   static constexpr int PANELS = (D >= 64) ? D / 64 : 1;
   static constexpr int BOXW = (D >= 64) ? 64 : D;       // TMA box inner width (elements)
@@ -52,12 +55,10 @@ struct FwdCfg {
   static constexpr int SBO = 8 * ROWB;
   static constexpr int Q_BYTES = TQ * D * 2;
   static constexpr int KV_BYTES = TK * D * 2;
-  static constexpr int P_BYTES = TQ * TK * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
-  static constexpr int OFF_ENT = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_ENT = OFF_V + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_ENT + kMaxStagedEnt * 4;
   static constexpr int N_BARS = 1 + 3 * STAGES + 8;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
@@ -135,15 +136,14 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
-  uint8_t* sP = smem + C::OFF_P;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_q = bars;
   uint64_t* bar_k_full = bars + 1;
   uint64_t* bar_v_full = bar_k_full + C::STAGES;
   uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
   uint64_t* bar_s_full = bar_kv_empty + C::STAGES;  // [2]
-  uint64_t* bar_s_empty = bar_s_full + 2;           // [2]
-  uint64_t* bar_p_full = bar_s_empty + 2;           // [2]
+  uint64_t* bar_s_empty = bar_s_full + 2;           // [2]  PV of the buffer's tile done
+  uint64_t* bar_p_full = bar_s_empty + 2;           // [2]  P written into TMEM
   uint64_t* bar_pv_done = bar_p_full + 2;           // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_s_full + s, 1);
-      mbar_init(bar_s_empty + s, 128);
+      mbar_init(bar_s_empty + s, 1);
       mbar_init(bar_p_full + s, 128);
       mbar_init(bar_pv_done + s, 1);
     }
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
   } else if (warp == 6) {
     // ------------------------------------------------------------ PV issuer: O += P_j V_j
     // S_j has completed before P_j exists, so this thread's commit after PV_j
-    // also releases the K half of the stage.
+    // also releases the K half of the stage and the S/P buffer of the tile.
     if (lane == 0 && n > 0) {
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, false, true);
       bool ok = true;
@@ -237,13 +237,13 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
              mbar_wait(bar_v_full + st, (jj / C::STAGES) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t p_base = smem_u32(sP + pb * C::P_BYTES);
         const uint32_t v_base = smem_u32(sV + st * C::KV_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < C::TK / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_O, make_desc(p_base + kk * 32, 16, 1024, kSwizzle128),
-                      mnmajor_desc<D>(v_base, C::TK, kk), idesc_pv, (jj > 0 || kk > 0));
+        for (int kk = 0; kk < C::TK / 16; ++kk)  // 16 keys of P = 8 TMEM columns per k-step
+          mma_bf16_ts(tmem + C::COL_O, tmem + pb * C::TK + kk * 8, mnmajor_desc<D>(v_base, C::TK, kk), idesc_pv,
+                      (jj > 0 || kk > 0));
         mma_commit(bar_pv_done + pb);
+        mma_commit(bar_s_empty + pb);
         mma_commit(bar_kv_empty + st);
       }
     }
@@ -279,8 +279,6 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
 #pragma unroll
       for (int i = 0; i < C::TK / 16; ++i) tmem_ld16(tmem + lane_base + sb * C::TK + i * 16, s + i * 16);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_s_empty + sb);
 
       const int e = entry_at(sEnt, gEnt, j);
       if (e & 1) {
@@ -326,11 +324,9 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
         }
         tmem_wait_st();
       }
-      // P buffer j&1 is free once PV of tile j-2 has completed.
-      if (j >= 2) ok = ok && mbar_wait(bar_pv_done + sb, ((j >> 1) - 1) & 1, abort_flag);
       const float neg = (m_used == -INFINITY) ? 0.f : -m_used;
       float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // partial row sums
-      uint8_t* pbuf = sP + sb * C::P_BYTES;
+      uint32_t pk[C::TK / 2];
 #pragma unroll
       for (int ch = 0; ch < C::TK / 8; ++ch) {
         float p[8];
@@ -339,16 +335,14 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
           p[u] = ex2(fmaf(s[ch * 8 + u], a.scale_log2, neg));
           rs8[u] += p[u];
         }
-        uint4 w;
-        w.x = pack_bf16(p[0], p[1]);
-        w.y = pack_bf16(p[2], p[3]);
-        w.z = pack_bf16(p[4], p[5]);
-        w.w = pack_bf16(p[6], p[7]);
-        *reinterpret_cast<uint4*>(pbuf + sw128_offset(row, ch)) = w;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) pk[ch * 4 + u] = pack_bf16(p[2 * u], p[2 * u + 1]);
       }
+      // P over the first TK/2 columns of its own S buffer (the S values are in registers)
+      tmem_st32(tmem + lane_base + sb * C::TK, pk);
+      tmem_wait_st();
       const float rsum = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l_sum = l_sum * factor + rsum;
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar_p_full + sb);
     }
