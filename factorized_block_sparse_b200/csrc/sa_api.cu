@@ -392,8 +392,10 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = make_maps(&mv, v, g, L->pattern, BwdCfg<D>::TK))) return st;
   DeviceCopy dc;
   if ((st = to_device(L, &dc))) return st;
-  auto kern = sa_bwd_kernel<D>;
-  if ((st = set_smem(kern, BwdCfg<D>::SMEM))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, false>, BwdCfg<D, false>::SMEM))) return st;
+  if constexpr (D <= 64) {
+    if ((st = set_smem(sa_bwd_kernel<D, true>, BwdCfg<D, true>::SMEM))) return st;
+  }
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* ld_nat = reinterpret_cast<float*>(wsb + w.ld_nat);
@@ -431,34 +433,37 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   const bool sec = (L->pattern == SA_STRIDED || L->pattern == SA_FIXED) && dc.bwd_sec.n_rows > 0;
   a.BH = g.BH;
   const int n_sm = sm_count();
+  // Tables whose items average many steps take the LONG shape of the kernel.
+  auto run = [&](int kind, const DevTable& t) -> int {
+    const long long items = static_cast<long long>(t.n_rows) * g.BH;
+    dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
+    const bool long_items = D <= 64 && t.nnz >= kBwdLongSteps * static_cast<long long>(t.n_rows);
+    return launch(kind, s, [&] {
+      if constexpr (D <= 64) {
+        if (long_items) {
+          sa_bwd_kernel<D, true><<<grid, BwdCfg<D, true>::THREADS, BwdCfg<D, true>::SMEM, s>>>(
+              mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col, a);
+          return;
+        }
+      }
+      sa_bwd_kernel<D, false><<<grid, BwdCfg<D, false>::THREADS, BwdCfg<D, false>::SMEM, s>>>(
+          mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col, a);
+    });
+  };
   if (sec) {
     a.sched = dc.bwd_sec.sched;
     a.ent = dc.bwd_sec.ent;
     a.n_slots = dc.bwd_sec.n_rows;
     a.key_view = (L->pattern == SA_STRIDED) ? SRC_T : SRC_S;
     a.add_part = 0;
-    const long long items = static_cast<long long>(a.n_slots) * g.BH;
-    dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
-    st = launch(K_BWD_SEC * 4 + L->pattern, s, [&] {
-      kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
-                                               mv.col, mv.sum, mdq_nat, mdq_col, a);
-    });
-    if (st) return st;
+    if ((st = run(K_BWD_SEC * 4 + L->pattern, dc.bwd_sec))) return st;
   }
   a.sched = dc.bwd_main.sched;
   a.ent = dc.bwd_main.ent;
   a.n_slots = dc.bwd_main.n_rows;
   a.key_view = SRC_N;
   a.add_part = sec ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
-  {
-    const long long items = static_cast<long long>(a.n_slots) * g.BH;
-    dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
-    st = launch(K_BWD_MAIN * 4 + L->pattern, s, [&] {
-      kern<<<grid, BwdCfg<D>::THREADS, BwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
-                                               mv.col, mv.sum, mdq_nat, mdq_col, a);
-    });
-    if (st) return st;
-  }
+  if ((st = run(K_BWD_MAIN * 4 + L->pattern, dc.bwd_main))) return st;
   const long long n8 = rows * D / 8;
   return launch(K_BWD_FINAL * 4 + L->pattern, s, [&] {
     sa_bwd_final_kernel<<<grid_for(n8, 256), 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);

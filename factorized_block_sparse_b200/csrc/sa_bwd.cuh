@@ -13,7 +13,8 @@
 // that see it.  Per step (global step counter g, continued across items):
 //   ST_g  = K Q^T, dPT_g = V dO^T  (keys on TMEM lanes, 64 columns each,
 //                                   double-buffered)
-//   P^T_g, dS^T_g in bf16 smem     (elementwise warps)
+//   P^T_g, dS^T_g in bf16          (elementwise warps; dS^T in smem, P^T in
+//                                   smem or, in the LONG shape, in TMEM)
 //   dV += P^T dO, dK += dS^T Q     (TMEM accumulators of the item)
 //   dQ = dS K for the 128 queries of the global step pair (g even, g odd),
 //   restricted to the item's own steps, then reduced into an fp32 workspace.
@@ -26,10 +27,11 @@
 // one warp per TMEM lane quarter each), warps 10..13 dQ reduction and the
 // dV/dK epilogue, warp 14 lane 0 issue of dV/dK/dQ.  Warp w may only touch
 // TMEM lanes 32*(w%4)..32*(w%4)+31, so every role picks its rows by w%4.
-// TMEM columns: ST = 0, dPT = 64 (one buffer each; the two elementwise
-// groups take it in turn), dV[b] = 128 + b*2D, dK[b] = dV[b] + D with b the
-// item parity (two buffers for D <= 64, so an item's dV/dK accumulate while
-// the previous item's are read out), then the dQ buffers:
+// TMEM columns: ST[b] = b*64, dPT[b] = NBUF*64 + b*64 (one buffer each that
+// the two elementwise groups take in turn, or one per group in the LONG
+// shape), dV[b] = 2*NBUF*64 + b*2D, dK[b] = dV[b] + D with b the item parity
+// (two buffers for D <= 64 outside the LONG shape, so an item's dV/dK
+// accumulate while the previous item's are read out), then the dQ buffers:
 //   dQ[b] = dK + D + b*D (two dQ buffers for D <= 64, one for D = 128).
 #pragma once
 
@@ -61,16 +63,24 @@ struct BwdArgs {
   float scale_log2;  // log2(e)/sqrt(D)
 };
 
-template <int D>
+// Two shapes of the same kernel.  LONG is for tables whose items run many
+// steps (D <= 64): P^T is written into TMEM over its own S^T columns and dV
+// is a TS-MMA with A read from TMEM, S^T/dP^T are double-buffered, and
+// there is one dV/dK and one K/V buffer (an item boundary costs a short
+// stall), so the shared memory of the P^T buffers and of the second K/V
+// buffer goes to a deeper Q/dO ring.  The other shape keeps P^T in shared
+// memory and double-buffers the per-item state, for items of a few steps.
+template <int D, bool LONG = false>
 struct BwdCfg {
   static constexpr int TK = 128, TQ = 64;
-  static constexpr int NBUF = 1;                       // ST/dPT buffers in TMEM
-  static constexpr int DKVB = (D >= 128) ? 1 : 2;      // dV/dK buffers (by item parity)
+  static constexpr bool PT_TMEM = LONG;
+  static constexpr int NBUF = LONG ? 2 : 1;            // ST/dPT buffers in TMEM
+  static constexpr int DKVB = (LONG || D >= 128) ? 1 : 2;  // dV/dK buffers (by item parity)
   // Q/dO ring (>= 2: see the S issuer).  A stage is held from its load
   // until dK of its step is done, which trails the S products by about two
   // steps, so the ring must be deep for the loads to run ahead.
-  static constexpr int STAGES = (D == 32) ? 3 : 2;
-  static constexpr int KVB = (D >= 128) ? 1 : 2;       // K/V buffers (next item's tiles load early)
+  static constexpr int STAGES = LONG ? ((D == 32) ? 8 : 5) : ((D == 32) ? 3 : 2);
+  static constexpr int KVB = (LONG || D >= 128) ? 1 : 2;  // K/V buffers (next item's tiles load early)
   // dQ is added to the fp32 workspace by TMA bulk reduce from a per-warp
   // staging buffer (32 query rows x D fp32, 128B-swizzled 32-column boxes);
   // D = 128 has no shared memory left for it and uses vector reductions.
@@ -91,7 +101,7 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + KVB * KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + STAGES * QS_BYTES;
   static constexpr int OFF_PT = OFF_DO + STAGES * QS_BYTES;
-  static constexpr int OFF_DST = OFF_PT + 2 * PT_BYTES;
+  static constexpr int OFF_DST = OFF_PT + (PT_TMEM ? 0 : 2 * PT_BYTES);
   static constexpr int OFF_LD = OFF_DST + DST_BUFS * DST_BYTES;  // float [STAGES][2][64]
   // 4 x DQS_WARP_BYTES; 1 KiB aligned (the 128-byte swizzle pattern is address based)
   static constexpr int OFF_DQS = (OFF_LD + STAGES * LD_BYTES + 1023) / 1024 * 1024;
@@ -108,6 +118,7 @@ struct BwdCfg {
   static_assert(COL_DQ + DQBUF * D <= TMEM_COLS, "TMEM budget");
   static_assert(STAGES >= 2, "the S issuer needs step j's Q/dO while step j-1's is still in use");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(!LONG || D <= 64, "TMEM budget of the LONG shape");
 };
 
 // K-major operand (rows x D) for k-step kk (16 elements of D).
@@ -216,7 +227,7 @@ __device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size
   }
 }
 
-template <int D>
+template <int D, bool LONG>
 __global__ void __launch_bounds__(480, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mdo_nat, const __grid_constant__ CUtensorMap mdo_col,
@@ -225,7 +236,7 @@ __global__ void __launch_bounds__(480, 1)
                   const __grid_constant__ CUtensorMap mv_col, const __grid_constant__ CUtensorMap mv_sum,
                   const __grid_constant__ CUtensorMap mdq_nat, const __grid_constant__ CUtensorMap mdq_col,
                   const BwdArgs a) {
-  using C = BwdCfg<D>;
+  using C = BwdCfg<D, LONG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + C::OFF_K;
@@ -363,7 +374,10 @@ __global__ void __launch_bounds__(480, 1)
           const int b = g % C::NBUF;
           ok = mbar_wait(bar_qdo_full + st, (g / C::STAGES) & 1, abort_flag);
           const int gp = g - C::NBUF;  // last user of TMEM buffer b
-          if (ok && gp >= 0) ok = mbar_wait(bar_st_free + (gp & 1), (gp >> 1) & 1, abort_flag);
+          // the S^T buffer is free once it has been read out or, when it
+          // holds P^T, once dV of that step has completed
+          if (ok && gp >= 0)
+            ok = mbar_wait((C::PT_TMEM ? bar_pt_free : bar_st_free) + (gp & 1), (gp >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
@@ -421,11 +435,19 @@ __global__ void __launch_bounds__(480, 1)
           const uint32_t dst_pair = smem_u32(sDST + (P % C::DST_BUFS) * C::DST_BYTES);
           if (!mbar_wait(bar_pt_full + pb, (g >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
+          if constexpr (C::PT_TMEM) {
+            const uint32_t pt_tmem = tmem + (g % C::NBUF) * 64;  // 16 queries = 8 columns per k-step
 #pragma unroll
-          for (int kk = 0; kk < C::TQ / 16; ++kk)
-            mma_bf16_ss(tmem + C::COL_DV + vb * 2 * D, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
-                        (jj > 0 || kk > 0));
+            for (int kk = 0; kk < C::TQ / 16; ++kk)
+              mma_bf16_ts(tmem + C::COL_DV + vb * 2 * D, pt_tmem + kk * 8, bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
+                          (jj > 0 || kk > 0));
+          } else {
+            const uint32_t pt_base = smem_u32(sPT + pb * C::PT_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < C::TQ / 16; ++kk)
+              mma_bf16_ss(tmem + C::COL_DV + vb * 2 * D, pt_kdesc(pt_base, kk), bwd_mndesc<D>(do_base, C::TQ, kk),
+                          id_kv, (jj > 0 || kk > 0));
+          }
           mma_commit(bar_pt_free + pb);
           if (!mbar_wait(bar_dst_full + pb, (g >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -489,7 +511,8 @@ __global__ void __launch_bounds__(480, 1)
         ok = ok && mbar_wait(bar_st_full + pb, (g >> 1) & 1, abort_flag);
         // P^T buffer pb is free once dV of step g-2 has completed; the dS^T
         // pair buffer once the product over pair P - DST_BUFS has.
-        if (g >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((g >> 1) - 1) & 1, abort_flag);
+        // (With P^T in TMEM, S^T_g having been computed implies dV_{g-2} is done.)
+        if (!C::PT_TMEM && g >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((g >> 1) - 1) & 1, abort_flag);
         if (P >= C::DST_BUFS)
           ok = ok && mbar_wait(bar_dst_free + (P % C::DST_BUFS), ((P / C::DST_BUFS) - 1) & 1, abort_flag);
         tc_fence_after();
@@ -504,8 +527,10 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
         for (int c16 = 0; c16 < 4; ++c16) tmem_ld16(tmem + lane_base + b * 64 + c16 * 16, sv + c16 * 16);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar_st_free + pb);
+        if constexpr (!C::PT_TMEM) {
+          tc_fence_before();
+          mbar_arrive(bar_st_free + pb);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float4 t = nlse4[i];
@@ -523,11 +548,23 @@ __global__ void __launch_bounds__(480, 1)
             if (x < kr.qlo || x > kr.qhi) sv[i] = 0.f;
           }
         }
+        if constexpr (C::PT_TMEM) {
+          // P^T row over the first 32 columns of its own S^T buffer
+          uint32_t pk[32];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(pt + sw128_offset(row, ch)) =
-              make_uint4(pack_bf16(sv[8 * ch], sv[8 * ch + 1]), pack_bf16(sv[8 * ch + 2], sv[8 * ch + 3]),
-                         pack_bf16(sv[8 * ch + 4], sv[8 * ch + 5]), pack_bf16(sv[8 * ch + 6], sv[8 * ch + 7]));
+          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(sv[2 * u], sv[2 * u + 1]);
+          tmem_st32(tmem + lane_base + b * 64, pk);
+          tmem_wait_st();
+          tc_fence_before();
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(pt + sw128_offset(row, ch)) =
+                make_uint4(pack_bf16(sv[8 * ch], sv[8 * ch + 1]), pack_bf16(sv[8 * ch + 2], sv[8 * ch + 3]),
+                           pack_bf16(sv[8 * ch + 4], sv[8 * ch + 5]), pack_bf16(sv[8 * ch + 6], sv[8 * ch + 7]));
+          fence_proxy_async_smem();
+        }
+        mbar_arrive(bar_pt_full + pb);  // dV of the step may start
         // (2) dP^T row in two halves (its TMEM buffer is released after the
         //     second); dS = P (dP - Delta) in fp32 pairs
         ok = ok && mbar_wait(bar_dpt_full + pb, (g >> 1) & 1, abort_flag);
@@ -561,7 +598,6 @@ __global__ void __launch_bounds__(480, 1)
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(bar_pt_full + pb);
         mbar_arrive(bar_dst_full + pb);
       }
       gs += it.n;

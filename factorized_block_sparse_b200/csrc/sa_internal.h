@@ -18,6 +18,9 @@ constexpr int kFwdTQ = 128;  // forward: query rows per CTA (tcgen05 M)
 constexpr int kFwdTK = 64;   // forward: keys per step (tcgen05 N of Q K^T)
 constexpr int kBwdTK = 128;  // backward: keys per CTA (tcgen05 M of K Q^T)
 constexpr int kBwdTQ = 64;   // backward: queries per step
+// Backward tables whose items average at least this many steps run the
+// kernel shape with the deeper Q/dO ring (P^T in TMEM).
+constexpr int kBwdLongSteps = 16;
 
 enum Src : int { SRC_N = 0, SRC_T = 1, SRC_S = 2 };
 
