@@ -32,6 +32,9 @@ SMALL = [
     ("local", 2, 1, 1024, 64, 100, 0, 16),      # window not aligned to blocks
     ("local", 1, 1, 512, 128, 1000, 0, 64),     # window wider than the sequence
     ("strided", 1, 1, 320, 64, 40, 0, 32),      # R = 8, ragged
+    # items of >= 16 steps on average: the LONG backward shape (P^T in TMEM)
+    ("all", 1, 1, 2112, 32, 1, 0, 64),          # D = 32, ragged last key tile
+    ("all", 2, 1, 2112, 64, 1, 0, 64),
 ]
 
 
