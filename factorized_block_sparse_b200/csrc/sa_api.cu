@@ -187,6 +187,60 @@ int make_dq_maps(CUtensorMap* nat, CUtensorMap* col, const float* base, const Ge
   return SA_OK;
 }
 
+// Maps of the dV/dK epilogue (D <= 64), boxes of 32 key rows:
+//   out_k/out_v: bf16 dK/dV [BH, N, D], natural {D, N, BH}, box {D, 32, 1}
+//   part_k/part_v: fp32 partials [BH, N, D] in the key view of the pass:
+//     natural {D, N, BH} box {32, 32, 1}; column-major {D, l, R, BH} box
+//     {32, 1, min(R, 32), 1}; summary {D, l, R, BH} box {32, min(c, 32),
+//     max(1, 32 / c), 1}; 128-byte swizzle (32 fp32 per box row).
+struct EpiMaps {
+  CUtensorMap out_k, out_v, part_k, part_v;
+};
+
+int make_epi_maps(EpiMaps* em, const void* dk, const void* dv, const float* dk_part, const float* dv_part,
+                  const Geo& g, int key_view) {
+  std::memset(em, 0, sizeof(*em));
+  if (g.D > 64) return SA_OK;  // D = 128 stores with plain instructions
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.N * g.D * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)g.D, 32, 1};
+    const auto swz = g.D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUtensorMap* outs[2] = {&em->out_k, &em->out_v};
+    const void* bases[2] = {dk, dv};
+    for (int i = 0; i < 2; ++i)
+      if (g_encode(outs[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(bases[i]), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return SA_ERR_CUDA;
+  }
+  CUtensorMap* parts[2] = {&em->part_k, &em->part_v};
+  const float* pbases[2] = {dk_part, dv_part};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r;
+    if (key_view == SRC_N) {
+      const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+      const cuuint64_t strides[2] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.N * g.D * 4};
+      const cuuint32_t box[3] = {32, 32, 1};
+      r = g_encode(parts[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(pbases[i]), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+      const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
+      const cuuint64_t strides[3] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.l * g.D * 4, (cuuint64_t)g.N * g.D * 4};
+      const cuuint32_t box[4] = {32, key_view == SRC_T ? 1u : (cuuint32_t)std::min(g.c, 32),
+                                 key_view == SRC_T ? (cuuint32_t)std::min(g.R, 32) : (cuuint32_t)std::max(1, 32 / g.c),
+                                 1};
+      r = g_encode(parts[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(pbases[i]), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
+    if (r != CUDA_SUCCESS) return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
 int make_maps(MapSet* ms, const void* base, const Geo& g, int pattern, int rows) {
   std::memset(ms, 0, sizeof(*ms));
   int st = map_nat(&ms->nat, base, g, rows);
@@ -435,6 +489,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   const int n_sm = sm_count();
   // Tables whose items average many steps take the LONG shape of the kernel.
   auto run = [&](int kind, const DevTable& t) -> int {
+    EpiMaps em;
+    const int mst = make_epi_maps(&em, dk, dv, dk_part, dv_part, g, a.key_view);
+    if (mst) return mst;
     const long long items = static_cast<long long>(t.n_rows) * g.BH;
     dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
     const bool long_items = D <= 64 && t.nnz >= kBwdLongSteps * static_cast<long long>(t.n_rows);
@@ -442,12 +499,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
       if constexpr (D <= 64) {
         if (long_items) {
           sa_bwd_kernel<D, true><<<grid, BwdCfg<D, true>::THREADS, BwdCfg<D, true>::SMEM, s>>>(
-              mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col, a);
+              mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col,
+              em.out_k, em.out_v, em.part_k, em.part_v, a);
           return;
         }
       }
       sa_bwd_kernel<D, false><<<grid, BwdCfg<D, false>::THREADS, BwdCfg<D, false>::SMEM, s>>>(
-          mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col, a);
+          mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col,
+          em.out_k, em.out_v, em.part_k, em.part_v, a);
     });
   };
   if (sec) {

@@ -106,7 +106,7 @@ struct BwdCfg {
   // 4 x DQS_WARP_BYTES; 1 KiB aligned (the 128-byte swizzle pattern is address based)
   static constexpr int OFF_DQS = (OFF_LD + STAGES * LD_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = OFF_DQS + 4 * DQS_WARP_BYTES;
-  static constexpr int N_BARS = 2 * KVB + 2 * STAGES + 2 * 7 + DST_BUFS + 2 * DQBUF + 2 * DKVB;
+  static constexpr int N_BARS = 2 * KVB + 2 * STAGES + 2 * 7 + DST_BUFS + 2 * DQBUF + 2 * DKVB + 4;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
@@ -235,6 +235,8 @@ __global__ void __launch_bounds__(480, 1)
                   const __grid_constant__ CUtensorMap mk_sum, const __grid_constant__ CUtensorMap mv_nat,
                   const __grid_constant__ CUtensorMap mv_col, const __grid_constant__ CUtensorMap mv_sum,
                   const __grid_constant__ CUtensorMap mdq_nat, const __grid_constant__ CUtensorMap mdq_col,
+                  const __grid_constant__ CUtensorMap mdk_out, const __grid_constant__ CUtensorMap mdv_out,
+                  const __grid_constant__ CUtensorMap mdk_part, const __grid_constant__ CUtensorMap mdv_part,
                   const BwdArgs a) {
   using C = BwdCfg<D, LONG>;
   extern __shared__ uint8_t smem_raw[];
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(480, 1)
   uint64_t* bar_dq_free = bar_dq_full + C::DQBUF;        // [DQBUF]
   uint64_t* bar_dkv_full = bar_dq_free + C::DQBUF;       // [DKVB] per non-empty item
   uint64_t* bar_dkv_free = bar_dkv_full + C::DKVB;       // [DKVB]
+  uint64_t* bar_epi = bar_dkv_free + C::DKVB;            // [4] partial rows landed (epilogue warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
@@ -301,6 +304,7 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(bar_dkv_full + b, 1);
       mbar_init(bar_dkv_free + b, 128);
     }
+    for (int w = 0; w < 4; ++w) mbar_init(bar_epi + w, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -608,7 +612,7 @@ __global__ void __launch_bounds__(480, 1)
     const int row = quarter * 32 + lane;  // query row of a dQ product; key row of the epilogue
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     bool ok = true;
-    int gs = 0, ne = 0, qi = 0;
+    int gs = 0, ne = 0, qi = 0, epi_n = 0;
     BwdItem nxt = (cta < n_items) ? bwd_item(a, cta) : BwdItem{0, 0, 0, 0};
     for (int k = 0, item = cta; ok && item < n_items;) {
       const BwdItem it = nxt;  // the next item's schedule entry is fetched one item ahead
@@ -689,6 +693,107 @@ __global__ void __launch_bounds__(480, 1)
         ok = ok && mbar_wait(bar_dkv_full + ne % C::DKVB, (ne / C::DKVB) & 1, abort_flag);
         tc_fence_after();
       }
+      if constexpr (C::DQ_TMA) {
+        // Through this warp's staging buffer: TMEM -> registers (+ the fp32
+        // partial rows, fetched by TMA) -> swizzled staging -> one TMA store
+        // of the warp's 32 key rows (bf16 dV/dK in the natural pass, fp32
+        // partials at the keys' natural positions in a secondary pass).
+        uint8_t* stg = smem + C::OFF_DQS + quarter * C::DQS_WARP_BYTES;
+        const int y0 = it.kt * C::TK + quarter * 32;  // first view key of the warp
+        const bool nat_out = a.key_view == SRC_N;
+        bool row_add = false;
+        if (nat_out && a.add_part == 1) row_add = kr.kvalid;
+        else if (nat_out && a.add_part == 2) row_add = kr.kvalid && (kr.knat % a.l) >= (a.l - a.c);
+        const bool warp_add = __any_sync(0xffffffffu, row_add);
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+          if (lane == 0) bulk_wait_read_all();  // earlier stores and reduces have read the staging
+          __syncwarp();
+          if (warp_add && lane == 0) {
+            mbar_arrive_expect_tx(bar_epi + quarter, 32 * D * 4);
+#pragma unroll
+            for (int bx = 0; bx < D / 32; ++bx)
+              tma_load_3d(stg + bx * 4096, which ? &mdk_part : &mdv_part, bar_epi + quarter, bx * 32, y0, it.bh);
+          }
+          const uint32_t col = (which ? C::COL_DK : C::COL_DV) + (ne % C::DKVB) * 2 * D;
+          const float mul = which ? a.scale : 1.f;
+          // 32 columns at a time; in the natural pass the bf16 row (D*2 bytes)
+          // lands over the first fp32 box, which every lane has read by then
+#pragma unroll
+          for (int h = 0; h < D / 32; ++h) {
+            float gv[32];
+            if (it.n > 0) {
+              tmem_ld16(tmem + lane_base + col + h * 32, gv);
+              tmem_ld16(tmem + lane_base + col + h * 32 + 16, gv + 16);
+              tmem_wait_ld();
+              if (which == 1 && h == D / 32 - 1) {
+                tc_fence_before();
+                mbar_arrive(bar_dkv_free + ne % C::DKVB);  // both accumulators have been read
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) gv[u] = 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 32; ++u) gv[u] *= mul;
+            if (h == 0 && warp_add) {  // the partial rows were requested before the TMEM reads
+              ok = ok && mbar_wait(bar_epi + quarter, epi_n & 1, abort_flag);
+              ++epi_n;
+            }
+            if (row_add) {
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) {
+                const float4 t = *reinterpret_cast<const float4*>(stg + h * 4096 + sw128_offset(lane, ch));
+                gv[ch * 4] += t.x;
+                gv[ch * 4 + 1] += t.y;
+                gv[ch * 4 + 2] += t.z;
+                gv[ch * 4 + 3] += t.w;
+              }
+            }
+            if (nat_out) {
+              if (h == 0 && warp_add) __syncwarp();
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4) {
+                const int ch = h * 4 + c4;  // 16-byte chunk of the bf16 row
+                const uint4 w = make_uint4(pack_bf16(gv[8 * c4], gv[8 * c4 + 1]), pack_bf16(gv[8 * c4 + 2], gv[8 * c4 + 3]),
+                                           pack_bf16(gv[8 * c4 + 4], gv[8 * c4 + 5]),
+                                           pack_bf16(gv[8 * c4 + 6], gv[8 * c4 + 7]));
+                *reinterpret_cast<uint4*>(stg + (D == 64 ? sw128_offset(lane, ch) : sw64_offset(lane, ch))) = w;
+              }
+            } else {
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<float4*>(stg + h * 4096 + sw128_offset(lane, ch)) =
+                    make_float4(gv[ch * 4], gv[ch * 4 + 1], gv[ch * 4 + 2], gv[ch * 4 + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (nat_out) {
+              tma_store_3d(which ? &mdk_out : &mdv_out, stg, 0, y0, it.bh);
+            } else {
+              const CUtensorMap* mp = which ? &mdk_part : &mdv_part;
+#pragma unroll
+              for (int bx = 0; bx < D / 32; ++bx) {
+                if (a.key_view == SRC_T) {
+                  const int rb = a.R < 32 ? a.R : 32;
+                  for (int s0 = 0; s0 < 32; s0 += rb) {
+                    const int t = y0 + s0;
+                    tma_store_4d(mp, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
+                  }
+                } else if (a.c >= 32) {
+                  tma_store_4d(mp, stg + bx * 4096, bx * 32, a.l - a.c + y0 % a.c, y0 / a.c, it.bh);
+                } else {
+                  tma_store_4d(mp, stg + bx * 4096, bx * 32, a.l - a.c, y0 / a.c, it.bh);
+                }
+              }
+            }
+            bulk_commit_group();
+          }
+        }
+        if (it.n > 0) ++ne;
+      } else {
       const size_t off = (static_cast<size_t>(it.bh) * a.N + (kr.kvalid ? kr.knat : 0)) * D;
       bool add = false;
       if (a.add_part == 1) add = true;
@@ -713,10 +818,11 @@ __global__ void __launch_bounds__(480, 1)
           store_grad_row<D, 16>(a, which, off, i * 16, gv, add);
         }
       }
-      if (it.n > 0) {
-        tc_fence_before();
-        mbar_arrive(bar_dkv_free + ne % C::DKVB);
-        ++ne;
+        if (it.n > 0) {
+          tc_fence_before();
+          mbar_arrive(bar_dkv_free + ne % C::DKVB);
+          ++ne;
+        }
       }
       gs += it.n;
     }
