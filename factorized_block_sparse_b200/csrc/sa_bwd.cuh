@@ -546,10 +546,14 @@ __global__ void __launch_bounds__(480, 1)
           sv[4 * i + 3] = ex2(x23.y);
         }
         if (partial) {
+          if constexpr (C::PT_TMEM) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int x = x0 + i;
-            if (x < kr.qlo || x > kr.qhi) sv[i] = 0.f;
+            for (int i = 0; i < 64; ++i) {
+              const int x = x0 + i;
+              if (x < kr.qlo || x > kr.qhi) sv[i] = 0.f;
+            }
+          } else {
+            mask_interval64(sv, kr.qlo - x0, kr.qhi - x0, 0.f);
           }
         }
         if constexpr (C::PT_TMEM) {

@@ -370,6 +370,24 @@ __device__ __forceinline__ void red_add_v4(float* gptr, float a, float b, float 
                : "memory");
 }
 
+// Keeps v[i] for lo <= i <= hi (i in [0, 64)) and sets the others to
+// `fill`: the interval becomes one 64-bit mask, then one bit test and one
+// select per element.
+__device__ __forceinline__ void mask_interval64(float* v, int lo, int hi, float fill) {
+  lo = max(lo, 0);
+  hi = min(hi, 63);
+  uint32_t m0 = 0u, m1 = 0u;
+  if (lo <= hi) {
+    const uint64_t m = (~0ull << lo) & (~0ull >> (63 - hi));
+    m0 = static_cast<uint32_t>(m);
+    m1 = static_cast<uint32_t>(m >> 32);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = ((m0 >> i) & 1u) ? v[i] : fill;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[32 + i] = ((m1 >> i) & 1u) ? v[32 + i] : fill;
+}
+
 // Byte offset of 16-byte chunk `chunk` of row `row` in a K-major tile whose
 // rows are 128 bytes (64 bf16) wide, swizzled 128B (8-row atoms of 1 KiB).
 __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {

@@ -286,11 +286,8 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
         const int k0 = (e >> 3) * C::TK;
         const int lo = src == SRC_N ? lo_n : (src == SRC_T ? lo_t : lo_s);
         const int hi = src == SRC_N ? hi_n : (src == SRC_T ? hi_t : hi_s);
-#pragma unroll
-        for (int i = 0; i < C::TK; ++i) {
-          const int key = k0 + i;
-          if (key < lo || key > hi) s[i] = -INFINITY;
-        }
+        static_assert(C::TK == 64, "interval mask of 64 keys");
+        mask_interval64(s, lo - k0, hi - k0, -INFINITY);
       }
       // row max as a tree (short dependency chains)
       float mx8[8];
