@@ -64,8 +64,11 @@ struct BwdArgs {
 };
 
 // Two shapes of the same kernel.  LONG is for tables whose items run many
-// steps (D <= 64): P^T is written into TMEM over its own S^T columns and dV
-// is a TS-MMA with A read from TMEM, S^T/dP^T are double-buffered, and
+// steps (D <= 64): P^T is written into TMEM over the second half of its
+// step's dP^T columns (once the elementwise thread holds that row in
+// registers) and dV is a TS-MMA with A read from TMEM; the dP^T buffer then
+// stays busy until dV completes, which is off the S^T -> exp -> dV loop
+// (S^T is released as soon as it is read).  S^T/dP^T are double-buffered, and
 // there is one dV/dK and one K/V buffer (an item boundary costs a short
 // stall), so the shared memory of the P^T buffers and of the second K/V
 // buffer goes to a deeper Q/dO ring.  The other shape keeps P^T in shared
@@ -378,10 +381,7 @@ __global__ void __launch_bounds__(480, 1)
           const int b = g % C::NBUF;
           ok = mbar_wait(bar_qdo_full + st, (g / C::STAGES) & 1, abort_flag);
           const int gp = g - C::NBUF;  // last user of TMEM buffer b
-          // the S^T buffer is free once it has been read out or, when it
-          // holds P^T, once dV of that step has completed
-          if (ok && gp >= 0)
-            ok = mbar_wait((C::PT_TMEM ? bar_pt_free : bar_st_free) + (gp & 1), (gp >> 1) & 1, abort_flag);
+          if (ok && gp >= 0) ok = mbar_wait(bar_st_free + (gp & 1), (gp >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t q_base = smem_u32(sQ + st * C::QS_BYTES);
@@ -391,7 +391,10 @@ __global__ void __launch_bounds__(480, 1)
             mma_bf16_ss(tmem + b * 64, bwd_kdesc<D>(k_base, C::TK, kk), bwd_kdesc<D>(q_base, C::TQ, kk), id_s,
                         kk > 0);
           mma_commit(bar_st_full + (g & 1));
-          if (gp >= 0 && !mbar_wait(bar_dpt_free + (gp & 1), (gp >> 1) & 1, abort_flag)) {
+          // the dP^T buffer is free once it has been read out or, when it
+          // holds P^T (LONG shape), once dV of that step has completed
+          if (gp >= 0 &&
+              !mbar_wait((C::PT_TMEM ? bar_pt_free : bar_dpt_free) + (gp & 1), (gp >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -440,7 +443,7 @@ __global__ void __launch_bounds__(480, 1)
           if (!mbar_wait(bar_pt_full + pb, (g >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           if constexpr (C::PT_TMEM) {
-            const uint32_t pt_tmem = tmem + (g % C::NBUF) * 64;  // 16 queries = 8 columns per k-step
+            const uint32_t pt_tmem = tmem + C::COL_DPT + (g % C::NBUF) * 64 + 32;  // 8 columns per k-step
 #pragma unroll
             for (int kk = 0; kk < C::TQ / 16; ++kk)
               mma_bf16_ts(tmem + C::COL_DV + vb * 2 * D, pt_tmem + kk * 8, bwd_mndesc<D>(do_base, C::TQ, kk), id_kv,
@@ -515,7 +518,6 @@ __global__ void __launch_bounds__(480, 1)
         ok = ok && mbar_wait(bar_st_full + pb, (g >> 1) & 1, abort_flag);
         // P^T buffer pb is free once dV of step g-2 has completed; the dS^T
         // pair buffer once the product over pair P - DST_BUFS has.
-        // (With P^T in TMEM, S^T_g having been computed implies dV_{g-2} is done.)
         if (!C::PT_TMEM && g >= 2) ok = ok && mbar_wait(bar_pt_free + pb, ((g >> 1) - 1) & 1, abort_flag);
         if (P >= C::DST_BUFS)
           ok = ok && mbar_wait(bar_dst_free + (P % C::DST_BUFS), ((P / C::DST_BUFS) - 1) & 1, abort_flag);
@@ -531,10 +533,8 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
         for (int c16 = 0; c16 < 4; ++c16) tmem_ld16(tmem + lane_base + b * 64 + c16 * 16, sv + c16 * 16);
         tmem_wait_ld();
-        if constexpr (!C::PT_TMEM) {
-          tc_fence_before();
-          mbar_arrive(bar_st_free + pb);
-        }
+        tc_fence_before();
+        mbar_arrive(bar_st_free + pb);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float4 t = nlse4[i];
@@ -556,25 +556,19 @@ __global__ void __launch_bounds__(480, 1)
             mask_interval64(sv, kr.qlo - x0, kr.qhi - x0, 0.f);
           }
         }
-        if constexpr (C::PT_TMEM) {
-          // P^T row over the first 32 columns of its own S^T buffer
-          uint32_t pk[32];
-#pragma unroll
-          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(sv[2 * u], sv[2 * u + 1]);
-          tmem_st32(tmem + lane_base + b * 64, pk);
-          tmem_wait_st();
-          tc_fence_before();
-        } else {
+        if constexpr (!C::PT_TMEM) {
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch)
             *reinterpret_cast<uint4*>(pt + sw128_offset(row, ch)) =
                 make_uint4(pack_bf16(sv[8 * ch], sv[8 * ch + 1]), pack_bf16(sv[8 * ch + 2], sv[8 * ch + 3]),
                            pack_bf16(sv[8 * ch + 4], sv[8 * ch + 5]), pack_bf16(sv[8 * ch + 6], sv[8 * ch + 7]));
           fence_proxy_async_smem();
+          mbar_arrive(bar_pt_full + pb);  // dV of the step may start
         }
-        mbar_arrive(bar_pt_full + pb);  // dV of the step may start
         // (2) dP^T row in two halves (its TMEM buffer is released after the
-        //     second); dS = P (dP - Delta) in fp32 pairs
+        //     second; in the LONG shape P^T is written over the second half
+        //     once both are in registers, and dV releases the buffer);
+        //     dS = P (dP - Delta) in fp32 pairs
         ok = ok && mbar_wait(bar_dpt_full + pb, (g >> 1) & 1, abort_flag);
         tc_fence_after();
 #pragma unroll
@@ -584,8 +578,22 @@ __global__ void __launch_bounds__(480, 1)
           tmem_ld16(tmem + lane_base + C::COL_DPT + b * 64 + hh * 32 + 16, dp + 16);
           tmem_wait_ld();
           if (hh == 1) {
-            tc_fence_before();
-            mbar_arrive(bar_dpt_free + pb);
+            if constexpr (C::PT_TMEM) {
+              const uint32_t pt_cols = tmem + lane_base + C::COL_DPT + b * 64 + 32;
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) pk[u] = pack_bf16(sv[16 * q8 + 2 * u], sv[16 * q8 + 2 * u + 1]);
+                tmem_st8(pt_cols + q8 * 8, pk);
+              }
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(bar_pt_full + pb);  // dV of the step may start
+            } else {
+              tc_fence_before();
+              mbar_arrive(bar_dpt_free + pb);
+            }
           }
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
