@@ -357,6 +357,12 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   if ((st = make_maps(&mq, q, g, L->pattern, FwdCfg<D>::TQ))) return st;
   if ((st = make_maps(&mk, k, g, L->pattern, FwdCfg<D>::TK))) return st;
   if ((st = make_maps(&mv, v, g, L->pattern, FwdCfg<D>::TK))) return st;
+  // Output maps of the epilogue: 32-row boxes, natural and column-major.
+  CUtensorMap mo_nat, mo_col;
+  std::memset(&mo_col, 0, sizeof(mo_col));
+  if ((st = map_nat(&mo_nat, o, g, 32))) return st;
+  if (L->pattern == SA_STRIDED && (st = map_grid(&mo_col, o, g, 1, static_cast<uint32_t>(std::min(g.R, 32)))))
+    return st;
   DeviceCopy dc;
   if ((st = to_device(L, &dc))) return st;
   auto kern = sa_fwd_kernel<D>;
@@ -379,7 +385,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     a.merge = 0;
     dim3 grid(g.BH, dc.fwd_col.n_rows);
     st = launch(K_FWD_COL * 4 + L->pattern, s, [&] {
-      kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
+      kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum,
+                                                                       mo_nat, mo_col, a);
     });
     if (st) return st;
   }
@@ -390,7 +397,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.merge = (two_pass && dc.fwd_col.n_rows > 0) ? 1 : 0;
   dim3 grid(g.BH, dc.fwd_main.n_rows);
   return launch(K_FWD_MAIN * 4 + L->pattern, s, [&] {
-    kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, a);
+    kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum,
+                                                                       mo_nat, mo_col, a);
   });
 }
 

@@ -60,7 +60,9 @@ struct FwdCfg {
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_ENT = OFF_V + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_ENT + kMaxStagedEnt * 4;
-  static constexpr int N_BARS = 1 + 3 * STAGES + 8;
+  static constexpr int N_BARS = 1 + 3 * STAGES + 8 + 4;
+  // The epilogue stages each warp's 32 output rows in the K ring.
+  static_assert(STAGES * KV_BYTES >= TQ * D * 2, "epilogue staging");
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 256;
@@ -129,6 +131,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
                   const __grid_constant__ CUtensorMap mk_nat, const __grid_constant__ CUtensorMap mk_col,
                   const __grid_constant__ CUtensorMap mk_sum, const __grid_constant__ CUtensorMap mv_nat,
                   const __grid_constant__ CUtensorMap mv_col, const __grid_constant__ CUtensorMap mv_sum,
+                  const __grid_constant__ CUtensorMap mo_nat, const __grid_constant__ CUtensorMap mo_col,
                   const FwdArgs a) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -145,6 +148,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
   uint64_t* bar_s_empty = bar_s_full + 2;           // [2]  PV of the buffer's tile done
   uint64_t* bar_p_full = bar_s_empty + 2;           // [2]  P written into TMEM
   uint64_t* bar_pv_done = bar_p_full + 2;           // [2]
+  uint64_t* bar_epi = bar_pv_done + 2;              // [4]  old O rows of a merge landed (per warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   int32_t* sEnt = reinterpret_cast<int32_t*>(smem + C::OFF_ENT);
@@ -171,6 +175,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
       mbar_init(bar_p_full + s, 128);
       mbar_init(bar_pv_done + s, 1);
     }
+    for (int w = 0; w < 4; ++w) mbar_init(bar_epi + w, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -356,7 +361,6 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
       tc_fence_after();
     }
     float w_new = 1.f, w_old = 0.f, lse_out = lse_row;
-    const size_t row_off = (static_cast<size_t>(bh) * a.N + (valid ? nat : 0)) * D;
     if (a.merge && valid) {
       const float lse_old = a.lse[static_cast<size_t>(bh) * a.N + nat];
       const float mm = fmaxf(lse_row, lse_old);
@@ -372,6 +376,21 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
         lse_out = mm + lg2(tot) * 0.6931471805599453f;
       }
     }
+    // Rows go out through this warp's slice of the K ring (idle once the
+    // last S product is done): a merge first brings the stored O rows in by
+    // TMA, each thread blends its own row in place, and one TMA store per
+    // warp (per 64-column panel) writes the 32 rows in the tile's view order.
+    uint8_t* stg = sK + quarter * (32 * D * 2);
+    constexpr int PB = 32 * C::ROWB;  // one 32-row panel
+    const int xw = qt * C::TQ + quarter * 32;  // view position of the warp's first row
+    if (a.merge) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_epi + quarter, 32 * D * 2);
+#pragma unroll
+        for (int p = 0; p < C::PANELS; ++p) tma_load_3d(stg + p * PB, &mo_nat, bar_epi + quarter, p * 64, xw, bh);
+      }
+      ok = ok && mbar_wait(bar_epi + quarter, 0, abort_flag);
+    }
 #pragma unroll
     for (int i = 0; i < D / 16; ++i) {
       float ov[16];
@@ -382,38 +401,51 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
 #pragma unroll
         for (int u = 0; u < 16; ++u) ov[u] = 0.f;
       }
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(a.o + row_off + i * 16);
-        float old[16];
-        if (a.merge) {
-          const uint4 o0 = dst[0], o1 = dst[1];
-          const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&o0);
-          const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&o1);
+      // the two 16-byte chunks of columns [16i, 16i + 16) in the swizzled row
+      const int ch = (i * 2) % (C::ROWB / 16);
+      const int pnl = (i * 16) / 64;
+      uint8_t* c0 = stg + (D >= 64 ? pnl * PB + sw128_offset(lane, ch) : sw64_offset(lane, ch));
+      uint8_t* c1 = stg + (D >= 64 ? pnl * PB + sw128_offset(lane, ch + 1) : sw64_offset(lane, ch + 1));
+      float r[16];
+      if (a.merge) {
+        const uint4 o0 = *reinterpret_cast<const uint4*>(c0), o1 = *reinterpret_cast<const uint4*>(c1);
+        const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&o0);
+        const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&o1);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 f0 = __bfloat1622float2(h0[u]);
-            const float2 f1 = __bfloat1622float2(h1[u]);
-            old[2 * u] = f0.x;
-            old[2 * u + 1] = f0.y;
-            old[8 + 2 * u] = f1.x;
-            old[8 + 2 * u + 1] = f1.y;
-          }
+        for (int u = 0; u < 4; ++u) {
+          const float2 f0 = __bfloat1622float2(h0[u]);
+          const float2 f1 = __bfloat1622float2(h1[u]);
+          r[2 * u] = w_new * ov[2 * u] * inv + w_old * f0.x;
+          r[2 * u + 1] = w_new * ov[2 * u + 1] * inv + w_old * f0.y;
+          r[8 + 2 * u] = w_new * ov[8 + 2 * u] * inv + w_old * f1.x;
+          r[8 + 2 * u + 1] = w_new * ov[8 + 2 * u + 1] * inv + w_old * f1.y;
         }
-        float r[16];
+      } else {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) r[u] = a.merge ? (w_new * ov[u] * inv + w_old * old[u]) : ov[u] * inv;
-        uint4 w0, w1;
-        w0.x = pack_bf16(r[0], r[1]);
-        w0.y = pack_bf16(r[2], r[3]);
-        w0.z = pack_bf16(r[4], r[5]);
-        w0.w = pack_bf16(r[6], r[7]);
-        w1.x = pack_bf16(r[8], r[9]);
-        w1.y = pack_bf16(r[10], r[11]);
-        w1.z = pack_bf16(r[12], r[13]);
-        w1.w = pack_bf16(r[14], r[15]);
-        dst[0] = w0;
-        dst[1] = w1;
+        for (int u = 0; u < 16; ++u) r[u] = ov[u] * inv;
       }
+      *reinterpret_cast<uint4*>(c0) =
+          make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]), pack_bf16(r[6], r[7]));
+      *reinterpret_cast<uint4*>(c1) = make_uint4(pack_bf16(r[8], r[9]), pack_bf16(r[10], r[11]),
+                                                 pack_bf16(r[12], r[13]), pack_bf16(r[14], r[15]));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int p = 0; p < C::PANELS; ++p) {
+        if (a.q_col) {
+          const int rb = a.R < 32 ? a.R : 32;
+          for (int s0 = 0; s0 < 32; s0 += rb) {
+            const int t = xw + s0;
+            tma_store_4d(&mo_col, stg + p * PB + s0 * C::ROWB, p * 64, t / a.R, t % a.R, bh);
+          }
+        } else {
+          tma_store_3d(&mo_nat, stg + p * PB, p * 64, xw, bh);
+        }
+      }
+      bulk_commit_group();
+      bulk_wait_all();
     }
     if (valid) a.lse[static_cast<size_t>(bh) * a.N + nat] = lse_out;
   }
