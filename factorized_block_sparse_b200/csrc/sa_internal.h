@@ -20,7 +20,7 @@ constexpr int kBwdTK = 128;  // backward: keys per CTA (tcgen05 M of K Q^T)
 constexpr int kBwdTQ = 64;   // backward: queries per step
 // Backward tables whose items average at least this many steps run the
 // kernel shape with the deeper Q/dO ring (P^T in TMEM).
-constexpr int kBwdLongSteps = 16;
+constexpr int kBwdLongSteps = 4;
 
 enum Src : int { SRC_N = 0, SRC_T = 1, SRC_S = 2 };
 
