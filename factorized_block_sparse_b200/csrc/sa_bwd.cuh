@@ -600,14 +600,28 @@ __global__ void __launch_bounds__(480, 1)
             const int c0 = hh * 32 + cc * 8;  // first of 8 columns
             const float4 d0 = ndel4[c0 / 4], d1 = ndel4[c0 / 4 + 1];
             const int l0 = cc * 8;
-            const float2 s01 = f2_unpack(f2_mul(f2_pack(sv[c0], sv[c0 + 1]),
-                                                f2_add(f2_pack(dp[l0], dp[l0 + 1]), f2_pack(d0.x, d0.y))));
-            const float2 s23 = f2_unpack(f2_mul(f2_pack(sv[c0 + 2], sv[c0 + 3]),
-                                                f2_add(f2_pack(dp[l0 + 2], dp[l0 + 3]), f2_pack(d0.z, d0.w))));
-            const float2 s45 = f2_unpack(f2_mul(f2_pack(sv[c0 + 4], sv[c0 + 5]),
-                                                f2_add(f2_pack(dp[l0 + 4], dp[l0 + 5]), f2_pack(d1.x, d1.y))));
-            const float2 s67 = f2_unpack(f2_mul(f2_pack(sv[c0 + 6], sv[c0 + 7]),
-                                                f2_add(f2_pack(dp[l0 + 6], dp[l0 + 7]), f2_pack(d1.z, d1.w))));
+            float2 s01, s23, s45, s67;
+            if constexpr (C::PT_TMEM) {
+              // scalar form: in this shape it compiles to a faster step than
+              // the packed pairs (same arithmetic)
+              const float nd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+              float ds[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) ds[u] = sv[c0 + u] * (dp[l0 + u] + nd[u]);
+              s01 = make_float2(ds[0], ds[1]);
+              s23 = make_float2(ds[2], ds[3]);
+              s45 = make_float2(ds[4], ds[5]);
+              s67 = make_float2(ds[6], ds[7]);
+            } else {
+              s01 = f2_unpack(f2_mul(f2_pack(sv[c0], sv[c0 + 1]),
+                                     f2_add(f2_pack(dp[l0], dp[l0 + 1]), f2_pack(d0.x, d0.y))));
+              s23 = f2_unpack(f2_mul(f2_pack(sv[c0 + 2], sv[c0 + 3]),
+                                     f2_add(f2_pack(dp[l0 + 2], dp[l0 + 3]), f2_pack(d0.z, d0.w))));
+              s45 = f2_unpack(f2_mul(f2_pack(sv[c0 + 4], sv[c0 + 5]),
+                                     f2_add(f2_pack(dp[l0 + 4], dp[l0 + 5]), f2_pack(d1.x, d1.y))));
+              s67 = f2_unpack(f2_mul(f2_pack(sv[c0 + 6], sv[c0 + 7]),
+                                     f2_add(f2_pack(dp[l0 + 6], dp[l0 + 7]), f2_pack(d1.z, d1.w))));
+            }
             *reinterpret_cast<uint4*>(dst + sw128_offset(row, c0 / 8)) =
                 make_uint4(pack_bf16(s01.x, s01.y), pack_bf16(s23.x, s23.y), pack_bf16(s45.x, s45.y),
                            pack_bf16(s67.x, s67.y));
