@@ -67,6 +67,63 @@ def flops(w, counts):
     return 4 * per * nnz, 10 * per * nnz
 
 
+def element_nnz(w):
+    """(query, key) pairs per head in the workload's mask (element level)."""
+    import numpy as np
+
+    N, l, c, mode = w["N"], w["l"], w["c"], w["mode"]
+    i = np.arange(N, dtype=np.int64)
+    if mode == "all":
+        return N * (N + 1) // 2
+    if mode == "local":
+        return int(np.minimum(i + 1, l).sum())
+    if mode == "strided":  # window of l (diagonal included) + earlier positions of the column
+        return int(np.minimum(i + 1, l).sum() + (i // l).sum())
+    if mode == "fixed":  # own block (causal) + the last c offsets of every earlier block
+        return int(((i % l) + 1).sum() + ((i // l) * c).sum())
+    raise ValueError(mode)
+
+
+def algorithmic_bytes(w):
+    """Minimal HBM bytes of forward + backward: q, k, v read and o, lse written (forward); q, k, v, o,
+    dO, lse read and dq, dk, dv written (backward); the strided merge re-reads and re-writes o, lse."""
+    D, rows = w["D"], w["B"] * w["H"] * w["N"]
+    b = rows * ((8 * D + 4) + (16 * D + 4))
+    if w["mode"] == "strided":
+        b += rows * (4 * D + 8)
+    return b
+
+
+def workload_lines(state, ktimes, pk):
+    """Per-workload kernel time (sum of its kernels' mean launch times, CUDA events), throughput
+    and fraction of the workload's own roofline max(flops / bf16 peak, algorithmic bytes / HBM peak)."""
+    modes = [s["w"]["mode"] for s in state]
+    if len(set(modes)) != len(modes):
+        return None  # kernel times are kept per pattern
+    out = {}
+    for s in state:
+        w, m = s["w"], s["w"]["mode"]
+        t = {"fwd": 0.0, "bwd": 0.0}
+        for name, (ms, c) in ktimes.items():
+            if c and name.endswith("." + m):
+                t["fwd" if name.startswith("sa_fwd") else "bwd"] += ms / c
+        ms = t["fwd"] + t["bwd"]
+        fl = s["flops"]
+        el = element_nnz(w) * w["B"] * w["H"] * 14 * w["D"]  # 4D (QK^T, PV) + 10D (backward) per pair
+        by = algorithmic_bytes(w)
+        t_tc = fl / (pk["bf16"] * 1e12) * 1e3
+        t_hbm = by / (pk["hbm"] * 1e9) * 1e3
+        out[s["name"]] = {
+            "fwd_ms": round(t["fwd"], 4), "bwd_ms": round(t["bwd"], 4),
+            "nonzero_block_tflops": round(fl / (ms * 1e-3) / 1e12, 2),
+            "element_tflops": round(el / (ms * 1e-3) / 1e12, 2),
+            "tokens_per_s": round(w["B"] * w["N"] / (ms * 1e-3), 1),
+            "roofline": {"bound": "tensor" if t_tc >= t_hbm else "hbm", "tensor_ms": round(t_tc, 4),
+                         "hbm_ms": round(t_hbm, 4), "frac": round(max(t_tc, t_hbm) / ms, 4)},
+        }
+    return out
+
+
 def kernel_units(w, counts):
     """Algorithmic work per launch of each kernel of a workload (flops or bytes)."""
     per = w["block"] ** 2 * w["D"] * w["B"] * w["H"]
@@ -334,7 +391,8 @@ def main():
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         ws = sa.workspace(w["B"], w["H"], w["N"], w["D"], lay, dev)
         lay.upload()
-        state.append(dict(w=w, lay=lay, x=x, q=q, k=k, v=v, dO=dO, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws))
+        state.append(dict(w=w, name=n, flops=f0 + f1, lay=lay, x=x, q=q, k=k, v=v, dO=dO, o=o, lse=lse, dq=dq,
+                          dk=dk, dv=dv, ws=ws))
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
 
@@ -421,6 +479,7 @@ def main():
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": "burst (of measured)" if pk["source"] == "measured" else "fallback"},
         "kernels": kernels,
+        "workloads": workload_lines(state, ktimes, pk),
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
