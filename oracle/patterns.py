@@ -27,12 +27,22 @@ Definitions, and the reading of the pages they follow:
 
 The two component heads of each factorized pattern (used for the
 two-step reachability property of "Factorized Attention Patterns") are
-exposed as ``component_heads``.
+exposed as ``component_heads``.  The pages also describe running the two
+parts as separate heads, each with its own softmax (same section: heads
+that attend to the row and to the column, or to the own block and to the
+summary cells).  Two of those heads are modes of their own:
+
+* ``column``  - the strided pattern's column head: every earlier position
+  of the same column and the position itself, ``(i - j) mod l == 0``.
+  Its row head is ``local``.
+* ``block``   - the fixed pattern's own-block head, ``j // l == i // l``,
+  causal.
+Both contain the diagonal, so no row is empty.
 """
 
 import numpy as np
 
-MODES = ("all", "local", "strided", "fixed")
+MODES = ("all", "local", "strided", "fixed", "column", "block")
 
 
 def _check(mode, N, l, c):
@@ -40,7 +50,7 @@ def _check(mode, N, l, c):
         raise ValueError(f"unknown mode {mode!r}")
     if N < 1:
         raise ValueError("N must be >= 1")
-    if mode in ("local", "strided", "fixed") and l < 1:
+    if mode in ("local", "strided", "fixed", "column", "block") and l < 1:
         raise ValueError("l must be >= 1")
     if mode == "fixed" and not (0 <= c <= l):
         raise ValueError("fixed needs 0 <= c <= l")
@@ -60,6 +70,10 @@ def pair_mask(mode, l, c, i, j):
         return causal & ((d < l) | (d % l == 0))
     if mode == "fixed":
         return causal & ((j // l == i // l) | (j % l >= l - c))
+    if mode == "column":
+        return causal & (d % l == 0)
+    if mode == "block":
+        return causal & (j // l == i // l)
     raise ValueError(f"unknown mode {mode!r}")
 
 

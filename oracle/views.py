@@ -26,6 +26,11 @@ into disjoint views, each dense in its own relabelled order:
   The view holds the summary keys of strictly earlier blocks,
   ``j // l < i // l``.  Summary keys of the own block are in view ``N``.
 
+The two single-head modes use one view each: ``column`` the column-major
+view ``T`` with the diagonal included (``i - j >= 0``, ``(i - j) mod l ==
+0``: there is no natural view to hold it), ``block`` the natural view of
+``fixed``.
+
 Block table of a view: cut its (queries x keys) matrix, in view order,
 into ``block x block`` tiles (a ragged last tile is padded with
 "not in mask").  A tile is present when any element is in the mask; it
@@ -50,6 +55,8 @@ def views_of(mode):
         return ("N", "T")
     if mode == "fixed":
         return ("N", "S")
+    if mode == "column":
+        return ("T",)
     return ("N",)
 
 
@@ -73,9 +80,11 @@ def _natural_view_predicate(view, mode, l, c, i, j):
             return causal
         if mode in ("local", "strided"):
             return causal & (i - j < l)
-        return causal & (j // l == i // l)  # fixed
+        return causal & (j // l == i // l)  # fixed, block
     if view == "T":
         d = i - j
+        if mode == "column":
+            return (d >= 0) & (d % l == 0)
         return (d > 0) & (d % l == 0)
     if view == "S":
         return (j // l < i // l) & (j % l >= l - c)

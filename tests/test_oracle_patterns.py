@@ -149,7 +149,8 @@ def test_summary_view_is_block_prefix():
 
 @pytest.mark.parametrize("mode,N,l,c", [("all", 64, 1, 0), ("local", 64, 6, 0),
                                         ("strided", 64, 8, 0), ("strided", 60, 6, 0),
-                                        ("fixed", 64, 8, 2), ("fixed", 72, 12, 5)])
+                                        ("fixed", 64, 8, 2), ("fixed", 72, 12, 5),
+                                        ("column", 64, 8, 0), ("column", 60, 6, 0), ("block", 64, 8, 0)])
 def test_views_partition_the_mask(mode, N, l, c):
     full = patterns.mask(mode, N, l, c)
     acc = np.zeros((N, N), np.int64)
@@ -185,7 +186,9 @@ def _brute_table(M, b):
 
 @pytest.mark.parametrize("mode,N,l,c,b", [("all", 64, 1, 0, 8), ("local", 64, 12, 0, 8),
                                           ("strided", 64, 8, 0, 4), ("strided", 96, 12, 0, 8),
-                                          ("fixed", 96, 12, 4, 8), ("fixed", 64, 16, 3, 4)])
+                                          ("fixed", 96, 12, 4, 8), ("fixed", 64, 16, 3, 4),
+                                          ("column", 64, 8, 0, 4), ("column", 96, 12, 0, 8),
+                                          ("block", 96, 12, 0, 8)])
 def test_block_tables_brute_force(mode, N, l, c, b):
     for v in views.views_of(mode):
         tab = views.block_table(v, mode, N, l, c, b)
