@@ -36,6 +36,8 @@ from factorized_block_sparse_b200 import synth  # noqa: E402
 METRIC = "fwd+bwd nonzero-block TFLOP/s (% of B200 BF16 peak) and tokens/s at N=12288"
 STEPS = {
     "n12288": ["text-fixed", "image64-strided"],
+    # the strided image64 pattern as two heads (row head + column head, own softmax each)
+    "image64-two-head": ["image64-local", "image64-column"],
 }
 for _n in synth.WORKLOADS:
     STEPS[_n] = [_n]
@@ -56,7 +58,7 @@ def block_counts(w, sa=None):
     """Nonzero public blocks per view of a workload (from the library's table)."""
     if sa is not None:
         lay = sa.Layout(w["mode"], w["N"], w["l"], w["c"], w["block"])
-        views = {"strided": ("N", "T"), "fixed": ("N", "S")}.get(w["mode"], ("N",))
+        views = {"strided": ("N", "T"), "fixed": ("N", "S"), "column": ("T",)}.get(w["mode"], ("N",))
         return {v: len(lay.export(v)["col_idx"]) for v in views}, lay
     raise ValueError("library needed")
 
@@ -81,6 +83,10 @@ def element_nnz(w):
         return int(np.minimum(i + 1, l).sum() + (i // l).sum())
     if mode == "fixed":  # own block (causal) + the last c offsets of every earlier block
         return int(((i % l) + 1).sum() + ((i // l) * c).sum())
+    if mode == "column":  # earlier positions of the column and the position itself
+        return int((i // l + 1).sum())
+    if mode == "block":  # own block, causal
+        return int(((i % l) + 1).sum())
     raise ValueError(mode)
 
 
@@ -131,14 +137,15 @@ def kernel_units(w, counts):
     D = w["D"]
     m = w["mode"]
     sec = counts.get("T", 0) + counts.get("S", 0)
-    fwd_main = counts["N"] + (counts.get("S", 0) if m == "fixed" else 0)
+    fwd_main = counts.get("N", 0) + (counts.get("S", 0) if m == "fixed" else 0)
     out = {
-        f"sa_fwd_natural_view.{m}": ("tensor", 4 * per * fwd_main),
-        f"sa_bwd_natural_view.{m}": ("tensor", 10 * per * counts["N"]),
         f"sa_bwd_preprocess.{m}": ("hbm", rows * (2 * D * 2 + 4)),
         f"sa_bwd_finalize_dq.{m}": ("hbm", rows * D * (4 + 2)),
     }
-    if m == "strided":
+    if "N" in counts:
+        out[f"sa_fwd_natural_view.{m}"] = ("tensor", 4 * per * fwd_main)
+        out[f"sa_bwd_natural_view.{m}"] = ("tensor", 10 * per * counts["N"])
+    if "T" in counts:
         out[f"sa_fwd_column_view.{m}"] = ("tensor", 4 * per * counts["T"])
     if sec:
         out[f"sa_bwd_secondary_view.{m}"] = ("tensor", 10 * per * sec)

@@ -29,16 +29,18 @@ enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_F
 const char* const kKernelNames[K_KERNELS] = {"sa_fwd_column_view", "sa_fwd_natural_view",
                                              "sa_bwd_preprocess",  "sa_bwd_secondary_view",
                                              "sa_bwd_natural_view", "sa_bwd_finalize_dq"};
-const char* const kPatternNames[4] = {"all", "local", "strided", "fixed"};
+constexpr int K_PATTERNS = 6;
+const char* const kPatternNames[K_PATTERNS] = {"all", "local", "strided", "fixed", "column", "block"};
 // Instrumentation kinds: one per (kernel, pattern), kind = kernel * 4 + pattern.
-constexpr int K_NUM = K_KERNELS * 4;
+constexpr int K_NUM = K_KERNELS * K_PATTERNS;
 char g_kind_names[K_NUM][48];
 std::once_flag g_names_once;
 
 const char* kind_name(int kind) {
   std::call_once(g_names_once, [] {
     for (int k = 0; k < K_NUM; ++k)
-      std::snprintf(g_kind_names[k], sizeof(g_kind_names[k]), "%s.%s", kKernelNames[k / 4], kPatternNames[k % 4]);
+      std::snprintf(g_kind_names[k], sizeof(g_kind_names[k]), "%s.%s", kKernelNames[k / K_PATTERNS],
+                    kPatternNames[k % K_PATTERNS]);
   });
   return g_kind_names[kind];
 }
@@ -175,7 +177,7 @@ int make_dq_maps(CUtensorMap* nat, CUtensorMap* col, const float* base, const Ge
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return SA_ERR_CUDA;
   }
-  if (pattern == SA_STRIDED) {
+  if (pattern == SA_STRIDED || pattern == SA_COLUMN) {
     const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
     const cuuint64_t strides[3] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.l * g.D * 4, (cuuint64_t)g.N * g.D * 4};
     const cuuint32_t box[4] = {32, 1, (cuuint32_t)std::min(g.R, 32), 1};
@@ -189,6 +191,8 @@ int make_dq_maps(CUtensorMap* nat, CUtensorMap* col, const float* base, const Ge
 
 // Maps of the dV/dK epilogue (D <= 64), boxes of 32 key rows:
 //   out_k/out_v: bf16 dK/dV [BH, N, D], natural {D, N, BH}, box {D, 32, 1}
+//     (column-major {D, l, R, BH}, box {D, 1, min(R, 32), 1}, for a
+//     column-view pass that writes final outputs)
 //   part_k/part_v: fp32 partials [BH, N, D] in the key view of the pass:
 //     natural {D, N, BH} box {32, 32, 1}; column-major {D, l, R, BH} box
 //     {32, 1, min(R, 32), 1}; summary {D, l, R, BH} box {32, min(c, 32),
@@ -203,17 +207,28 @@ int make_epi_maps(EpiMaps* em, const void* dk, const void* dv, const float* dk_p
   if (g.D > 64) return SA_OK;  // D = 128 stores with plain instructions
   const cuuint32_t es[4] = {1, 1, 1, 1};
   {
-    const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.N, (cuuint64_t)g.BH};
-    const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.N * g.D * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)g.D, 32, 1};
     const auto swz = g.D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap* outs[2] = {&em->out_k, &em->out_v};
     const void* bases[2] = {dk, dv};
-    for (int i = 0; i < 2; ++i)
-      if (g_encode(outs[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(bases[i]), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return SA_ERR_CUDA;
+    for (int i = 0; i < 2; ++i) {
+      CUresult r;
+      if (key_view == SRC_T) {  // column-major rows: {D, l, R, BH}, box {D, 1, min(R, 32), 1}
+        const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
+        const cuuint64_t strides[3] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.l * g.D * 2, (cuuint64_t)g.N * g.D * 2};
+        const cuuint32_t box[4] = {(cuuint32_t)g.D, 1, (cuuint32_t)std::min(g.R, 32), 1};
+        r = g_encode(outs[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(bases[i]), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      } else {
+        const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+        const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.N * g.D * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)g.D, 32, 1};
+        r = g_encode(outs[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(bases[i]), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      }
+      if (r != CUDA_SUCCESS) return SA_ERR_CUDA;
+    }
   }
   CUtensorMap* parts[2] = {&em->part_k, &em->part_v};
   const float* pbases[2] = {dk_part, dv_part};
@@ -245,7 +260,7 @@ int make_maps(MapSet* ms, const void* base, const Geo& g, int pattern, int rows)
   std::memset(ms, 0, sizeof(*ms));
   int st = map_nat(&ms->nat, base, g, rows);
   if (st) return st;
-  if (pattern == SA_STRIDED) {
+  if (pattern == SA_STRIDED || pattern == SA_COLUMN) {
     st = map_grid(&ms->col, base, g, 1, (uint32_t)std::min(g.R, rows));
     if (st) return st;
   }
@@ -316,7 +331,7 @@ int check_call(int B, int H, int N, int D, const sa_layout* L) {
   if (static_cast<long long>(B) * H > 0x7fffffffLL) return SA_ERR_INVALID_ARG;
   if (L->N != N) return SA_ERR_LUT;
   if (D != 32 && D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
-  if (L->pattern == SA_STRIDED) {
+  if (L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) {
     const int R = L->R;
     if (R % 8 != 0 || !(R % 128 == 0 || 128 % R == 0)) return SA_ERR_UNSUPPORTED;
   }
@@ -335,7 +350,7 @@ Geo make_geo(int B, int H, int N, int D, const sa_layout* L) {
   g.D = D;
   g.l = (L->pattern == SA_ALL) ? 1 : L->l;
   g.c = L->c > 0 ? L->c : 1;
-  g.R = (L->pattern == SA_STRIDED || L->pattern == SA_FIXED) ? L->R : 1;
+  g.R = (L->pattern == SA_STRIDED || L->pattern == SA_FIXED || L->pattern == SA_COLUMN) ? L->R : 1;
   g.boxw = D >= 64 ? 64 : D;
   g.swz = D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   return g;
@@ -361,7 +376,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   CUtensorMap mo_nat, mo_col;
   std::memset(&mo_col, 0, sizeof(mo_col));
   if ((st = map_nat(&mo_nat, o, g, 32))) return st;
-  if (L->pattern == SA_STRIDED && (st = map_grid(&mo_col, o, g, 1, static_cast<uint32_t>(std::min(g.R, 32)))))
+  if ((L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) &&
+      (st = map_grid(&mo_col, o, g, 1, static_cast<uint32_t>(std::min(g.R, 32)))))
     return st;
   DeviceCopy dc;
   if ((st = to_device(L, &dc))) return st;
@@ -376,15 +392,17 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.R = g.R;
   a.pattern = L->pattern;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  const bool two_pass = (L->pattern == SA_STRIDED);
-  if (two_pass && dc.fwd_col.n_rows > 0) {
+  // Column view first (SA_STRIDED, SA_COLUMN); the natural view then merges
+  // into its result (SA_STRIDED) or runs alone (the other patterns).
+  const bool col_pass = dc.fwd_col.n_rows > 0;
+  if (col_pass) {
     a.row_ptr = dc.fwd_col.row_ptr;
     a.ent = dc.fwd_col.ent;
     a.order = dc.fwd_col.order;
     a.q_col = 1;
     a.merge = 0;
     dim3 grid(g.BH, dc.fwd_col.n_rows);
-    st = launch(K_FWD_COL * 4 + L->pattern, s, [&] {
+    st = launch(K_FWD_COL * K_PATTERNS + L->pattern, s, [&] {
       kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum,
                                                                        mo_nat, mo_col, a);
     });
@@ -394,9 +412,10 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.ent = dc.fwd_main.ent;
   a.order = dc.fwd_main.order;
   a.q_col = 0;
-  a.merge = (two_pass && dc.fwd_col.n_rows > 0) ? 1 : 0;
+  a.merge = col_pass ? 1 : 0;
+  if (dc.fwd_main.n_rows == 0) return SA_OK;  // SA_COLUMN: no natural view
   dim3 grid(g.BH, dc.fwd_main.n_rows);
-  return launch(K_FWD_MAIN * 4 + L->pattern, s, [&] {
+  return launch(K_FWD_MAIN * K_PATTERNS + L->pattern, s, [&] {
     kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum,
                                                                        mo_nat, mo_col, a);
   });
@@ -426,7 +445,7 @@ WsLayout ws_layout(int B, int H, int N, int D, const sa_layout* L) {
   const size_t ld_bytes = align256(BH * w.n_pad * 8);  // two floats per query position
   w.ld_nat = 0;
   w.ld_col = ld_bytes;
-  const bool col = L->pattern == SA_STRIDED;
+  const bool col = L->pattern == SA_STRIDED || L->pattern == SA_COLUMN;
   w.dq = w.ld_col + (col ? ld_bytes : 0);
   w.dk = w.dq + align256(rows * D * 4);
   const bool sec = L->pattern == SA_STRIDED || L->pattern == SA_FIXED;
@@ -461,7 +480,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* ld_nat = reinterpret_cast<float*>(wsb + w.ld_nat);
-  float* ld_col = (L->pattern == SA_STRIDED) ? reinterpret_cast<float*>(wsb + w.ld_col) : nullptr;
+  float* ld_col = (L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) ? reinterpret_cast<float*>(wsb + w.ld_col)
+                                                                        : nullptr;
   float* dq_acc = reinterpret_cast<float*>(wsb + w.dq);
   float* dk_part = reinterpret_cast<float*>(wsb + w.dk);
   float* dv_part = reinterpret_cast<float*>(wsb + w.dv);
@@ -469,7 +489,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   CUtensorMap mdq_nat, mdq_col;
   if ((st = make_dq_maps(&mdq_nat, &mdq_col, dq_acc, g, L->pattern))) return st;
 
-  st = launch(K_BWD_PRE * 4 + L->pattern, s, [&] {
+  st = launch(K_BWD_PRE * K_PATTERNS + L->pattern, s, [&] {
     sa_bwd_pre_kernel<D><<<grid_for(rows * (D / 8), 256), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ld_nat, ld_col, dq_acc,
         g.BH, N, w.n_pad, g.l, g.R);
@@ -492,7 +512,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.pattern = L->pattern;
   a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  const bool sec = (L->pattern == SA_STRIDED || L->pattern == SA_FIXED) && dc.bwd_sec.n_rows > 0;
+  const bool sec = dc.bwd_sec.n_rows > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN
+  // SA_COLUMN has no natural view: its column-view pass writes the final dK/dV.
+  const bool sec_final = L->pattern == SA_COLUMN;
   a.BH = g.BH;
   const int n_sm = sm_count();
   // Tables whose items average many steps take the LONG shape of the kernel.
@@ -521,18 +543,22 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.sched = dc.bwd_sec.sched;
     a.ent = dc.bwd_sec.ent;
     a.n_slots = dc.bwd_sec.n_rows;
-    a.key_view = (L->pattern == SA_STRIDED) ? SRC_T : SRC_S;
+    a.key_view = (L->pattern == SA_FIXED) ? SRC_S : SRC_T;
     a.add_part = 0;
-    if ((st = run(K_BWD_SEC * 4 + L->pattern, dc.bwd_sec))) return st;
+    a.final_out = sec_final ? 1 : 0;
+    if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec))) return st;
   }
-  a.sched = dc.bwd_main.sched;
-  a.ent = dc.bwd_main.ent;
-  a.n_slots = dc.bwd_main.n_rows;
-  a.key_view = SRC_N;
-  a.add_part = sec ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
-  if ((st = run(K_BWD_MAIN * 4 + L->pattern, dc.bwd_main))) return st;
+  if (dc.bwd_main.n_rows > 0) {
+    a.sched = dc.bwd_main.sched;
+    a.ent = dc.bwd_main.ent;
+    a.n_slots = dc.bwd_main.n_rows;
+    a.key_view = SRC_N;
+    a.add_part = (sec && !sec_final) ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
+    a.final_out = 1;
+    if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main))) return st;
+  }
   const long long n8 = rows * D / 8;
-  return launch(K_BWD_FINAL * 4 + L->pattern, s, [&] {
+  return launch(K_BWD_FINAL * K_PATTERNS + L->pattern, s, [&] {
     sa_bwd_final_kernel<<<grid_for(n8, 256), 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
   });
 }
@@ -548,11 +574,12 @@ extern "C" {
 int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** out) {
   if (!out) return SA_ERR_INVALID_ARG;
   *out = nullptr;
-  if (pattern < SA_ALL || pattern > SA_FIXED || N < 1 || block < 1) return SA_ERR_INVALID_ARG;
+  if (pattern < SA_ALL || pattern > SA_BLOCK || N < 1 || block < 1) return SA_ERR_INVALID_ARG;
   if (pattern != SA_ALL && l < 1) return SA_ERR_INVALID_ARG;
   if (pattern == SA_FIXED && (c < 1 || c > l)) return SA_ERR_INVALID_ARG;
   if (N % block != 0) return SA_ERR_UNSUPPORTED;
-  if ((pattern == SA_STRIDED || pattern == SA_FIXED) && N % l != 0) return SA_ERR_UNSUPPORTED;
+  const bool grid2d = pattern == SA_STRIDED || pattern == SA_FIXED || pattern == SA_COLUMN;  // R = N / l rows
+  if (grid2d && N % l != 0) return SA_ERR_UNSUPPORTED;
   sa_layout* L = new (std::nothrow) sa_layout();
   if (!L) return SA_ERR_INVALID_ARG;
   L->pattern = pattern;
@@ -560,7 +587,7 @@ int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** 
   L->l = (pattern == SA_ALL) ? 1 : l;
   L->c = (pattern == SA_FIXED) ? c : 0;
   L->block = block;
-  L->R = (pattern == SA_STRIDED || pattern == SA_FIXED) ? N / l : 1;
+  L->R = grid2d ? N / l : 1;
   const int st = build_layout(L);
   if (st != SA_OK) {
     delete L;

@@ -59,6 +59,7 @@ struct BwdArgs {
   int pattern;
   int key_view;  // SRC_N, SRC_T or SRC_S
   int add_part;  // main pass: add secondary partials (1 strided: all keys; 2 fixed: summary keys)
+  int final_out; // 1: write bf16 dK/dV (natural pass; SA_COLUMN's column pass), 0: fp32 partials
   float scale;       // 1/sqrt(D)
   float scale_log2;  // log2(e)/sqrt(D)
 };
@@ -178,7 +179,7 @@ __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
   else if (a.key_view == SRC_S) k.knat = (k.y / a.c) * a.l + (a.l - a.c) + k.y % a.c;
   else k.knat = k.y;
   if (a.key_view == SRC_T) {
-    k.qlo = k.y + 1;
+    k.qlo = (a.pattern == SA_COLUMN) ? k.y : k.y + 1;  // the column head keeps its diagonal
     k.qhi = (k.y / a.R) * a.R + a.R - 1;
   } else if (a.key_view == SRC_S) {
     k.qlo = (k.y / a.c + 1) * a.l;
@@ -186,7 +187,7 @@ __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
   } else {
     k.qlo = k.y;
     if (a.pattern == SA_ALL) k.qhi = a.N - 1;
-    else if (a.pattern == SA_FIXED) k.qhi = (k.y / a.l) * a.l + a.l - 1;
+    else if (a.pattern == SA_FIXED || a.pattern == SA_BLOCK) k.qhi = (k.y / a.l) * a.l + a.l - 1;
     else k.qhi = k.y + a.l - 1;
   }
   if (k.qhi > a.N - 1) k.qhi = a.N - 1;
@@ -200,7 +201,7 @@ __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
 template <int D, int NC>
 __device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size_t off, int c0, float* g,
                                                bool add) {
-  if (a.key_view != SRC_N) {
+  if (!a.final_out) {
     float* dstp = (which ? a.dk_part : a.dv_part) + off + c0;
 #pragma unroll
     for (int u = 0; u < NC; u += 4)
@@ -726,7 +727,7 @@ __global__ void __launch_bounds__(480, 1)
         // partials at the keys' natural positions in a secondary pass).
         uint8_t* stg = smem + C::OFF_DQS + quarter * C::DQS_WARP_BYTES;
         const int y0 = it.kt * C::TK + quarter * 32;  // first view key of the warp
-        const bool nat_out = a.key_view == SRC_N;
+        const bool nat_out = a.final_out;  // bf16 rows (else fp32 partials)
         bool row_add = false;
         if (nat_out && a.add_part == 1) row_add = kr.kvalid;
         else if (nat_out && a.add_part == 2) row_add = kr.kvalid && (kr.knat % a.l) >= (a.l - a.c);
@@ -796,7 +797,13 @@ __global__ void __launch_bounds__(480, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (nat_out) {
+            if (nat_out && a.key_view == SRC_T) {  // SA_COLUMN: rows of the column runs
+              const int rb = a.R < 32 ? a.R : 32;
+              for (int s0 = 0; s0 < 32; s0 += rb) {
+                const int t = y0 + s0;
+                tma_store_4d(which ? &mdk_out : &mdv_out, stg + s0 * (D * 2), 0, t / a.R, t % a.R, it.bh);
+              }
+            } else if (nat_out) {
               tma_store_3d(which ? &mdk_out : &mdv_out, stg, 0, y0, it.bh);
             } else {
               const CUtensorMap* mp = which ? &mdk_part : &mdv_part;

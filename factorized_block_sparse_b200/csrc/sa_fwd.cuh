@@ -264,13 +264,13 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
     int lo_n, hi_n;
     if (a.pattern == SA_ALL) {
       lo_n = 0;
-    } else if (a.pattern == SA_FIXED) {
+    } else if (a.pattern == SA_FIXED || a.pattern == SA_BLOCK) {
       lo_n = (nat / a.l) * a.l;
     } else {
       lo_n = max(0, nat - a.l + 1);
     }
     hi_n = nat;
-    const int lo_t = (x / a.R) * a.R, hi_t = x - 1;
+    const int lo_t = (x / a.R) * a.R, hi_t = (a.pattern == SA_COLUMN) ? x : x - 1;  // column head: diagonal too
     const int lo_s = 0, hi_s = (nat / a.l) * a.c - 1;
 
     float m_used = -INFINITY;

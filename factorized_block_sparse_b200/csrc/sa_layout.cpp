@@ -38,12 +38,12 @@ Interval key_interval(const sa_layout* L, int view, long long x) {
       case SA_LOCAL:
       case SA_STRIDED:
         return {std::max(0LL, x - l + 1), x};
-      default:  // SA_FIXED: own l-block, causal
+      default:  // SA_FIXED, SA_BLOCK: own l-block, causal
         return {(x / l) * l, x};
     }
   }
-  if (view == SA_VIEW_COLUMN) {  // strict, inside the column run of length R
-    return {(x / R) * R, x - 1};
+  if (view == SA_VIEW_COLUMN) {  // inside the column run of length R; strict unless the
+    return {(x / R) * R, L->pattern == SA_COLUMN ? x : x - 1};  // view stands alone
   }
   // SA_VIEW_SUMMARY: summary keys of strictly earlier blocks
   return {0, (x / l) * c - 1};
@@ -193,8 +193,8 @@ int view_keys(const sa_layout* L, int view) {
 
 int build_layout(sa_layout* L) {
   const int p = L->pattern;
-  L->has[SA_VIEW_NATURAL] = true;
-  L->has[SA_VIEW_COLUMN] = (p == SA_STRIDED);
+  L->has[SA_VIEW_NATURAL] = (p != SA_COLUMN);
+  L->has[SA_VIEW_COLUMN] = (p == SA_STRIDED || p == SA_COLUMN);
   L->has[SA_VIEW_SUMMARY] = (p == SA_FIXED);
   for (int v = 0; v < 3; ++v) {
     if (!L->has[v]) continue;
@@ -205,7 +205,7 @@ int build_layout(sa_layout* L) {
   const int b = L->block;
 
   // Forward, natural query tiles: summary entries first (fixed), then natural.
-  {
+  if (L->has[SA_VIEW_NATURAL]) {
     auto nat = coarsen(L->view[SA_VIEW_NATURAL], b, kFwdTQ, kFwdTK, N, N);
     std::vector<CoarseRow> sum;
     if (L->has[SA_VIEW_SUMMARY])
@@ -217,6 +217,8 @@ int build_layout(sa_layout* L) {
       for (auto& e : nat[r].ent) rows[r].push_back(pack_entry(e.first, SRC_N, e.second));
     }
     finish_table(L->fwd_main, rows);
+  } else {
+    finish_table(L->fwd_main, {});
   }
   // Forward, column-order query tiles (strided).
   if (L->has[SA_VIEW_COLUMN]) {
@@ -229,12 +231,14 @@ int build_layout(sa_layout* L) {
     finish_table(L->fwd_col, {});
   }
   // Backward, natural key tiles -> natural query tiles.
-  {
+  if (L->has[SA_VIEW_NATURAL]) {
     auto kt = coarsen(L->viewT[SA_VIEW_NATURAL], b, kBwdTK, kBwdTQ, N, N);
     std::vector<std::vector<int32_t>> rows(kt.size());
     for (size_t r = 0; r < kt.size(); ++r)
       for (auto& e : kt[r].ent) rows[r].push_back(pack_entry(e.first, SRC_N, e.second));
     finish_table(L->bwd_main, rows);
+  } else {
+    finish_table(L->bwd_main, {});
   }
   // Backward, secondary view key tiles (T order or summary order).
   if (L->has[SA_VIEW_COLUMN] || L->has[SA_VIEW_SUMMARY]) {

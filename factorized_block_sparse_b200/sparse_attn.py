@@ -15,7 +15,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
 
-PATTERNS = {"all": 0, "local": 1, "strided": 2, "fixed": 3}
+PATTERNS = {"all": 0, "local": 1, "strided": 2, "fixed": 3, "column": 4, "block": 5}
 VIEWS = {"N": 0, "T": 1, "S": 2}
 VIEW_TRANSPOSED = 4
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_LUT, SA_ERR_TIMEOUT, SA_ERR_WORKSPACE = range(7)

@@ -31,6 +31,9 @@ WORKLOADS = {
     "image64-all": dict(mode="all", B=1, H=16, N=12288, D=64, l=192, c=0, block=64),
     # raw audio, 65536 samples
     "audio-strided": dict(mode="strided", B=1, H=4, N=65536, D=64, l=256, c=0, block=64),
+    # the image64 strided pattern in its two-head form: row head and column head
+    "image64-local": dict(mode="local", B=1, H=16, N=12288, D=64, l=192, c=0, block=64),
+    "image64-column": dict(mode="column", B=1, H=16, N=12288, D=64, l=192, c=0, block=64),
 }
 
 

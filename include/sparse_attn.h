@@ -22,6 +22,15 @@
  *   SA_STRIDED  0 <= i - j < l  or  (i - j) mod l == 0    (row + column)
  *   SA_FIXED    j <= i and ( j / l == i / l  or  j mod l >= l - c )
  *               (own l-block + the last c "summary" offsets of each block)
+ *   SA_COLUMN   j <= i and (i - j) mod l == 0
+ *               (the column head of SA_STRIDED run as a head of its own;
+ *               its row head is SA_LOCAL)
+ *   SA_BLOCK    j <= i and j / l == i / l
+ *               (the own-block head of SA_FIXED run as a head of its own)
+ * SA_COLUMN and SA_BLOCK are the two-head form of the factorized patterns:
+ * the two parts of a pattern in separate heads, each with its own softmax
+ * ("OpenAI Sparse Transformer", "Factorized Attention Patterns"; pcnews
+ * translation, "Разреженное внимание").
  *
  * The backward pass recomputes P from the saved lse and never stores an
  * N x N matrix, the memory-saving recomputation of "Generating Long
@@ -53,15 +62,17 @@ extern "C" {
 
 typedef struct sa_layout sa_layout; /* opaque, owned by the library */
 
-enum sa_pattern { SA_ALL = 0, SA_LOCAL = 1, SA_STRIDED = 2, SA_FIXED = 3 };
+enum sa_pattern { SA_ALL = 0, SA_LOCAL = 1, SA_STRIDED = 2, SA_FIXED = 3, SA_COLUMN = 4, SA_BLOCK = 5 };
 
 /* Views of a pattern.  Each view is dense in its own relabelled order:
- *   SA_VIEW_NATURAL : natural order, queries and keys (every pattern).
- *   SA_VIEW_COLUMN  : strided only.  Positions relabelled column-major,
- *       t(p) = (p mod l) * R + p / l with R = N / l; holds the strictly
- *       earlier positions of the same column (attending along a column is
- *       attending along a row of the transposed 2-D array: pcnews
- *       translation, "Разреженное внимание").
+ *   SA_VIEW_NATURAL : natural order, queries and keys (every pattern but
+ *       SA_COLUMN).
+ *   SA_VIEW_COLUMN  : SA_STRIDED and SA_COLUMN.  Positions relabelled
+ *       column-major, t(p) = (p mod l) * R + p / l with R = N / l; holds the
+ *       strictly earlier positions of the same column (attending along a
+ *       column is attending along a row of the transposed 2-D array: pcnews
+ *       translation, "Разреженное внимание"), and for SA_COLUMN, which has
+ *       no natural view, the position itself too.
  *   SA_VIEW_SUMMARY : fixed only.  Queries natural; keys are the summary
  *       positions j mod l >= l - c numbered consecutively,
  *       sigma(j) = (j / l) * c + (j mod l - (l - c)); holds the summary keys
@@ -105,7 +116,7 @@ enum sa_block_kind { SA_BLOCK_FULL = 0, SA_BLOCK_PARTIAL = 1 };
  * Arguments: pattern (sa_pattern); N >= 1 sequence length; l >= 1 row
  * length / window (ignored for SA_ALL); c summary columns, 1 <= c <= l
  * (SA_FIXED only, ignored otherwise); block >= 1 with N % block == 0.
- * SA_STRIDED and SA_FIXED need N % l == 0.  *out receives a layout the
+ * SA_STRIDED, SA_FIXED and SA_COLUMN need N % l == 0.  *out receives a layout the
  * caller releases with sparse_attn_layout_free.
  * Errors: SA_ERR_INVALID_ARG (bad pattern, sizes, null out),
  * SA_ERR_UNSUPPORTED (N % block or N % l not zero).
@@ -139,7 +150,8 @@ void sparse_attn_layout_free(sa_layout* layout);
  * sparse_attn_fwd - forward pass.  Writes o [B,H,N,D] (bf16) and lse
  * [B,H,N] (fp32, natural log).  For SA_STRIDED the column view runs first
  * and its partial result is merged exactly (log-sum-exp) into the natural
- * view's.  layout must have been built for this N.
+ * view's; SA_COLUMN runs the column view alone.  layout must have been
+ * built for this N.
  * Errors: SA_ERR_INVALID_ARG (null pointer, B/H < 1), SA_ERR_LUT (layout N
  * differs), SA_ERR_UNSUPPORTED (D not 32/64/128, column geometry the
  * kernels do not tile: R = N/l must be a multiple of 8 and divide or be

@@ -62,6 +62,10 @@ def test_argument_errors(sa):
     assert L(0, 64, 1, 0, 0, ctypes.byref(h)) == sa.SA_ERR_INVALID_ARG
     assert L(0, 60, 1, 0, 16, ctypes.byref(h)) == sa.SA_ERR_UNSUPPORTED   # N % block
     assert L(2, 64, 12, 0, 16, ctypes.byref(h)) == sa.SA_ERR_UNSUPPORTED  # N % l
+    assert L(4, 64, 12, 0, 16, ctypes.byref(h)) == sa.SA_ERR_UNSUPPORTED  # column: N % l
+    assert L(6, 64, 8, 0, 16, ctypes.byref(h)) == sa.SA_ERR_INVALID_ARG   # no pattern 6
+    assert L(5, 64, 12, 0, 16, ctypes.byref(h)) == sa.SA_OK               # block: any l
+    sa.lib.sparse_attn_layout_free(h)
     assert L(0, 64, 1, 0, 16, None) == sa.SA_ERR_INVALID_ARG
     lay = sa.Layout("strided", 256, 16, 0, 16)
     n = ctypes.c_int()
@@ -78,7 +82,7 @@ def test_argument_errors(sa):
     assert sa.lib.sparse_attn_fwd(fake, fake, fake, fake, fake, 0, 1, 256, 32, lay.handle, None) \
         == sa.SA_ERR_INVALID_ARG
     assert sa.strerror(sa.SA_ERR_TIMEOUT) == "device-side wait timed out"
-    assert sa.lib.sparse_attn_kernel_kinds() == 24
+    assert sa.lib.sparse_attn_kernel_kinds() == 36  # 6 kernels x 6 patterns
 
 
 def _compare(sa, mode, N, l, c, b, rows=None):
@@ -133,6 +137,9 @@ def test_layout_bit_exact_audio_sampled_rows(sa):
     ("strided", 64, 8, 0, 3 * 0 + 4), ("strided", 96, 6, 0, 48),
     ("fixed", 128, 16, 16, 16), ("fixed", 128, 16, 1, 8), ("fixed", 144, 12, 5, 16),
     ("fixed", 96, 24, 3, 48), ("fixed", 64, 64, 8, 16),
+    ("column", 128, 16, 0, 16), ("column", 144, 12, 0, 8), ("column", 128, 1, 0, 16),
+    ("column", 128, 128, 0, 16), ("column", 96, 6, 0, 48),
+    ("block", 128, 16, 0, 16), ("block", 120, 7, 0, 8), ("block", 64, 64, 0, 16), ("block", 96, 1, 0, 8),
 ])
 def test_layout_bit_exact_degenerate_and_ragged(sa, mode, N, l, c, b):
     _compare(sa, mode, N, l, c, b)

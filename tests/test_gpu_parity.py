@@ -35,6 +35,14 @@ SMALL = [
     # items of >= 16 steps on average: the LONG backward shape (P^T in TMEM)
     ("all", 1, 1, 2112, 32, 1, 0, 64),          # D = 32, ragged last key tile
     ("all", 2, 1, 2112, 64, 1, 0, 64),
+    # single-head modes: the strided column head and the fixed own-block head
+    ("column", 1, 2, 2048, 64, 64, 0, 64),      # R = 32: four columns per 128-key tile
+    ("column", 1, 1, 1024, 32, 8, 0, 32),       # R = 128: one column per tile
+    ("column", 2, 1, 2048, 128, 16, 0, 64),     # D = 128, R = 128
+    ("column", 1, 1, 4096, 64, 16, 0, 64),      # R = 256: two tiles per column
+    ("block", 1, 2, 1024, 64, 128, 0, 64),
+    ("block", 2, 1, 960, 32, 100, 0, 64),       # l does not divide N
+    ("block", 1, 1, 1024, 128, 256, 0, 64),
 ]
 
 
@@ -86,6 +94,7 @@ def _sampled(name, n_rows=12, n_cols=6, slices=((0, 0),), seed=0):
 
 
 @pytest.mark.parametrize("name", ["image32-strided", "text-fixed", "image64-strided", "image64-all",
+                                  "image64-local", "image64-column",
                                   "audio-strided"])
 def test_parity_full_size_sampled(cuda_device, name):
     w = synth.WORKLOADS[name]

@@ -59,6 +59,10 @@ def _closed_form(mode, N, l, c):
         return l * (l + 1) // 2 + (N - l) * l
     if mode == "strided":
         return l * (l + 1) // 2 + (N - l) * l + l * m * (m - 1) // 2
+    if mode == "column":
+        return N + l * m * (m - 1) // 2
+    if mode == "block":
+        return m * l * (l + 1) // 2
     return m * l * (l + 1) // 2 + c * l * m * (m - 1) // 2
 
 
