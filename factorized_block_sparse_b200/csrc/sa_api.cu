@@ -390,7 +390,9 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.l = g.l;
   a.c = g.c;
   a.R = g.R;
-  a.pattern = L->pattern;
+  // the kernels see SA_BLOCK as SA_FIXED: the same natural view, no summary view
+  a.pattern = (L->pattern == SA_BLOCK) ? SA_FIXED : L->pattern;
+  a.t_open = (L->pattern == SA_COLUMN) ? 0 : 1;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   // Column view first (SA_STRIDED, SA_COLUMN); the natural view then merges
   // into its result (SA_STRIDED) or runs alone (the other patterns).
@@ -473,9 +475,11 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = make_maps(&mv, v, g, L->pattern, BwdCfg<D>::TK))) return st;
   DeviceCopy dc;
   if ((st = to_device(L, &dc))) return st;
-  if ((st = set_smem(sa_bwd_kernel<D, false>, BwdCfg<D, false>::SMEM))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, false, false>, BwdCfg<D, false>::SMEM))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, false, true>, BwdCfg<D, false>::SMEM))) return st;
   if constexpr (D <= 64) {
-    if ((st = set_smem(sa_bwd_kernel<D, true>, BwdCfg<D, true>::SMEM))) return st;
+    if ((st = set_smem(sa_bwd_kernel<D, true, false>, BwdCfg<D, true>::SMEM))) return st;
+    if ((st = set_smem(sa_bwd_kernel<D, true, true>, BwdCfg<D, true>::SMEM))) return st;
   }
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -509,7 +513,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.l = g.l;
   a.c = g.c;
   a.R = g.R;
-  a.pattern = L->pattern;
+  // the kernels see SA_BLOCK as SA_FIXED: the same natural view, no summary view
+  a.pattern = (L->pattern == SA_BLOCK) ? SA_FIXED : L->pattern;
   a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   const bool sec = dc.bwd_sec.n_rows > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN
@@ -525,18 +530,23 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     const long long items = static_cast<long long>(t.n_rows) * g.BH;
     dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
     const bool long_items = D <= 64 && t.nnz >= kBwdLongSteps * static_cast<long long>(t.n_rows);
+    const bool final_t = sec_final && a.key_view == SRC_T;
+    auto go = [&](auto kernel, int threads, int smem) {
+      kernel<<<grid, threads, smem, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col,
+                                         mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v, em.part_k, em.part_v, a);
+    };
     return launch(kind, s, [&] {
       if constexpr (D <= 64) {
         if (long_items) {
-          sa_bwd_kernel<D, true><<<grid, BwdCfg<D, true>::THREADS, BwdCfg<D, true>::SMEM, s>>>(
-              mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col,
-              em.out_k, em.out_v, em.part_k, em.part_v, a);
+          using CL = BwdCfg<D, true>;
+          if (final_t) go(sa_bwd_kernel<D, true, true>, CL::THREADS, CL::SMEM);
+          else go(sa_bwd_kernel<D, true, false>, CL::THREADS, CL::SMEM);
           return;
         }
       }
-      sa_bwd_kernel<D, false><<<grid, BwdCfg<D, false>::THREADS, BwdCfg<D, false>::SMEM, s>>>(
-          mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col,
-          em.out_k, em.out_v, em.part_k, em.part_v, a);
+      using CS = BwdCfg<D, false>;
+      if (final_t) go(sa_bwd_kernel<D, false, true>, CS::THREADS, CS::SMEM);
+      else go(sa_bwd_kernel<D, false, false>, CS::THREADS, CS::SMEM);
     });
   };
   if (sec) {
@@ -545,7 +555,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_sec.n_rows;
     a.key_view = (L->pattern == SA_FIXED) ? SRC_S : SRC_T;
     a.add_part = 0;
-    a.final_out = sec_final ? 1 : 0;
     if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec))) return st;
   }
   if (dc.bwd_main.n_rows > 0) {
@@ -554,7 +563,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_main.n_rows;
     a.key_view = SRC_N;
     a.add_part = (sec && !sec_final) ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
-    a.final_out = 1;
     if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main))) return st;
   }
   const long long n8 = rows * D / 8;

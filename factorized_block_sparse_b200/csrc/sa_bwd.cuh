@@ -59,7 +59,6 @@ struct BwdArgs {
   int pattern;
   int key_view;  // SRC_N, SRC_T or SRC_S
   int add_part;  // main pass: add secondary partials (1 strided: all keys; 2 fixed: summary keys)
-  int final_out; // 1: write bf16 dK/dV (natural pass; SA_COLUMN's column pass), 0: fp32 partials
   float scale;       // 1/sqrt(D)
   float scale_log2;  // log2(e)/sqrt(D)
 };
@@ -169,7 +168,9 @@ struct KeyRow {
   bool kvalid;
 };
 
-template <int D>
+// T_DIAG: the column view holds the diagonal (SA_COLUMN, whose column view
+// stands alone); otherwise it is strict (SA_STRIDED).
+template <int D, bool T_DIAG>
 __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
   KeyRow k;
   k.y = kt * BwdCfg<D>::TK + row;
@@ -179,7 +180,7 @@ __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
   else if (a.key_view == SRC_S) k.knat = (k.y / a.c) * a.l + (a.l - a.c) + k.y % a.c;
   else k.knat = k.y;
   if (a.key_view == SRC_T) {
-    k.qlo = (a.pattern == SA_COLUMN) ? k.y : k.y + 1;  // the column head keeps its diagonal
+    k.qlo = T_DIAG ? k.y : k.y + 1;
     k.qhi = (k.y / a.R) * a.R + a.R - 1;
   } else if (a.key_view == SRC_S) {
     k.qlo = (k.y / a.c + 1) * a.l;
@@ -187,7 +188,7 @@ __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
   } else {
     k.qlo = k.y;
     if (a.pattern == SA_ALL) k.qhi = a.N - 1;
-    else if (a.pattern == SA_FIXED || a.pattern == SA_BLOCK) k.qhi = (k.y / a.l) * a.l + a.l - 1;
+    else if (a.pattern == SA_FIXED) k.qhi = (k.y / a.l) * a.l + a.l - 1;  // also SA_BLOCK (same view)
     else k.qhi = k.y + a.l - 1;
   }
   if (k.qhi > a.N - 1) k.qhi = a.N - 1;
@@ -200,8 +201,8 @@ __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
 // (secondary pass).  g holds NC fp32 values, already scaled.
 template <int D, int NC>
 __device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size_t off, int c0, float* g,
-                                               bool add) {
-  if (!a.final_out) {
+                                               bool partial_out, bool add) {
+  if (partial_out) {
     float* dstp = (which ? a.dk_part : a.dv_part) + off + c0;
 #pragma unroll
     for (int u = 0; u < NC; u += 4)
@@ -231,7 +232,9 @@ __device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size
   }
 }
 
-template <int D, bool LONG>
+// FINAL_T: the pass writes final bf16 dK/dV in column-major order (the
+// column view of SA_COLUMN, which has no natural view).
+template <int D, bool LONG, bool FINAL_T>
 __global__ void __launch_bounds__(480, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mdo_nat, const __grid_constant__ CUtensorMap mdo_col,
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(480, 1)
       item = zigzag_item(++k, cta, n_ctas);
       if (item < n_items) nxt = bwd_item(a, item);
       if (it.n == 0) continue;
-      const KeyRow kr = key_row<D>(a, it.kt, row);
+      const KeyRow kr = key_row<D, FINAL_T>(a, it.kt, row);
       for (int j = (half - gs) & 1; j < it.n; j += 2) {
         const int g = gs + j;
         const int e = a.ent[it.e0 + j];
@@ -715,7 +718,7 @@ __global__ void __launch_bounds__(480, 1)
         ++qi;
       }
       // ---- dV / dK of this item (thread = key row)
-      const KeyRow kr = key_row<D>(a, it.kt, row);
+      const KeyRow kr = key_row<D, FINAL_T>(a, it.kt, row);
       if (it.n > 0) {
         ok = ok && mbar_wait(bar_dkv_full + ne % C::DKVB, (ne / C::DKVB) & 1, abort_flag);
         tc_fence_after();
@@ -727,7 +730,7 @@ __global__ void __launch_bounds__(480, 1)
         // partials at the keys' natural positions in a secondary pass).
         uint8_t* stg = smem + C::OFF_DQS + quarter * C::DQS_WARP_BYTES;
         const int y0 = it.kt * C::TK + quarter * 32;  // first view key of the warp
-        const bool nat_out = a.final_out;  // bf16 rows (else fp32 partials)
+        const bool nat_out = a.key_view == SRC_N || FINAL_T;  // bf16 rows (else fp32 partials)
         bool row_add = false;
         if (nat_out && a.add_part == 1) row_add = kr.kvalid;
         else if (nat_out && a.add_part == 2) row_add = kr.kvalid && (kr.knat % a.l) >= (a.l - a.c);
@@ -797,7 +800,7 @@ __global__ void __launch_bounds__(480, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (nat_out && a.key_view == SRC_T) {  // SA_COLUMN: rows of the column runs
+            if constexpr (FINAL_T) {  // rows of the column runs
               const int rb = a.R < 32 ? a.R : 32;
               for (int s0 = 0; s0 < 32; s0 += rb) {
                 const int t = y0 + s0;
@@ -848,7 +851,7 @@ __global__ void __launch_bounds__(480, 1)
           if (!kr.kvalid) continue;
 #pragma unroll
           for (int u = 0; u < 16; ++u) gv[u] *= mul;
-          store_grad_row<D, 16>(a, which, off, i * 16, gv, add);
+          store_grad_row<D, 16>(a, which, off, i * 16, gv, a.key_view != SRC_N && !FINAL_T, add);
         }
       }
         if (it.n > 0) {

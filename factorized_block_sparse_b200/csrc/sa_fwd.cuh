@@ -41,6 +41,7 @@ struct FwdArgs {
   int pattern;  // sa_pattern
   int q_col;    // 1: query tiles are in column-major (T) order
   int merge;    // 1: combine with the partial (o, lse) already stored
+  int t_open;   // column view: 1 when it excludes the diagonal (SA_STRIDED), 0 when it stands alone
   float scale_log2;
 };
 
@@ -264,13 +265,13 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
     int lo_n, hi_n;
     if (a.pattern == SA_ALL) {
       lo_n = 0;
-    } else if (a.pattern == SA_FIXED || a.pattern == SA_BLOCK) {
+    } else if (a.pattern == SA_FIXED) {  // also SA_BLOCK (same natural view)
       lo_n = (nat / a.l) * a.l;
     } else {
       lo_n = max(0, nat - a.l + 1);
     }
     hi_n = nat;
-    const int lo_t = (x / a.R) * a.R, hi_t = (a.pattern == SA_COLUMN) ? x : x - 1;  // column head: diagonal too
+    const int lo_t = (x / a.R) * a.R, hi_t = x - a.t_open;
     const int lo_s = 0, hi_s = (nat / a.l) * a.c - 1;
 
     float m_used = -INFINITY;
