@@ -365,7 +365,7 @@ int set_smem(K kernel, int bytes) {
 
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-             const sa_layout* L, cudaStream_t s) {
+             float scale, const sa_layout* L, cudaStream_t s) {
   const Geo g = make_geo(B, H, N, D, L);
   MapSet mq, mk, mv;
   int st;
@@ -393,7 +393,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   // the kernels see SA_BLOCK as SA_FIXED: the same natural view, no summary view
   a.pattern = (L->pattern == SA_BLOCK) ? SA_FIXED : L->pattern;
   a.t_open = (L->pattern == SA_COLUMN) ? 0 : 1;
-  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   // Column view first (SA_STRIDED, SA_COLUMN); the natural view then merges
   // into its result (SA_STRIDED) or runs alone (the other patterns).
   const bool col_pass = dc.fwd_col.n_rows > 0;
@@ -424,6 +424,9 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The default softmax scale 1/sqrt(D).
+float default_scale(int D) { return static_cast<float>(1.0 / std::sqrt(static_cast<double>(D > 0 ? D : 1))); }
 
 int sm_count() {
   int dev = 0, n = 148;
@@ -465,7 +468,7 @@ int grid_for(long long work_items, int per_block) {
 
 template <int D>
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-             void* dq, void* dk, void* dv, int B, int H, int N, const sa_layout* L, void* ws, cudaStream_t s) {
+             void* dq, void* dk, void* dv, int B, int H, int N, float scale, const sa_layout* L, void* ws, cudaStream_t s) {
   const Geo g = make_geo(B, H, N, D, L);
   MapSet mq, mdo, mk, mv;
   int st;
@@ -515,8 +518,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.R = g.R;
   // the kernels see SA_BLOCK as SA_FIXED: the same natural view, no summary view
   a.pattern = (L->pattern == SA_BLOCK) ? SA_FIXED : L->pattern;
-  a.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
-  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  a.scale = scale;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   const bool sec = dc.bwd_sec.n_rows > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN
   // SA_COLUMN has no natural view: its column-view pass writes the final dK/dV.
   const bool sec_final = L->pattern == SA_COLUMN;
@@ -659,16 +662,22 @@ void sparse_attn_layout_free(sa_layout* L) {
 
 int sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
                     const sa_layout* L, void* stream) {
+  return sparse_attn_fwd_ex(q, k, v, o, lse, B, H, N, D, default_scale(D), L, stream);
+}
+
+int sparse_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
+                       float scale, const sa_layout* L, void* stream) {
   if (!q || !k || !v || !o || !lse) return SA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return SA_ERR_INVALID_ARG;
   int st = check_call(B, H, N, D, L);
   if (st) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
-    case 32: return fwd_impl<32>(q, k, v, o, lse, B, H, N, L, s);
-    case 64: return fwd_impl<64>(q, k, v, o, lse, B, H, N, L, s);
-    default: return fwd_impl<128>(q, k, v, o, lse, B, H, N, L, s);
+    case 32: return fwd_impl<32>(q, k, v, o, lse, B, H, N, scale, L, s);
+    case 64: return fwd_impl<64>(q, k, v, o, lse, B, H, N, scale, L, s);
+    default: return fwd_impl<128>(q, k, v, o, lse, B, H, N, scale, L, s);
   }
 }
 
@@ -680,7 +689,15 @@ size_t sparse_attn_bwd_workspace_size(int B, int H, int N, int D, const sa_layou
 int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                     void* dq, void* dk, void* dv, int B, int H, int N, int D, const sa_layout* L, void* workspace,
                     size_t ws_bytes, void* stream) {
+  return sparse_attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, D, default_scale(D), L, workspace, ws_bytes,
+                            stream);
+}
+
+int sparse_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                       void* dq, void* dk, void* dv, int B, int H, int N, int D, float scale, const sa_layout* L,
+                       void* workspace, size_t ws_bytes, void* stream) {
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return SA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
   for (const void* p : ptrs)
     if (!aligned16(p)) return SA_ERR_INVALID_ARG;
@@ -691,9 +708,9 @@ int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, 
     return SA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (D) {
-    case 32: return bwd_impl<32>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, L, workspace, s);
-    case 64: return bwd_impl<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, L, workspace, s);
-    default: return bwd_impl<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, L, workspace, s);
+    case 32: return bwd_impl<32>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, scale, L, workspace, s);
+    case 64: return bwd_impl<64>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, scale, L, workspace, s);
+    default: return bwd_impl<128>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, scale, L, workspace, s);
   }
 }
 

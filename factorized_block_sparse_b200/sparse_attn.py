@@ -23,8 +23,9 @@ SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_LUT, SA_ERR_T
 # Every entry point declared in include/sparse_attn.h.
 EXPORTS = (
     "sparse_attn_layout", "sparse_attn_layout_export", "sparse_attn_layout_info",
-    "sparse_attn_layout_upload", "sparse_attn_layout_free", "sparse_attn_fwd",
-    "sparse_attn_bwd_workspace_size", "sparse_attn_bwd", "sparse_attn_bwd_noalloc", "sparse_attn_status",
+    "sparse_attn_layout_upload", "sparse_attn_layout_free", "sparse_attn_fwd", "sparse_attn_fwd_ex",
+    "sparse_attn_bwd_workspace_size", "sparse_attn_bwd", "sparse_attn_bwd_ex", "sparse_attn_bwd_noalloc",
+    "sparse_attn_status",
     "sparse_attn_strerror", "sparse_attn_kernel_kinds", "sparse_attn_timing_enable",
     "sparse_attn_timing_reset", "sparse_attn_timing_read", "sparse_attn_launch_count",
 )
@@ -54,10 +55,14 @@ def _load():
     lib.sparse_attn_layout_free.restype = None
     lib.sparse_attn_fwd.argtypes = [VP, VP, VP, VP, VP, I, I, I, I, VP, VP]
     lib.sparse_attn_fwd.restype = I
+    lib.sparse_attn_fwd_ex.argtypes = [VP, VP, VP, VP, VP, I, I, I, I, ctypes.c_float, VP, VP]
+    lib.sparse_attn_fwd_ex.restype = I
     lib.sparse_attn_bwd_workspace_size.argtypes = [I, I, I, I, VP]
     lib.sparse_attn_bwd_workspace_size.restype = ctypes.c_size_t
     lib.sparse_attn_bwd.argtypes = [VP] * 9 + [I, I, I, I, VP, VP, ctypes.c_size_t, VP]
     lib.sparse_attn_bwd.restype = I
+    lib.sparse_attn_bwd_ex.argtypes = [VP] * 9 + [I, I, I, I, ctypes.c_float, VP, VP, ctypes.c_size_t, VP]
+    lib.sparse_attn_bwd_ex.restype = I
     lib.sparse_attn_bwd_noalloc.argtypes = [VP] * 9 + [I, I, I, I, VP, VP]
     lib.sparse_attn_bwd_noalloc.restype = I
     lib.sparse_attn_status.argtypes = [VP]
@@ -157,24 +162,33 @@ def _shape(q):
     return tuple(int(x) for x in q.shape)
 
 
-def sparse_attn_fwd(q, k, v, o, lse, layout, stream=None):
-    """Writes ``o`` and ``lse`` in place (C ABI call)."""
+def sparse_attn_fwd(q, k, v, o, lse, layout, stream=None, scale=None):
+    """Writes ``o`` and ``lse`` in place (C ABI call); ``scale`` None is 1/sqrt(D)."""
     B, H, N, D = _shape(q)
-    _check(lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, D,
-                               layout.handle, _stream_ptr(stream)), "sparse_attn_fwd")
+    if scale is None:
+        _check(lib.sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, D,
+                                   layout.handle, _stream_ptr(stream)), "sparse_attn_fwd")
+    else:
+        _check(lib.sparse_attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, D, float(scale),
+                                      layout.handle, _stream_ptr(stream)), "sparse_attn_fwd_ex")
 
 
 def sparse_attn_bwd_workspace_size(B, H, N, D, layout):
     return int(lib.sparse_attn_bwd_workspace_size(B, H, N, D, layout.handle))
 
 
-def sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, layout, workspace, stream=None):
-    """Writes ``dq``, ``dk``, ``dv`` in place (C ABI call)."""
+def sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, layout, workspace, stream=None, scale=None):
+    """Writes ``dq``, ``dk``, ``dv`` in place (C ABI call); ``scale`` None is 1/sqrt(D)."""
     B, H, N, D = _shape(q)
-    _check(lib.sparse_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
-                               _ptr(dk), _ptr(dv), B, H, N, D, layout.handle, _ptr(workspace),
-                               workspace.numel() * workspace.element_size(), _stream_ptr(stream)),
-           "sparse_attn_bwd")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if scale is None:
+        _check(lib.sparse_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                                   _ptr(dk), _ptr(dv), B, H, N, D, layout.handle, _ptr(workspace),
+                                   ws_bytes, _stream_ptr(stream)), "sparse_attn_bwd")
+    else:
+        _check(lib.sparse_attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq),
+                                      _ptr(dk), _ptr(dv), B, H, N, D, float(scale), layout.handle,
+                                      _ptr(workspace), ws_bytes, _stream_ptr(stream)), "sparse_attn_bwd_ex")
 
 
 def sparse_attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, layout, stream=None):
@@ -197,14 +211,14 @@ def sparse_attn_status(stream=None):
 
 
 # ------------------------------------------------------------ conveniences
-def forward(q, k, v, layout, stream=None):
+def forward(q, k, v, layout, stream=None, scale=None):
     """Allocates ``o`` (bf16) and ``lse`` (fp32) with torch and runs the forward pass."""
     import torch
 
     B, H, N, D = _shape(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    sparse_attn_fwd(q, k, v, o, lse, layout, stream)
+    sparse_attn_fwd(q, k, v, o, lse, layout, stream, scale)
     return o, lse
 
 
@@ -215,7 +229,7 @@ def workspace(B, H, N, D, layout, device):
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 
-def backward(q, k, v, o, lse, dO, layout, ws=None, stream=None):
+def backward(q, k, v, o, lse, dO, layout, ws=None, stream=None, scale=None):
     """Allocates ``dq``, ``dk``, ``dv`` (and a workspace if none is given)."""
     import torch
 
@@ -223,7 +237,7 @@ def backward(q, k, v, o, lse, dO, layout, ws=None, stream=None):
     if ws is None:
         ws = workspace(B, H, N, D, layout, q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, layout, ws, stream)
+    sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, layout, ws, stream, scale)
     return dq, dk, dv
 
 

@@ -160,6 +160,17 @@ void sparse_attn_layout_free(sa_layout* layout);
 int sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int H, int N, int D, const sa_layout* layout, void* stream);
 
+/*
+ * sparse_attn_fwd_ex - sparse_attn_fwd with the softmax scale given: scores
+ * are scale * q.k (sparse_attn_fwd uses 1/sqrt(D); the pages do not fix the
+ * scale, see "Insights: 희소 어텐션 (Sparse Attention)", the attention_impl
+ * paragraph).  lse = log sum_j exp(scale * q_i.k_j).  scale must be finite
+ * and > 0, else SA_ERR_INVALID_ARG (returned before any launch); the other
+ * arguments and errors are those of sparse_attn_fwd.
+ */
+int sparse_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int N, int D, float scale, const sa_layout* layout, void* stream);
+
 /* Bytes of device workspace sparse_attn_bwd needs for this shape. */
 size_t sparse_attn_bwd_workspace_size(int B, int H, int N, int D, const sa_layout* layout);
 
@@ -177,6 +188,18 @@ int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                     const float* lse, const void* dO, void* dq, void* dk, void* dv, int B, int H,
                     int N, int D, const sa_layout* layout, void* workspace, size_t ws_bytes,
                     void* stream);
+
+/*
+ * sparse_attn_bwd_ex - sparse_attn_bwd with the softmax scale given (the
+ * scale the forward pass that produced o and lse used; dQ and dK carry the
+ * factor scale).  scale must be finite and > 0, else SA_ERR_INVALID_ARG
+ * (returned before any launch); the other arguments and errors are those of
+ * sparse_attn_bwd.
+ */
+int sparse_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                       int H, int N, int D, float scale, const sa_layout* layout, void* workspace,
+                       size_t ws_bytes, void* stream);
 
 /*
  * sparse_attn_bwd_noalloc - the backward pass for callers that cannot

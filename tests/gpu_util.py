@@ -26,15 +26,15 @@ def assert_close(name, got, ref, max_abs=MAX_ABS, rel_l2=REL_L2):
     return ma, rl
 
 
-def run_library(mode, B, H, N, D, l, c, block, seed_offset=0, device="cuda:0"):
+def run_library(mode, B, H, N, D, l, c, block, seed_offset=0, device="cuda:0", scale=None):
     """fwd + bwd through the C ABI; returns host inputs and float64 outputs."""
     from factorized_block_sparse_b200 import sparse_attn as sa
 
     x = synth.inputs(B, H, N, D, seed_offset)
     lay = sa.Layout(mode, N, l, c, block)
     q, k, v, dO = (x[n].to(device) for n in ("q", "k", "v", "dO"))
-    o, lse = sa.forward(q, k, v, lay)
-    dq, dk, dv = sa.backward(q, k, v, o, lse, dO, lay)
+    o, lse = sa.forward(q, k, v, lay, scale=scale)
+    dq, dk, dv = sa.backward(q, k, v, o, lse, dO, lay, scale=scale)
     torch.cuda.synchronize()
     st = sa.sparse_attn_status()
     assert st == 0, f"device status {st}: {sa.strerror(st)}"
@@ -43,8 +43,8 @@ def run_library(mode, B, H, N, D, l, c, block, seed_offset=0, device="cuda:0"):
     return x, out, lay
 
 
-def oracle_full(x, mode, l, c):
+def oracle_full(x, mode, l, c, scale=None):
     q, k, v, dO = (synth.to_f64(x[n]) for n in ("q", "k", "v", "dO"))
-    O, L = attention.forward(q, k, v, mode, l, c)
-    dq, dk, dv = attention.backward(q, k, v, dO, mode, l, c, lse=L)
+    O, L = attention.forward(q, k, v, mode, l, c, scale=scale)
+    dq, dk, dv = attention.backward(q, k, v, dO, mode, l, c, scale=scale, lse=L)
     return {"o": O, "lse": L, "dq": dq, "dk": dk, "dv": dv}

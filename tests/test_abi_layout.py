@@ -81,6 +81,12 @@ def test_argument_errors(sa):
         == sa.SA_ERR_UNSUPPORTED
     assert sa.lib.sparse_attn_fwd(fake, fake, fake, fake, fake, 0, 1, 256, 32, lay.handle, None) \
         == sa.SA_ERR_INVALID_ARG
+    # an explicit softmax scale must be finite and positive (checked before any launch)
+    for bad in (0.0, -0.5, float("nan"), float("inf")):
+        assert sa.lib.sparse_attn_fwd_ex(fake, fake, fake, fake, fake, 1, 1, 256, 32, bad, lay.handle, None) \
+            == sa.SA_ERR_INVALID_ARG
+        assert sa.lib.sparse_attn_bwd_ex(*([fake] * 9), 1, 1, 256, 32, bad, lay.handle, fake, 1 << 20, None) \
+            == sa.SA_ERR_INVALID_ARG
     assert sa.strerror(sa.SA_ERR_TIMEOUT) == "device-side wait timed out"
     assert sa.lib.sparse_attn_kernel_kinds() == 36  # 6 kernels x 6 patterns
 

@@ -55,6 +55,27 @@ def test_parity_elementwise(cuda_device, mode, B, H, N, D, l, c, block):
         assert_close(f"{mode} N={N} D={D} {name}", got[name], ref[name])
 
 
+@pytest.mark.parametrize("mode,B,H,N,D,l,c,block,scale", [
+    ("strided", 1, 2, 1024, 64, 32, 0, 64, 0.05),   # flat softmax
+    ("fixed", 1, 1, 1024, 32, 128, 32, 64, 0.3),    # sharper than 1/sqrt(32)
+    ("column", 1, 1, 1024, 64, 32, 0, 64, 0.2),
+])
+def test_parity_explicit_scale(cuda_device, mode, B, H, N, D, l, c, block, scale):
+    x, got, _ = run_library(mode, B, H, N, D, l, c, block, scale=scale)
+    ref = oracle_full(x, mode, l, c, scale=scale)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert np.isfinite(got[name]).all(), name
+        assert_close(f"{mode} scale={scale} {name}", got[name], ref[name])
+
+
+def test_default_scale_is_inverse_sqrt_d(cuda_device):
+    # the plain entry points are the _ex ones with scale 1/sqrt(D), bit for bit
+    a = run_library("fixed", 1, 1, 1024, 32, 128, 32, 64)[1]
+    b = run_library("fixed", 1, 1, 1024, 32, 128, 32, 64, scale=1.0 / np.sqrt(32))[1]
+    for name in ("o", "lse", "dk", "dv"):
+        assert np.array_equal(a[name], b[name]), name
+
+
 def test_dk_dv_deterministic(cuda_device):
     a = run_library("strided", 1, 2, 2048, 64, 64, 0, 64)[1]
     b = run_library("strided", 1, 2, 2048, 64, 64, 0, 64)[1]
