@@ -235,6 +235,13 @@ def max_over_ranks(value, world, device):
     return float(t.item())
 
 
+def whole_job(world, step_flops, step_tokens, local_ms_total, steps, device=None):
+    """Whole-job throughput of a weak-scaled run: every rank does the same work
+    on its own data; the time is the slowest rank's (max over ranks)."""
+    ms_step = max_over_ranks(local_ms_total, world, device) / steps
+    return world * step_flops / (ms_step * 1e-3) / 1e12, world * step_tokens / (ms_step * 1e-3), ms_step
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -441,11 +448,9 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status after timing: {sa.strerror(st)}")
     local_ms = sum(a.elapsed_time(b) for a, b in evs)
-    total_ms = max_over_ranks(local_ms, world, dev)
-    ms_step = total_ms / args.steps
     step_flops = fl_fwd + fl_bwd
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
-    tokens = world * sum(s["w"]["B"] * s["w"]["N"] for s in state)
+    value, tokens_per_s, ms_step = whole_job(world, step_flops, sum(s["w"]["B"] * s["w"]["N"] for s in state),
+                                             local_ms, args.steps, dev)
 
     # dominant kernel of the timed region
     dom, dom_ms = None, -1.0
@@ -477,7 +482,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded iid N(0,1), rounded to bf16)",
         "config": config_dict(names, args),
-        "tokens_per_s": round(tokens / (ms_step * 1e-3), 1),
+        "tokens_per_s": round(tokens_per_s, 1),
         "pct_of_bf16_peak": round(100 * value / (world * pk["bf16"]), 2),
         "pct_of_bf16_sustained": round(100 * value / (world * pk["bf16_sustained"]), 2),
         "peak_source": pk["source"],
