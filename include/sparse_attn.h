@@ -180,8 +180,8 @@ size_t sparse_attn_bwd_workspace_size(int B, int H, int N, int D, const sa_layou
  * workspace: caller-owned device memory of at least
  * sparse_attn_bwd_workspace_size() bytes, 256-byte aligned; its contents on
  * entry do not matter and on exit are unspecified.  dq accumulates in
- * float32 with atomic adds, so its last bits may vary from run to run; dk
- * and dv are deterministic.
+ * float32 by bulk reduce-adds in arrival order, so its last bits may vary
+ * from run to run; dk and dv are deterministic.
  * Errors: as sparse_attn_fwd, plus SA_ERR_WORKSPACE.
  */
 int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -231,7 +231,8 @@ int sparse_attn_bwd_ex(const void* q, const void* k, const void* v, const void* 
  *    streams, or different host threads) race on the array and give wrong
  *    results: order them on one stream or with events.
  * Results equal those of sparse_attn_bwd (dq up to the run-to-run rounding of
- * its atomic accumulation).  Errors: as sparse_attn_bwd.
+ * its fp32 reductions, which add in arrival order).  Errors: as
+ * sparse_attn_bwd.
  */
 #define SA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 int sparse_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
