@@ -124,3 +124,22 @@ def _sampled(name, n_rows=12, n_cols=6, slices=((0, 0),), seed=0):
 def test_parity_full_size_sampled(cuda_device, name):
     w = synth.WORKLOADS[name]
     _sampled(name, slices=((0, 0), (w["B"] - 1, w["H"] - 1)) if w["N"] <= 3072 else ((0, 0),))
+
+
+def test_long_sequence_sampled(cuda_device):
+    """A strided head at N = 2^18 (l = 512, R = 512): sampled rows and key
+    columns against the oracle, and properties at every position."""
+    mode, B, H, N, D, l, c, block = "strided", 1, 1, 1 << 18, 64, 512, 0, 64
+    x, got, _ = run_library(mode, B, H, N, D, l, c, block)
+    q, k, v, dO = (synth.to_f64(x[n]) for n in ("q", "k", "v", "dO"))
+    rows = np.array([0, 1, 777, 131071, 200000, N - 1])
+    Or, Lr = attention.forward_rows(q, k, v, mode, l, c, rows)
+    assert_close("long o", got["o"][:, :, rows], Or)
+    assert_close("long lse", got["lse"][:, :, rows], Lr)
+    assert_close("long dq", got["dq"][:, :, rows], attention.dq_rows(q, k, v, dO, mode, l, c, rows))
+    cols = np.array([5, 100003, N - 1])
+    dkc, dvc = attention.dkv_cols(q, k, v, dO, mode, l, c, cols)
+    assert_close("long dk", got["dk"][:, :, cols], dkc)
+    assert_close("long dv", got["dv"][:, :, cols], dvc)
+    for k_ in ("o", "lse", "dq", "dk", "dv"):
+        assert np.isfinite(got[k_]).all(), k_
