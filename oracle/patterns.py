@@ -38,6 +38,11 @@ summary cells).  Two of those heads are modes of their own:
 * ``block``   - the fixed pattern's own-block head, ``j // l == i // l``,
   causal.
 Both contain the diagonal, so no row is empty.
+
+A caller's own block mask (the ``SparseAttention(q, k, v, mask)`` form of
+the "Insights: 희소 어텐션" page, where the sparsity pattern is given as a
+mask of blocks) is a ``BlockMask``: element (i, j) is in the mask when its
+block (i // b, j // b) is and j <= i.  It stands wherever a mode string does.
 """
 
 import numpy as np
@@ -45,7 +50,42 @@ import numpy as np
 MODES = ("all", "local", "strided", "fixed", "column", "block")
 
 
+class BlockMask:
+    """Lower-triangular block mask of an N-position sequence in blocks of ``b``.
+
+    ``row_ptr`` / ``col_idx`` list, per query block r, the key blocks s <= r
+    in the mask (ascending); every row holds its diagonal block, so no row
+    is empty.  Element (i, j) is in the mask when block (i // b, j // b) is
+    and j <= i.
+    """
+
+    def __init__(self, N, block, row_ptr, col_idx):
+        if N % block:
+            raise ValueError("N must be a multiple of block")
+        nb = N // block
+        row_ptr = np.asarray(row_ptr, dtype=np.int64)
+        col_idx = np.asarray(col_idx, dtype=np.int64)
+        if len(row_ptr) != nb + 1 or row_ptr[0] != 0 or row_ptr[-1] != len(col_idx):
+            raise ValueError("row_ptr does not describe the column list")
+        self.N, self.block = int(N), int(block)
+        self.blocks = np.zeros((nb, nb), dtype=bool)
+        for r in range(nb):
+            cols = col_idx[row_ptr[r]:row_ptr[r + 1]]
+            if len(cols) == 0 or cols[-1] != r or np.any(np.diff(cols) <= 0) or cols[0] < 0:
+                raise ValueError(f"block row {r}: ascending columns <= {r} ending with the diagonal")
+            self.blocks[r, cols] = True
+
+    def pairs(self, i, j):
+        i = np.asarray(i, dtype=np.int64)
+        j = np.asarray(j, dtype=np.int64)
+        return (j <= i) & self.blocks[i // self.block, j // self.block]
+
+
 def _check(mode, N, l, c):
+    if isinstance(mode, BlockMask):
+        if N != mode.N:
+            raise ValueError("block mask built for another N")
+        return
     if mode not in MODES:
         raise ValueError(f"unknown mode {mode!r}")
     if N < 1:
@@ -58,6 +98,8 @@ def _check(mode, N, l, c):
 
 def pair_mask(mode, l, c, i, j):
     """Membership of the pairs (i, j) (broadcasting integer arrays)."""
+    if isinstance(mode, BlockMask):
+        return mode.pairs(i, j)
     i = np.asarray(i, dtype=np.int64)
     j = np.asarray(j, dtype=np.int64)
     causal = j <= i

@@ -29,7 +29,7 @@ into disjoint views, each dense in its own relabelled order:
 The two single-head modes use one view each: ``column`` the column-major
 view ``T`` with the diagonal included (``i - j >= 0``, ``(i - j) mod l ==
 0``: there is no natural view to hold it), ``block`` the natural view of
-``fixed``.
+``fixed``.  A caller's ``BlockMask`` is one natural view.
 
 Block table of a view: cut its (queries x keys) matrix, in view order,
 into ``block x block`` tiles (a ragged last tile is padded with
@@ -41,7 +41,7 @@ the transposed CSR (key-block major) serves the backward pass.
 
 import numpy as np
 
-from .patterns import MODES
+from .patterns import MODES, BlockMask
 
 VIEWS = ("N", "T", "S")
 FULL, PARTIAL = 0, 1
@@ -49,6 +49,8 @@ FULL, PARTIAL = 0, 1
 
 def views_of(mode):
     """Which views a mode is split into."""
+    if isinstance(mode, BlockMask):
+        return ("N",)
     if mode not in MODES:
         raise ValueError(mode)
     if mode == "strided":
@@ -76,6 +78,8 @@ def _natural_view_predicate(view, mode, l, c, i, j):
     """Membership of natural pair (i, j) in a view (broadcasting arrays)."""
     causal = j <= i
     if view == "N":
+        if isinstance(mode, BlockMask):
+            return mode.pairs(i, j)
         if mode == "all":
             return causal
         if mode in ("local", "strided"):
