@@ -29,8 +29,8 @@ enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_F
 const char* const kKernelNames[K_KERNELS] = {"sa_fwd_column_view", "sa_fwd_natural_view",
                                              "sa_bwd_preprocess",  "sa_bwd_secondary_view",
                                              "sa_bwd_natural_view", "sa_bwd_finalize_dq"};
-constexpr int K_PATTERNS = 6;
-const char* const kPatternNames[K_PATTERNS] = {"all", "local", "strided", "fixed", "column", "block"};
+constexpr int K_PATTERNS = 7;
+const char* const kPatternNames[K_PATTERNS] = {"all", "local", "strided", "fixed", "column", "block", "blocks"};
 // Instrumentation kinds: one per (kernel, pattern), kind = kernel * 4 + pattern.
 constexpr int K_NUM = K_KERNELS * K_PATTERNS;
 char g_kind_names[K_NUM][48];
@@ -363,6 +363,16 @@ int set_smem(K kernel, int bytes) {
              : SA_ERR_CUDA;
 }
 
+// The pattern whose interval rules the kernels apply: SA_BLOCK has the
+// natural view of SA_FIXED (no summary view); SA_BLOCKS is causal inside
+// the listed blocks, the rule of SA_ALL (its tables hold only listed blocks,
+// and every kernel tile lies inside one block).
+int kernel_pattern(int pattern) {
+  if (pattern == SA_BLOCK) return SA_FIXED;
+  if (pattern == SA_BLOCKS) return SA_ALL;
+  return pattern;
+}
+
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
              float scale, const sa_layout* L, cudaStream_t s) {
@@ -390,8 +400,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.l = g.l;
   a.c = g.c;
   a.R = g.R;
-  // the kernels see SA_BLOCK as SA_FIXED: the same natural view, no summary view
-  a.pattern = (L->pattern == SA_BLOCK) ? SA_FIXED : L->pattern;
+  a.pattern = kernel_pattern(L->pattern);
   a.t_open = (L->pattern == SA_COLUMN) ? 0 : 1;
   a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   // Column view first (SA_STRIDED, SA_COLUMN); the natural view then merges
@@ -516,8 +525,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.l = g.l;
   a.c = g.c;
   a.R = g.R;
-  // the kernels see SA_BLOCK as SA_FIXED: the same natural view, no summary view
-  a.pattern = (L->pattern == SA_BLOCK) ? SA_FIXED : L->pattern;
+  a.pattern = kernel_pattern(L->pattern);
   a.scale = scale;
   a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   const bool sec = dc.bwd_sec.n_rows > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN
@@ -581,6 +589,28 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
 using namespace sa;
 
 extern "C" {
+
+int sparse_attn_layout_blocks(int N, int block, const int32_t* row_ptr, const int32_t* col_idx, sa_layout** out) {
+  if (!out) return SA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!row_ptr || !col_idx || N < 1 || block < 1) return SA_ERR_INVALID_ARG;
+  if (block % kFwdTQ != 0 || block % kBwdTK != 0 || N % block != 0) return SA_ERR_UNSUPPORTED;
+  sa_layout* L = new (std::nothrow) sa_layout();
+  if (!L) return SA_ERR_INVALID_ARG;
+  L->pattern = SA_BLOCKS;
+  L->N = N;
+  L->l = 1;
+  L->c = 0;
+  L->block = block;
+  L->R = 1;
+  const int st = build_layout_blocks(L, row_ptr, col_idx);
+  if (st != SA_OK) {
+    delete L;
+    return st;
+  }
+  *out = L;
+  return SA_OK;
+}
 
 int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** out) {
   if (!out) return SA_ERR_INVALID_ARG;

@@ -77,6 +77,9 @@ struct sa_layout {
 namespace sa {
 // Builds every table of a layout (host only).  Returns an sa_status.
 int build_layout(sa_layout* L);
+// Builds the tables of a caller's block mask (SA_BLOCKS; L->N, L->block set,
+// N % block == 0); row_ptr has N / block + 1 entries.  Returns an sa_status.
+int build_layout_blocks(sa_layout* L, const int32_t* row_ptr, const int32_t* col_idx);
 // Number of key positions of a view (summary view: R * c).
 int view_keys(const sa_layout* L, int view);
 }  // namespace sa

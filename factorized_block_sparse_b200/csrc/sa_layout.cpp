@@ -191,16 +191,10 @@ int view_keys(const sa_layout* L, int view) {
   return L->N;
 }
 
-int build_layout(sa_layout* L) {
-  const int p = L->pattern;
-  L->has[SA_VIEW_NATURAL] = (p != SA_COLUMN);
-  L->has[SA_VIEW_COLUMN] = (p == SA_STRIDED || p == SA_COLUMN);
-  L->has[SA_VIEW_SUMMARY] = (p == SA_FIXED);
-  for (int v = 0; v < 3; ++v) {
-    if (!L->has[v]) continue;
-    L->view[v] = build_public(L, v);
-    L->viewT[v] = transpose(L->view[v]);
-  }
+namespace {
+
+// Kernel tile tables from the public tables in L->view / L->viewT.
+void build_kernel_tables(sa_layout* L) {
   const long long N = L->N;
   const int b = L->block;
 
@@ -252,6 +246,48 @@ int build_layout(sa_layout* L) {
   } else {
     finish_table(L->bwd_sec, {});
   }
+}
+
+}  // namespace
+
+int build_layout(sa_layout* L) {
+  const int p = L->pattern;
+  L->has[SA_VIEW_NATURAL] = (p != SA_COLUMN);
+  L->has[SA_VIEW_COLUMN] = (p == SA_STRIDED || p == SA_COLUMN);
+  L->has[SA_VIEW_SUMMARY] = (p == SA_FIXED);
+  for (int v = 0; v < 3; ++v) {
+    if (!L->has[v]) continue;
+    L->view[v] = build_public(L, v);
+    L->viewT[v] = transpose(L->view[v]);
+  }
+  build_kernel_tables(L);
+  return SA_OK;
+}
+
+int build_layout_blocks(sa_layout* L, const int32_t* row_ptr, const int32_t* col_idx) {
+  // The caller's table is the natural view: per query block, ascending key
+  // blocks at or below the diagonal, the diagonal block last.  Diagonal
+  // blocks hold the causal triangle (PARTIAL); the others are FULL.
+  const int nb = L->N / L->block;
+  if (row_ptr[0] != 0) return SA_ERR_INVALID_ARG;
+  Csr t;
+  t.n_rows = t.n_cols = nb;
+  t.row_ptr.assign(1, 0);
+  for (int r = 0; r < nb; ++r) {
+    const int32_t e0 = row_ptr[r], e1 = row_ptr[r + 1];
+    if (e1 <= e0 || col_idx[e1 - 1] != r) return SA_ERR_INVALID_ARG;  // empty, or no diagonal block
+    for (int32_t e = e0; e < e1; ++e) {
+      const int32_t cb = col_idx[e];
+      if (cb < 0 || (e > e0 && cb <= col_idx[e - 1])) return SA_ERR_INVALID_ARG;
+      t.col_idx.push_back(cb);
+      t.kind.push_back(cb == r ? SA_BLOCK_PARTIAL : SA_BLOCK_FULL);
+    }
+    t.row_ptr.push_back(static_cast<int32_t>(t.col_idx.size()));
+  }
+  L->has[SA_VIEW_NATURAL] = true;
+  L->view[SA_VIEW_NATURAL] = t;
+  L->viewT[SA_VIEW_NATURAL] = transpose(t);
+  build_kernel_tables(L);
   return SA_OK;
 }
 

@@ -15,14 +15,15 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
 
-PATTERNS = {"all": 0, "local": 1, "strided": 2, "fixed": 3, "column": 4, "block": 5}
+PATTERNS = {"all": 0, "local": 1, "strided": 2, "fixed": 3, "column": 4, "block": 5,
+            "blocks": 6}  # "blocks": a caller's block mask (Layout.from_blocks)
 VIEWS = {"N": 0, "T": 1, "S": 2}
 VIEW_TRANSPOSED = 4
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_LUT, SA_ERR_TIMEOUT, SA_ERR_WORKSPACE = range(7)
 
 # Every entry point declared in include/sparse_attn.h.
 EXPORTS = (
-    "sparse_attn_layout", "sparse_attn_layout_export", "sparse_attn_layout_info",
+    "sparse_attn_layout", "sparse_attn_layout_blocks", "sparse_attn_layout_export", "sparse_attn_layout_info",
     "sparse_attn_layout_upload", "sparse_attn_layout_free", "sparse_attn_fwd", "sparse_attn_fwd_ex",
     "sparse_attn_bwd_workspace_size", "sparse_attn_bwd", "sparse_attn_bwd_ex", "sparse_attn_bwd_noalloc",
     "sparse_attn_status",
@@ -45,6 +46,8 @@ def _load():
     P, I, F, VP = ctypes.POINTER, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
     lib.sparse_attn_layout.argtypes = [I, I, I, I, I, P(VP)]
     lib.sparse_attn_layout.restype = I
+    lib.sparse_attn_layout_blocks.argtypes = [I, I, VP, VP, P(VP)]
+    lib.sparse_attn_layout_blocks.restype = I
     lib.sparse_attn_layout_export.argtypes = [VP, I, VP, VP, VP, P(I), P(I)]
     lib.sparse_attn_layout_export.restype = I
     lib.sparse_attn_layout_info.argtypes = [VP, P(I), P(I), P(I), P(I), P(I)]
@@ -105,6 +108,24 @@ class Layout:
         _check(lib.sparse_attn_layout(PATTERNS[pattern], self.N, self.l, self.c, self.block,
                                       ctypes.byref(h)), "sparse_attn_layout")
         self._h = h
+
+    @classmethod
+    def from_blocks(cls, N, block, row_ptr, col_idx):
+        """Layout of a caller's block mask (``sparse_attn_layout_blocks``): per
+        query block, the ascending key blocks at or below the diagonal, the
+        diagonal block last; block a multiple of 128."""
+        self = cls.__new__(cls)
+        self.pattern = "blocks"
+        self.N, self.l, self.c, self.block = int(N), 1, 0, int(block)
+        rp = np.ascontiguousarray(row_ptr, dtype=np.int32)
+        ci = np.ascontiguousarray(col_idx, dtype=np.int32)
+        if ci.size == 0:
+            ci = np.zeros(1, dtype=np.int32)
+        h = ctypes.c_void_p()
+        _check(lib.sparse_attn_layout_blocks(self.N, self.block, rp.ctypes.data, ci.ctypes.data, ctypes.byref(h)),
+               "sparse_attn_layout_blocks")
+        self._h = h
+        return self
 
     @property
     def handle(self):

@@ -27,6 +27,10 @@
  *               its row head is SA_LOCAL)
  *   SA_BLOCK    j <= i and j / l == i / l
  *               (the own-block head of SA_FIXED run as a head of its own)
+ *   SA_BLOCKS   j <= i and block (i / b, j / b) is in a caller's block mask
+ *               (built with sparse_attn_layout_blocks: the sparsity pattern
+ *               given as a mask over blocks, the SparseAttention(q, k, v,
+ *               mask) form of "Insights: 희소 어텐션 (Sparse Attention)")
  * SA_COLUMN and SA_BLOCK are the two-head form of the factorized patterns:
  * the two parts of a pattern in separate heads, each with its own softmax
  * ("OpenAI Sparse Transformer", "Factorized Attention Patterns"; pcnews
@@ -62,7 +66,15 @@ extern "C" {
 
 typedef struct sa_layout sa_layout; /* opaque, owned by the library */
 
-enum sa_pattern { SA_ALL = 0, SA_LOCAL = 1, SA_STRIDED = 2, SA_FIXED = 3, SA_COLUMN = 4, SA_BLOCK = 5 };
+enum sa_pattern {
+  SA_ALL = 0,
+  SA_LOCAL = 1,
+  SA_STRIDED = 2,
+  SA_FIXED = 3,
+  SA_COLUMN = 4,
+  SA_BLOCK = 5,
+  SA_BLOCKS = 6
+};
 
 /* Views of a pattern.  Each view is dense in its own relabelled order:
  *   SA_VIEW_NATURAL : natural order, queries and keys (every pattern but
@@ -122,6 +134,23 @@ enum sa_block_kind { SA_BLOCK_FULL = 0, SA_BLOCK_PARTIAL = 1 };
  * SA_ERR_UNSUPPORTED (N % block or N % l not zero).
  */
 int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** out);
+
+/*
+ * sparse_attn_layout_blocks - a layout (pattern SA_BLOCKS) from a caller's
+ * block mask: the sparsity pattern given as a mask over blocks (the
+ * SparseAttention(q, k, v, mask) form of "Insights: 희소 어텐션 (Sparse
+ * Attention)").  row_ptr [N/block + 1] and col_idx (host memory, read
+ * during the call only) list, per query block r, the key blocks s in the
+ * mask, ascending, with 0 <= s <= r and the diagonal block s = r last (so
+ * no row is empty).  Element (i, j) attends when its block is listed and
+ * j <= i.  block must be a multiple of 128 (the kernels' tile: every tile
+ * then lies inside one block) and divide N.
+ * Errors: SA_ERR_INVALID_ARG (null pointer, N < 1, a row that is empty,
+ * unsorted, above the diagonal or without its diagonal block),
+ * SA_ERR_UNSUPPORTED (block not a multiple of 128, N % block not zero).
+ */
+int sparse_attn_layout_blocks(int N, int block, const int32_t* row_ptr, const int32_t* col_idx,
+                              sa_layout** out);
 
 /*
  * sparse_attn_layout_export - host copy of one view's block table.

@@ -26,12 +26,12 @@ def assert_close(name, got, ref, max_abs=MAX_ABS, rel_l2=REL_L2):
     return ma, rl
 
 
-def run_library(mode, B, H, N, D, l, c, block, seed_offset=0, device="cuda:0", scale=None):
+def run_library(mode, B, H, N, D, l, c, block, seed_offset=0, device="cuda:0", scale=None, layout=None):
     """fwd + bwd through the C ABI; returns host inputs and float64 outputs."""
     from factorized_block_sparse_b200 import sparse_attn as sa
 
     x = synth.inputs(B, H, N, D, seed_offset)
-    lay = sa.Layout(mode, N, l, c, block)
+    lay = layout if layout is not None else sa.Layout(mode, N, l, c, block)
     q, k, v, dO = (x[n].to(device) for n in ("q", "k", "v", "dO"))
     o, lse = sa.forward(q, k, v, lay, scale=scale)
     dq, dk, dv = sa.backward(q, k, v, o, lse, dO, lay, scale=scale)

@@ -88,7 +88,7 @@ def test_argument_errors(sa):
         assert sa.lib.sparse_attn_bwd_ex(*([fake] * 9), 1, 1, 256, 32, bad, lay.handle, fake, 1 << 20, None) \
             == sa.SA_ERR_INVALID_ARG
     assert sa.strerror(sa.SA_ERR_TIMEOUT) == "device-side wait timed out"
-    assert sa.lib.sparse_attn_kernel_kinds() == 36  # 6 kernels x 6 patterns
+    assert sa.lib.sparse_attn_kernel_kinds() == 42  # 6 kernels x 7 patterns
 
 
 def _compare(sa, mode, N, l, c, b, rows=None):
@@ -149,3 +149,45 @@ def test_layout_bit_exact_audio_sampled_rows(sa):
 ])
 def test_layout_bit_exact_degenerate_and_ragged(sa, mode, N, l, c, b):
     _compare(sa, mode, N, l, c, b)
+
+
+def _random_blocks(nb, seed, p=0.35):
+    rng = np.random.default_rng(seed)
+    rp, ci = [0], []
+    for r in range(nb):
+        ci += [s for s in range(r) if rng.random() < p] + [r]
+        rp.append(len(ci))
+    return rp, ci
+
+
+@pytest.mark.parametrize("N,b,seed", [(1024, 128, 0), (2048, 256, 1), (1536, 128, 2)])
+def test_layout_blocks_bit_exact(sa, N, b, seed):
+    from oracle import patterns
+
+    rp, ci = _random_blocks(N // b, seed)
+    lay = sa.Layout.from_blocks(N, b, rp, ci)
+    bm = patterns.BlockMask(N, b, rp, ci)
+    got, ref = lay.export("N"), views.block_table("N", bm, N, 1, 0, b)
+    for k in ("row_ptr", "col_idx", "kind"):
+        assert np.array_equal(got[k], ref[k]), k
+    gt, rt = lay.export("N", transposed=True), views.transpose_table(ref)
+    for k in ("row_ptr", "col_idx", "kind"):
+        assert np.array_equal(gt[k], rt[k]), k
+    assert lay.export("T")["n_rows"] == 0 and lay.export("S")["n_rows"] == 0
+
+
+def test_layout_blocks_errors(sa):
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.Layout.from_blocks(256, 128, [0, 1, 2], [0, 0])          # row 1 without its diagonal
+    assert e.value.status == sa.SA_ERR_INVALID_ARG
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.Layout.from_blocks(384, 128, [0, 1, 3, 5], [0, 1, 0, 0, 2])  # unsorted row 1
+    assert e.value.status == sa.SA_ERR_INVALID_ARG
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.Layout.from_blocks(256, 64, [0, 1, 3, 4, 6], [0, 0, 1, 2, 2, 3])  # block not a multiple of 128
+    assert e.value.status == sa.SA_ERR_UNSUPPORTED
+    with pytest.raises(sa.SparseAttnError) as e:
+        sa.Layout.from_blocks(300, 128, [0, 1, 3], [0, 0, 1])        # N % block
+    assert e.value.status == sa.SA_ERR_UNSUPPORTED
+    h = ctypes.c_void_p()
+    assert sa.lib.sparse_attn_layout(6, 256, 1, 0, 128, ctypes.byref(h)) == sa.SA_ERR_INVALID_ARG

@@ -143,3 +143,39 @@ def test_long_sequence_sampled(cuda_device):
     assert_close("long dv", got["dv"][:, :, cols], dvc)
     for k_ in ("o", "lse", "dq", "dk", "dv"):
         assert np.isfinite(got[k_]).all(), k_
+
+
+def _random_blocks(nb, seed, p=0.35):
+    rng = np.random.default_rng(seed)
+    rp, ci = [0], []
+    for r in range(nb):
+        ci += [s for s in range(r) if rng.random() < p] + [r]
+        rp.append(len(ci))
+    return rp, ci
+
+
+@pytest.mark.parametrize("B,H,N,D,b,seed", [(1, 2, 2048, 64, 128, 0), (2, 1, 1024, 32, 256, 1),
+                                            (1, 1, 1024, 128, 128, 2)])
+def test_parity_block_mask(cuda_device, B, H, N, D, b, seed):
+    """A caller's block mask (sparse_attn_layout_blocks) against the oracle's BlockMask."""
+    from factorized_block_sparse_b200 import sparse_attn as sa
+    from oracle import patterns
+
+    rp, ci = _random_blocks(N // b, seed)
+    lay = sa.Layout.from_blocks(N, b, rp, ci)
+    x, got, _ = run_library("blocks", B, H, N, D, 1, 0, b, layout=lay)
+    ref = oracle_full(x, patterns.BlockMask(N, b, rp, ci), 1, 0)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert np.isfinite(got[name]).all(), name
+        assert_close(f"blocks N={N} D={D} {name}", got[name], ref[name])
+
+
+def test_block_mask_of_all_lower_blocks_equals_all(cuda_device):
+    from factorized_block_sparse_b200 import sparse_attn as sa
+
+    N, b = 1024, 128
+    rp, ci = _random_blocks(N // b, 0, p=1.0)
+    a = run_library("blocks", 1, 2, N, 64, 1, 0, b, layout=sa.Layout.from_blocks(N, b, rp, ci))[1]
+    r = run_library("all", 1, 2, N, 64, 1, 0, b)[1]
+    for name in ("o", "lse", "dk", "dv"):
+        assert np.array_equal(a[name], r[name]), name
