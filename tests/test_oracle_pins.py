@@ -18,6 +18,16 @@ from factorized_block_sparse_b200 import synth
 MODES = ("all", "local", "strided", "fixed")
 
 
+def _block_mask(N, b, seed, p=0.4):
+    """A caller block mask (lower blocks kept at random, diagonal always)."""
+    rng = np.random.default_rng(seed)
+    rp, ci = [0], []
+    for r in range(N // b):
+        ci += [s for s in range(r) if rng.random() < p] + [r]
+        rp.append(len(ci))
+    return patterns.BlockMask(N, b, rp, ci)
+
+
 def _rand(shape, seed):
     return np.random.default_rng(seed).standard_normal(shape)
 
@@ -49,7 +59,8 @@ def test_all_mode_equals_library_causal_attention():
 
 
 @pytest.mark.parametrize("mode,l,c", [("local", 5, 0), ("strided", 6, 0), ("strided", 7, 0),
-                                      ("fixed", 8, 2), ("fixed", 5, 1)])
+                                      ("fixed", 8, 2), ("fixed", 5, 1), ("column", 6, 0), ("block", 7, 0),
+                                      (_block_mask(50, 5, 1), 1, 0)])
 def test_sparse_modes_equal_library_masked_attention(mode, l, c):
     B, H, N, D = 1, 2, 50, 8
     q, k, v, dO = (_rand((B, H, N, D), 10 + s) for s in range(4))
@@ -63,7 +74,8 @@ def test_sparse_modes_equal_library_masked_attention(mode, l, c):
 
 @pytest.mark.parametrize("mode,N,l,c", [("all", 16, 1, 0), ("local", 16, 4, 0),
                                         ("strided", 16, 4, 0), ("strided", 32, 4, 0),
-                                        ("fixed", 16, 4, 1), ("fixed", 32, 4, 2)])
+                                        ("fixed", 16, 4, 1), ("fixed", 32, 4, 2), ("column", 16, 4, 0),
+                                        ("block", 16, 4, 0), (_block_mask(16, 4, 2), 16, 1, 0)])
 def test_finite_difference_gradients(mode, N, l, c):
     D = 8
     q, k, v, dO = (_rand((1, 1, N, D), 100 + s) for s in range(4))
@@ -87,7 +99,8 @@ def test_finite_difference_gradients(mode, N, l, c):
         assert rel <= 1e-6, (name, rel)
 
 
-@pytest.mark.parametrize("mode,l,c", [("all", 1, 0), ("strided", 8, 0), ("fixed", 8, 3)])
+@pytest.mark.parametrize("mode,l,c", [("all", 1, 0), ("strided", 8, 0), ("fixed", 8, 3), ("column", 8, 0),
+                                      ("block", 8, 0), (_block_mask(64, 8, 3), 1, 0)])
 def test_invariants(mode, l, c):
     B, H, N, D = 1, 2, 64, 8
     q, k, v, dO = (_rand((B, H, N, D), 200 + s) for s in range(4))
@@ -99,7 +112,8 @@ def test_invariants(mode, l, c):
     np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
 
 
-@pytest.mark.parametrize("mode,l,c", [("strided", 16, 0), ("fixed", 16, 4), ("all", 1, 0)])
+@pytest.mark.parametrize("mode,l,c", [("strided", 16, 0), ("fixed", 16, 4), ("all", 1, 0), ("column", 16, 0),
+                                      ("block", 16, 0), (_block_mask(96, 16, 4), 1, 0)])
 def test_sampled_rows_and_columns_match_full(mode, l, c):
     B, H, N, D = 1, 2, 96, 8
     q, k, v, dO = (_rand((B, H, N, D), 300 + s) for s in range(4))
