@@ -46,7 +46,8 @@
  *       major, D fastest), device pointers, 16-byte aligned, owned by the
  *       caller.  bfloat16 values are passed as raw 16-bit patterns.
  *   lse : float32 [B, H, N], natural logarithm, device pointer.
- *   D   : 32, 64 or 128.  Scale is fixed at 1/sqrt(D).
+ *   D   : 32, 64 or 128.  The softmax scale is 1/sqrt(D) in the plain entry
+ *         points; sparse_attn_fwd_ex / sparse_attn_bwd_ex take it explicitly.
  *   stream : a cudaStream_t passed as void*; NULL means the legacy default
  *       stream.  Every compute call only enqueues work on that stream and
  *       returns; none synchronises except sparse_attn_status().
@@ -241,9 +242,13 @@ int sparse_attn_bwd_ex(const void* q, const void* k, const void* v, const void* 
  * sparse_attn_bwd needs.  This entry point takes the same arguments minus the
  * workspace and uses instead a scratch array compiled into the library: a
  * file-scope __device__ array of SA_NOALLOC_SCRATCH_BYTES bytes, which every
- * GPU that loads the library holds until the process exits.
+ * GPU that loads the library holds until the process exits.  That memory is
+ * taken when the library's device code is loaded on a device (with lazy
+ * module loading, at the first launch of any of its kernels there), so a
+ * caller's device-memory budget must count it from then on.
  *
- * Limits and behaviour:
+ * Limits and behaviour (the checks run in this order, before any device
+ * work: pointer and shape arguments, then the size, then the layout):
  *  - shapes whose sparse_attn_bwd_workspace_size() exceeds
  *    SA_NOALLOC_SCRATCH_BYTES are rejected with SA_ERR_WORKSPACE;
  *  - it calls no cudaMalloc, cudaFree or other allocating routine, so the

@@ -191,3 +191,11 @@ def test_layout_blocks_errors(sa):
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
     h = ctypes.c_void_p()
     assert sa.lib.sparse_attn_layout(6, 256, 1, 0, 128, ctypes.byref(h)) == sa.SA_ERR_INVALID_ARG
+
+
+def test_noalloc_scratch_size_matches_header(sa):
+    # the binding's copy of SA_NOALLOC_SCRATCH_BYTES must follow the header's macro
+    text = open(os.path.join(ROOT, "include", "sparse_attn.h")).read()
+    m = re.search(r"#define\s+SA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*\*\s*(\d+)u\s*\*\s*(\d+)u\)", text)
+    assert m, "SA_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == sa.NOALLOC_SCRATCH_BYTES

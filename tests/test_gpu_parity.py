@@ -43,6 +43,10 @@ SMALL = [
     ("block", 1, 2, 1024, 64, 128, 0, 64),
     ("block", 2, 1, 960, 32, 100, 0, 64),       # l does not divide N
     ("block", 1, 1, 1024, 128, 256, 0, 64),
+    # strided with l = 192 (R = 16): the natural view's key tiles see about five
+    # 64-query steps each, so its backward takes the LONG shape element by element
+    ("strided", 1, 1, 3072, 64, 192, 0, 64),
+    ("strided", 1, 2, 6144, 64, 192, 0, 64),    # R = 32, image64's row length
 ]
 
 
@@ -80,35 +84,54 @@ def test_default_scale_is_inverse_sqrt_d(cuda_device):
         assert np.array_equal(a[name], b[name]), name
 
 
-def test_dk_dv_deterministic(cuda_device):
-    a = run_library("strided", 1, 2, 2048, 64, 64, 0, 64)[1]
-    b = run_library("strided", 1, 2, 2048, 64, 64, 0, 64)[1]
+@pytest.mark.parametrize("mode,B,H,N,D,l,c,block", [
+    ("strided", 1, 2, 2048, 64, 64, 0, 64),
+    # fixed at N = 4096: its summary view's key tiles see about 30 query steps
+    # each (the LONG backward shape, the text workload's dominant pass)
+    ("fixed", 1, 2, 4096, 64, 128, 32, 64),
+])
+def test_dk_dv_deterministic(cuda_device, mode, B, H, N, D, l, c, block):
+    a = run_library(mode, B, H, N, D, l, c, block)[1]
+    b = run_library(mode, B, H, N, D, l, c, block)[1]
     for name in ("o", "lse", "dk", "dv"):
         assert np.array_equal(a[name], b[name]), name
 
 
-def _sampled(name, n_rows=12, n_cols=6, slices=((0, 0),), seed=0):
+def _tiles(N, n_mid, rng, extra=()):
+    """Whole 128-position tiles: the first, the last, n_mid random ones and the
+    tiles holding the positions in ``extra``; returns sorted positions."""
+    n_t = (N + 127) // 128
+    ts = {0, n_t - 1, *rng.integers(0, n_t, n_mid).tolist(), *(int(p) // 128 for p in extra)}
+    return np.concatenate([np.arange(t * 128, min(N, t * 128 + 128)) for t in sorted(ts)])
+
+
+def _sampled(name, n_mid=2, slices=((0, 0),), seed=0):
+    """Whole 128-row query tiles (O, lse, dQ) and whole 128-key key tiles (dK,
+    dV) of a full-size workload against the oracle, which computes them one
+    row or key column at a time: the first and last tiles, random ones and,
+    for the fixed pattern, key tiles holding summary keys of an early and a
+    late block."""
     w = synth.WORKLOADS[name]
     mode, B, H, N, D, l, c, block = (w[k] for k in ("mode", "B", "H", "N", "D", "l", "c", "block"))
     x, got, _ = run_library(mode, B, H, N, D, l, c, block)
     rng = np.random.default_rng(seed)
-    # first rows, a ragged spread, the last rows; columns likewise
-    rows = np.unique(np.concatenate([[0, 1, N - 1], rng.integers(0, N, n_rows)]))
-    cols = np.unique(np.concatenate([[0, N - 1], rng.integers(0, N, n_cols)]))
-    if mode == "fixed":  # include summary keys of an early and a late block
-        cols = np.unique(np.concatenate([cols, [l - 1, (N // l - 2) * l + l - c]]))
+    rows = _tiles(N, n_mid, rng)
+    extra = [l - 1, (N // l - 2) * l + l - c] if mode == "fixed" else []
+    if N <= 16384:
+        cols = _tiles(N, n_mid, rng, extra)
+    else:  # an early key is seen by ~N/l column rows of N keys each: the last tile + single columns
+        cols = np.unique(np.concatenate([[0, 1], rng.integers(0, N, 8), np.arange(N - 128, N)]))
     for b, h in slices:
-        if True:
-            sl = (slice(b, b + 1), slice(h, h + 1))
-            q, k, v, dO = (synth.to_f64(x[n][sl]) for n in ("q", "k", "v", "dO"))
-            Or, Lr = attention.forward_rows(q, k, v, mode, l, c, rows)
-            assert_close(f"{name} o", got["o"][sl][:, :, rows], Or)
-            assert_close(f"{name} lse", got["lse"][sl][:, :, rows], Lr)
-            dqr = attention.dq_rows(q, k, v, dO, mode, l, c, rows)
-            assert_close(f"{name} dq", got["dq"][sl][:, :, rows], dqr)
-            dkc, dvc = attention.dkv_cols(q, k, v, dO, mode, l, c, cols)
-            assert_close(f"{name} dk", got["dk"][sl][:, :, cols], dkc)
-            assert_close(f"{name} dv", got["dv"][sl][:, :, cols], dvc)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        q, k, v, dO = (synth.to_f64(x[n][sl]) for n in ("q", "k", "v", "dO"))
+        Or, Lr = attention.forward_rows(q, k, v, mode, l, c, rows)
+        assert_close(f"{name} o", got["o"][sl][:, :, rows], Or)
+        assert_close(f"{name} lse", got["lse"][sl][:, :, rows], Lr)
+        dqr = attention.dq_rows(q, k, v, dO, mode, l, c, rows)
+        assert_close(f"{name} dq", got["dq"][sl][:, :, rows], dqr)
+        dkc, dvc = attention.dkv_cols(q, k, v, dO, mode, l, c, cols)
+        assert_close(f"{name} dk", got["dk"][sl][:, :, cols], dkc)
+        assert_close(f"{name} dv", got["dv"][sl][:, :, cols], dvc)
     # properties at every position: finite outputs, lse at least the diagonal score
     for k_ in ("o", "lse", "dq", "dk", "dv"):
         assert np.isfinite(got[k_]).all(), k_
@@ -124,6 +147,21 @@ def _sampled(name, n_rows=12, n_cols=6, slices=((0, 0),), seed=0):
 def test_parity_full_size_sampled(cuda_device, name):
     w = synth.WORKLOADS[name]
     _sampled(name, slices=((0, 0), (w["B"] - 1, w["H"] - 1)) if w["N"] <= 3072 else ((0, 0),))
+
+
+@pytest.mark.parametrize("name,sl", [("text-fixed", (0, 0)), ("text-fixed", (1, 7)),
+                                     ("image64-strided", (0, 0)), ("image64-strided", (0, 15))])
+def test_parity_full_size_whole_head(cuda_device, name, sl):
+    """One whole (batch, head) slice of an N = 12288 workload, every element of
+    O, lse, dQ, dK, dV against the oracle (the launch configuration the
+    benchmark times: all heads of the workload in one call)."""
+    w = synth.WORKLOADS[name]
+    mode, B, H, N, D, l, c, block = (w[k] for k in ("mode", "B", "H", "N", "D", "l", "c", "block"))
+    x, got, _ = run_library(mode, B, H, N, D, l, c, block)
+    ref = oracle_full(x, mode, l, c, sl=sl)
+    b, h = sl
+    for n in ("o", "lse", "dq", "dk", "dv"):
+        assert_close(f"{name} ({b},{h}) {n}", got[n][b:b + 1, h:h + 1], ref[n])
 
 
 def test_long_sequence_sampled(cuda_device):

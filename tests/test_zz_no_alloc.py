@@ -56,6 +56,33 @@ def test_noalloc_backward_matches_workspace_backward(cuda_device, mode, B, H, N,
         assert np.array_equal(got[1], ref[1]) and np.array_equal(got[2], ref[2])
 
 
+def test_noalloc_after_a_larger_different_call(cuda_device):
+    """A larger strided call fills more of the scratch array (column-order lse
+    blocks, secondary partials) than a smaller fixed or dense call reads; the
+    smaller call must not pick up anything the larger one left behind."""
+    from factorized_block_sparse_b200 import sparse_attn as sa
+
+    first = ("strided", 1, 4, 4096, 64, 64, 0, 64)
+    for second in (("fixed", 1, 1, 1024, 64, 128, 32, 64), ("all", 1, 1, 640, 32, 1, 0, 64)):
+        runs = []
+        for mode, B, H, N, D, l, c, block in (first, second):
+            x = synth.inputs(B, H, N, D, seed_offset=7)
+            q, k, v, dO = (x[n].to(cuda_device) for n in ("q", "k", "v", "dO"))
+            lay = sa.Layout(mode, N, l, c, block)
+            assert sa.sparse_attn_bwd_workspace_size(B, H, N, D, lay) <= sa.NOALLOC_SCRATCH_BYTES
+            lay.upload()
+            o, lse = sa.forward(q, k, v, lay)
+            outs = [torch.full_like(q, float("nan")) for _ in range(3)]
+            sa.sparse_attn_bwd_noalloc(q, k, v, o, lse, dO, *outs, lay)
+            assert sa.sparse_attn_status() == 0
+            runs.append((q, k, v, o, lse, dO, lay, outs))
+        q, k, v, o, lse, dO, lay, outs = runs[1]
+        ref = [t.float().cpu().numpy() for t in sa.backward(q, k, v, o, lse, dO, lay)]
+        got = [t.float().cpu().numpy() for t in outs]
+        assert_close(f"{second[0]} after strided dq", got[0], ref[0], MAX_ABS, REL_L2)
+        assert np.array_equal(got[1], ref[1]) and np.array_equal(got[2], ref[2]), second[0]
+
+
 def test_noalloc_refuses_instead_of_allocating(cuda_device):
     from factorized_block_sparse_b200 import sparse_attn as sa
 
