@@ -372,6 +372,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", type=int, default=1, help="1: also time every other named configuration")
     args = ap.parse_args()
     names = STEPS[args.workload]
     if args.warmup < 3:
@@ -424,30 +425,39 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {sa.strerror(st)}")
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    def timed(per_kernel):
+        """K steps, each bracketed by CUDA events on the launching stream, L2
+        flushed before each; with per_kernel the library also brackets every
+        launch with events (which serialises the launches)."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        sa.timing_reset()
+        sa.timing_enable(per_kernel)
+        n0 = sa.launch_count()
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        n = sa.launch_count() - n0
+        sa.timing_enable(False)
+        kt = sa.kernel_times()
+        st = sa.sparse_attn_status()
+        if st != 0:
+            raise RuntimeError(f"device status after timing: {sa.strerror(st)}")
+        return sum(a.elapsed_time(b) for a, b in evs), n, kt
+
+    # the headline: K steps with no per-launch events in between
     sampler = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    sa.timing_reset()
-    sa.timing_enable(True)
-    launches0 = sa.launch_count()
     sampler.start()
     time.sleep(0.3)
-    for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
+    local_ms, launches, _ = timed(False)
     clocks = sampler.stop()
-    launches = sa.launch_count() - launches0
-    sa.timing_enable(False)
-    ktimes = sa.kernel_times()
-    st = sa.sparse_attn_status()
-    if st != 0:
-        raise RuntimeError(f"device status after timing: {sa.strerror(st)}")
-    local_ms = sum(a.elapsed_time(b) for a, b in evs)
+    # the per-kernel breakdown and the roofline: K more steps with every launch bracketed by events
+    kernel_pass_ms, _, ktimes = timed(True)
     step_flops = fl_fwd + fl_bwd
     value, tokens_per_s, ms_step = whole_job(world, step_flops, sum(s["w"]["B"] * s["w"]["N"] for s in state),
                                              local_ms, args.steps, dev)
@@ -472,6 +482,11 @@ def main():
                        "unit": "TFLOP/s" if units[n][0] == "tensor" else "GB/s"} if n in units else {})}
                for n, (ms, c) in ktimes.items() if c}
 
+    # every other named configuration, one at a time (extra keys; the headline stays the step above)
+    configs = None
+    if args.configs and world == 1:
+        configs = measure_configs(sa, [n for n in CONFIGS if n not in names], pk, dev, stream, flush)
+
     # end to end through the C ABI with pinned host buffers
     e2e = None
     if args.e2e_steps > 0:
@@ -491,7 +506,11 @@ def main():
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": "burst (of measured)" if pk["source"] == "measured" else "fallback"},
         "kernels": kernels,
+        "kernel_pass": {"ms_per_step": round(max_over_ranks(kernel_pass_ms, world, dev) / args.steps, 4),
+                        "note": "per-kernel events are taken in a second pass of K steps with every launch "
+                                "bracketed by events; the headline steps run without them"},
         "workloads": workload_lines(state, ktimes, pk),
+        "configs": configs,
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
@@ -505,6 +524,67 @@ def main():
 
         dist.destroy_process_group()
     return 0
+
+
+# The configurations the metric names besides the step's own (the tiny,
+# image32, dense image64 and audio shapes) and the two longer sequences.
+CONFIGS = ["tiny-strided", "image32-strided", "image64-all", "audio-strided", "long-strided-262144",
+           "long-strided-1048576"]
+
+
+def measure_configs(sa, names, pk, dev, stream, flush, steps=10, warmup=3):
+    """fwd + bwd of each named workload alone: ms per step (CUDA events around
+    each step, L2 flushed before it), nonzero-block TFLOP/s, tokens/s and the
+    fraction of the workload's own roofline max(flops / bf16 peak, algorithmic
+    bytes / HBM peak).  Inputs: seeded N(0, 1) drawn on the device."""
+    import torch
+
+    out = {}
+    for n in names:
+        w = synth.WORKLOADS[n]
+        counts, lay = block_counts(w, sa)
+        f0, f1 = flops(w, counts)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1234)
+        shape = (w["B"], w["H"], w["N"], w["D"])
+        q, k, v, dO = (torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+                       for _ in range(4))
+        o = torch.empty_like(q)
+        lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = sa.workspace(w["B"], w["H"], w["N"], w["D"], lay, dev)
+        lay.upload()
+        sptr = stream.cuda_stream
+
+        def one():
+            sa.sparse_attn_fwd(q, k, v, o, lse, lay, sptr)
+            sa.sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, lay, ws, sptr)
+
+        for _ in range(warmup):
+            one()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            one()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        st = sa.sparse_attn_status()
+        if st != 0:
+            raise RuntimeError(f"device status after {n}: {sa.strerror(st)}")
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        t_tc = (f0 + f1) / (pk["bf16"] * 1e12) * 1e3
+        t_hbm = algorithmic_bytes(w) / (pk["hbm"] * 1e9) * 1e3
+        out[n] = {"workload": f"{w['mode']}, B={w['B']}, H={w['H']}, N={w['N']}, D={w['D']}, l={w['l']}"
+                              + (f", c={w['c']}" if w["mode"] == "fixed" else "") + f", block={w['block']}",
+                  "ms_per_step": round(ms, 4), "nonzero_block_tflops": round((f0 + f1) / (ms * 1e-3) / 1e12, 2),
+                  "tokens_per_s": round(w["B"] * w["N"] / (ms * 1e-3), 1),
+                  "roofline": {"bound": "tensor" if t_tc >= t_hbm else "hbm", "frac": round(max(t_tc, t_hbm) / ms, 4)}}
+        del q, k, v, dO, o, lse, dq, dk, dv, ws
+        lay.close()
+        torch.cuda.empty_cache()
+    return out
 
 
 def measure_e2e(sa, state, stream, steps, step_flops, world, dev):

@@ -14,9 +14,14 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsparse_attn.so")
+# The failure-detection tests' build: short device-side wait limits, a flag
+# that withholds one load, range checks of the device tables, and two
+# exported test hooks.  Never used by the product path.
+TEST_LIB = os.path.join(HERE, "libsparse_attn_test.so")
 SOURCES = [os.path.join(HERE, "csrc", "sa_api.cu"), os.path.join(HERE, "csrc", "sa_layout.cpp")]
 HEADERS = [os.path.join(ROOT, "include", "sparse_attn.h")] + [
-    os.path.join(HERE, "csrc", f) for f in ("sa_internal.h", "sa_device.cuh", "sa_fwd.cuh", "sa_bwd.cuh")]
+    os.path.join(HERE, "csrc", f) for f in ("sa_internal.h", "sa_device.cuh", "sa_fwd.cuh", "sa_bwd.cuh",
+                                            "sa_bwd_wide.cuh", "sa_tail.cuh")]
 
 
 def nvcc_path():
@@ -48,6 +53,18 @@ def build(force=False, verbose=False, extra=()):
     return LIB
 
 
+def build_test_lib(force=False, verbose=False):
+    """Compile the test build (-DSA_TEST_HOOKS) if it is out of date; return its path."""
+    if not force and up_to_date(TEST_LIB):
+        return TEST_LIB
+    cmd = command(out=TEST_LIB, extra=["-DSA_TEST_HOOKS"])
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    return TEST_LIB
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
           extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
+    build_test_lib(force="--force" in sys.argv, verbose=True)

@@ -10,28 +10,32 @@
 #include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <new>
 #include <vector>
 
 #include "sa_bwd.cuh"
+#include "sa_bwd_wide.cuh"
 #include "sa_device.cuh"
 #include "sa_fwd.cuh"
 #include "sa_internal.h"
+#include "sa_tail.cuh"
 #include "sparse_attn.h"
 
 namespace sa {
 namespace {
 
 // ------------------------------------------------------------ instrumentation
-enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_FINAL, K_KERNELS };
-const char* const kKernelNames[K_KERNELS] = {"sa_fwd_column_view", "sa_fwd_natural_view",
-                                             "sa_bwd_preprocess",  "sa_bwd_secondary_view",
-                                             "sa_bwd_natural_view", "sa_bwd_finalize_dq"};
+enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_FINAL, K_FWD_TAIL, K_BWD_TAIL, K_KERNELS };
+const char* const kKernelNames[K_KERNELS] = {"sa_fwd_column_view",  "sa_fwd_natural_view", "sa_bwd_preprocess",
+                                             "sa_bwd_secondary_view", "sa_bwd_natural_view", "sa_bwd_finalize_dq",
+                                             "sa_fwd_partial_row",  "sa_bwd_partial_row"};
 constexpr int K_PATTERNS = 7;
 const char* const kPatternNames[K_PATTERNS] = {"all", "local", "strided", "fixed", "column", "block", "blocks"};
-// Instrumentation kinds: one per (kernel, pattern), kind = kernel * 4 + pattern.
+// Instrumentation kinds: one per (kernel, pattern), kind = kernel * K_PATTERNS + pattern.
 constexpr int K_NUM = K_KERNELS * K_PATTERNS;
 char g_kind_names[K_NUM][48];
 std::once_flag g_names_once;
@@ -109,6 +113,69 @@ int launch(int kind, cudaStream_t s, F&& f) {
   return err == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
+// Launches a kernel with programmatic stream serialisation, so that it can
+// start its set-up while the previous kernel in the stream drains (every
+// kernel of the library waits for its predecessor with griddepcontrol.wait
+// before touching global memory).  SA_NO_PDL=1 in the environment launches
+// normally instead.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SA_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+template <class... P, class... A>
+void launch_kernel(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
+#ifdef SA_TEST_HOOKS
+// Range check of a device tile table (test build): row pointers start at 0,
+// never decrease and end at nnz; every entry's tile index lies in
+// [0, max_tile); every launch slot names a row and that row's entries.
+// Records SA_ERR_LUT in the status word; the kernels launched after it then
+// return before touching any table or tensor.
+__global__ void sa_check_table_kernel(DevTable t, int max_tile) {
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x, nth = gridDim.x * blockDim.x;
+  bool bad = false;
+  if (tid == 0) bad = t.row_ptr[0] != 0 || t.row_ptr[t.n_rows] != t.nnz;
+  for (int i = tid; i < t.n_rows; i += nth) {
+    bad |= t.row_ptr[i + 1] < t.row_ptr[i];
+    const int o = t.order[i];
+    bad |= o < 0 || o >= t.n_rows;
+    const int4 sc = *reinterpret_cast<const int4*>(t.sched + 4 * i);
+    bad |= sc.x < 0 || sc.x >= t.n_rows || sc.y < 0 || sc.z < 0 || sc.y + sc.z > t.nnz;
+  }
+  for (int i = tid; i < t.nnz; i += nth) {
+    const int tile = t.ent[i] >> 3;
+    bad |= tile < 0 || tile >= max_tile || ((t.ent[i] >> 1) & 3) > SRC_S;
+  }
+  if (bad) atomicExch(&g_status, kStatusLut);
+}
+
+int check_tables(const DeviceCopy& dc, int N, cudaStream_t s) {
+  const DevTable* ts[6] = {&dc.fwd_main, &dc.fwd_col, &dc.bwd_main, &dc.bwd_sec, &dc.bwd_main_w, &dc.bwd_sec_w};
+  for (const DevTable* t : ts) {
+    if (t->n_rows == 0) continue;
+    sa_check_table_kernel<<<8, 256, 0, s>>>(*t, N / 64 + 2);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+#endif
+
 // ------------------------------------------------------------ tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -144,7 +211,7 @@ int map_nat(CUtensorMap* m, const void* base, const Geo& g, int rows) {
 
 // The sequence as a 2-D array with rows of length l: {D, l, R, BH}.
 // Column view box {boxw, 1, min(R, rows), 1}; summary box
-// {boxw, min(c, rows), max(1, rows / c), 1}.
+// {boxw, cb, gb, 1} from summary_box(c, rows).
 int map_grid(CUtensorMap* m, const void* base, const Geo& g, uint32_t b1, uint32_t b2) {
   const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
   const cuuint64_t strides[3] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.l * g.D * 2, (cuuint64_t)g.N * g.D * 2};
@@ -180,7 +247,7 @@ int make_dq_maps(CUtensorMap* nat, CUtensorMap* col, const float* base, const Ge
   if (pattern == SA_STRIDED || pattern == SA_COLUMN) {
     const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
     const cuuint64_t strides[3] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.l * g.D * 4, (cuuint64_t)g.N * g.D * 4};
-    const cuuint32_t box[4] = {32, 1, (cuuint32_t)std::min(g.R, 32), 1};
+    const cuuint32_t box[4] = {32, 1, (cuuint32_t)gcd_int(g.R, 32), 1};
     if (g_encode(col, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(base), dims, strides, box, es,
                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -215,7 +282,7 @@ int make_epi_maps(EpiMaps* em, const void* dk, const void* dv, const float* dk_p
       if (key_view == SRC_T) {  // column-major rows: {D, l, R, BH}, box {D, 1, min(R, 32), 1}
         const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
         const cuuint64_t strides[3] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.l * g.D * 2, (cuuint64_t)g.N * g.D * 2};
-        const cuuint32_t box[4] = {(cuuint32_t)g.D, 1, (cuuint32_t)std::min(g.R, 32), 1};
+        const cuuint32_t box[4] = {(cuuint32_t)g.D, 1, (cuuint32_t)gcd_int(g.R, 32), 1};
         r = g_encode(outs[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(bases[i]), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -244,9 +311,10 @@ int make_epi_maps(EpiMaps* em, const void* dk, const void* dv, const float* dk_p
     } else {
       const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
       const cuuint64_t strides[3] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.l * g.D * 4, (cuuint64_t)g.N * g.D * 4};
-      const cuuint32_t box[4] = {32, key_view == SRC_T ? 1u : (cuuint32_t)std::min(g.c, 32),
-                                 key_view == SRC_T ? (cuuint32_t)std::min(g.R, 32) : (cuuint32_t)std::max(1, 32 / g.c),
-                                 1};
+      int cb = 1, gb = 1;
+      summary_box(g.c, 32, &cb, &gb);
+      const cuuint32_t box[4] = {32, key_view == SRC_T ? 1u : (cuuint32_t)cb,
+                                 key_view == SRC_T ? (cuuint32_t)gcd_int(g.R, 32) : (cuuint32_t)gb, 1};
       r = g_encode(parts[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(pbases[i]), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -261,11 +329,13 @@ int make_maps(MapSet* ms, const void* base, const Geo& g, int pattern, int rows)
   int st = map_nat(&ms->nat, base, g, rows);
   if (st) return st;
   if (pattern == SA_STRIDED || pattern == SA_COLUMN) {
-    st = map_grid(&ms->col, base, g, 1, (uint32_t)std::min(g.R, rows));
+    st = map_grid(&ms->col, base, g, 1, (uint32_t)gcd_int(g.R, rows));
     if (st) return st;
   }
   if (pattern == SA_FIXED) {
-    st = map_grid(&ms->sum, base, g, (uint32_t)std::min(g.c, rows), (uint32_t)std::max(1, rows / g.c));
+    int cb = 1, gb = 1;
+    summary_box(g.c, rows, &cb, &gb);
+    st = map_grid(&ms->sum, base, g, (uint32_t)cb, (uint32_t)gb);
     if (st) return st;
   }
   return SA_OK;
@@ -281,10 +351,11 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
       *out = d;
       return SA_OK;
     }
-  const TileTable* tabs[4] = {&L->fwd_main, &L->fwd_col, &L->bwd_main, &L->bwd_sec};
+  constexpr int NT = 6;
+  const TileTable* tabs[NT] = {&L->fwd_main, &L->fwd_col, &L->bwd_main, &L->bwd_sec, &L->bwd_main_w, &L->bwd_sec_w};
   std::vector<int32_t> blob;
-  size_t offs[4][4];
-  for (int t = 0; t < 4; ++t) {
+  size_t offs[NT][4];
+  for (int t = 0; t < NT; ++t) {
     const TileTable& tt = *tabs[t];
     offs[t][3] = blob.size();  // 16-byte aligned: every section is padded to 4 ints
     blob.insert(blob.end(), tt.sched.begin(), tt.sched.end());
@@ -308,9 +379,9 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
   DeviceCopy d;
   d.device = dev;
   d.blob = dptr;
-  DevTable* dts[4] = {&d.fwd_main, &d.fwd_col, &d.bwd_main, &d.bwd_sec};
+  DevTable* dts[NT] = {&d.fwd_main, &d.fwd_col, &d.bwd_main, &d.bwd_sec, &d.bwd_main_w, &d.bwd_sec_w};
   const int32_t* base = static_cast<const int32_t*>(dptr);
-  for (int t = 0; t < 4; ++t) {
+  for (int t = 0; t < NT; ++t) {
     dts[t]->row_ptr = base + offs[t][0];
     dts[t]->ent = base + offs[t][1];
     dts[t]->order = base + offs[t][2];
@@ -331,13 +402,12 @@ int check_call(int B, int H, int N, int D, const sa_layout* L) {
   if (static_cast<long long>(B) * H > 0x7fffffffLL) return SA_ERR_INVALID_ARG;
   if (L->N != N) return SA_ERR_LUT;
   if (D != 32 && D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
-  if (L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) {
-    const int R = L->R;
-    if (R % 8 != 0 || !(R % 128 == 0 || 128 % R == 0)) return SA_ERR_UNSUPPORTED;
-  }
-  if (L->pattern == SA_FIXED) {
-    const int c = L->c;
-    if (!(64 % c == 0 || c % 128 == 0)) return SA_ERR_UNSUPPORTED;
+  if (D == 32) {
+    // Rows of 64 bytes: a TMA box must start on a 128-byte boundary of shared
+    // memory, so the column and summary views cannot be moved in runs of an
+    // odd number of rows (odd R; odd c above 1).
+    if ((L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) && (L->R & 1)) return SA_ERR_UNSUPPORTED;
+    if (L->pattern == SA_FIXED && L->c > 1 && (L->c & 1)) return SA_ERR_UNSUPPORTED;
   }
   if (!have_encode()) return SA_ERR_CUDA;
   return SA_OK;
@@ -387,10 +457,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   std::memset(&mo_col, 0, sizeof(mo_col));
   if ((st = map_nat(&mo_nat, o, g, 32))) return st;
   if ((L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) &&
-      (st = map_grid(&mo_col, o, g, 1, static_cast<uint32_t>(std::min(g.R, 32)))))
+      (st = map_grid(&mo_col, o, g, 1, static_cast<uint32_t>(gcd_int(g.R, 32)))))
     return st;
   DeviceCopy dc;
   if ((st = to_device(L, &dc))) return st;
+#ifdef SA_TEST_HOOKS
+  if ((st = check_tables(dc, N, s))) return st;
+#endif
   auto kern = sa_fwd_kernel<D>;
   if ((st = set_smem(kern, FwdCfg<D>::SMEM))) return st;
   FwdArgs a;
@@ -414,8 +487,21 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     a.merge = 0;
     dim3 grid(g.BH, dc.fwd_col.n_rows);
     st = launch(K_FWD_COL * K_PATTERNS + L->pattern, s, [&] {
-      kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum,
-                                                                       mo_nat, mo_col, a);
+      launch_kernel(kern, grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s, mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat,
+                    mv.col, mv.sum, mo_nat, mo_col, a);
+    });
+    if (st) return st;
+  }
+  // The partial last row of a strided pattern (N not a multiple of l): its
+  // column part on CUDA cores, merged below like the column view's.
+  const int r_tail = (L->pattern == SA_STRIDED && L->R > 0) ? N - L->R * L->l : 0;
+  if (r_tail > 0) {
+    const long long warps = static_cast<long long>(g.BH) * r_tail;
+    st = launch(K_FWD_TAIL * K_PATTERNS + L->pattern, s, [&] {
+      launch_kernel(sa_tail_fwd_kernel<D>, static_cast<unsigned>((warps + 3) / 4), 128, 0, s,
+                    static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                    static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(o), lse, g.BH, N, L->l, L->R,
+                    a.scale_log2);
     });
     if (st) return st;
   }
@@ -423,12 +509,12 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.ent = dc.fwd_main.ent;
   a.order = dc.fwd_main.order;
   a.q_col = 0;
-  a.merge = col_pass ? 1 : 0;
+  a.merge = (col_pass || r_tail > 0) ? 1 : 0;
   if (dc.fwd_main.n_rows == 0) return SA_OK;  // SA_COLUMN: no natural view
   dim3 grid(g.BH, dc.fwd_main.n_rows);
   return launch(K_FWD_MAIN * K_PATTERNS + L->pattern, s, [&] {
-    kern<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s>>>(mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum,
-                                                                       mo_nat, mo_col, a);
+    launch_kernel(kern, grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s, mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat,
+                  mv.col, mv.sum, mo_nat, mo_col, a);
   });
 }
 
@@ -455,7 +541,7 @@ WsLayout ws_layout(int B, int H, int N, int D, const sa_layout* L) {
   const size_t BH = static_cast<size_t>(B) * H;
   const size_t rows = BH * N;
   WsLayout w;
-  w.n_pad = (N + BwdCfg<64>::TQ - 1) / BwdCfg<64>::TQ * BwdCfg<64>::TQ;
+  w.n_pad = (N + kBwdWideTQ - 1) / kBwdWideTQ * kBwdWideTQ;  // whole steps of either kernel shape
   const size_t ld_bytes = align256(BH * w.n_pad * 8);  // two floats per query position
   w.ld_nat = 0;
   w.ld_col = ld_bytes;
@@ -487,11 +573,22 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = make_maps(&mv, v, g, L->pattern, BwdCfg<D>::TK))) return st;
   DeviceCopy dc;
   if ((st = to_device(L, &dc))) return st;
+#ifdef SA_TEST_HOOKS
+  if ((st = check_tables(dc, N, s))) return st;
+#endif
   if ((st = set_smem(sa_bwd_kernel<D, false, false>, BwdCfg<D, false>::SMEM))) return st;
   if ((st = set_smem(sa_bwd_kernel<D, false, true>, BwdCfg<D, false>::SMEM))) return st;
   if constexpr (D <= 64) {
     if ((st = set_smem(sa_bwd_kernel<D, true, false>, BwdCfg<D, true>::SMEM))) return st;
     if ((st = set_smem(sa_bwd_kernel<D, true, true>, BwdCfg<D, true>::SMEM))) return st;
+  }
+  // Q / dO maps with 128-row boxes for the wide-step shape (D = 64)
+  MapSet mq_w, mdo_w;
+  if constexpr (D == 64) {
+    if ((st = set_smem(sa_bwd_wide_kernel<false>, WideCfg::SMEM))) return st;
+    if ((st = set_smem(sa_bwd_wide_kernel<true>, WideCfg::SMEM))) return st;
+    if ((st = make_maps(&mq_w, q, g, L->pattern, WideCfg::TQ))) return st;
+    if ((st = make_maps(&mdo_w, dO, g, L->pattern, WideCfg::TQ))) return st;
   }
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -506,9 +603,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = make_dq_maps(&mdq_nat, &mdq_col, dq_acc, g, L->pattern))) return st;
 
   st = launch(K_BWD_PRE * K_PATTERNS + L->pattern, s, [&] {
-    sa_bwd_pre_kernel<D><<<grid_for(rows * (D / 8), 256), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ld_nat, ld_col, dq_acc,
-        g.BH, N, w.n_pad, g.l, g.R);
+    launch_kernel(sa_bwd_pre_kernel<D>, grid_for(rows * (D / 8), 256), 256, 0, s,
+                  static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ld_nat, ld_col,
+                  dq_acc, g.BH, N, w.n_pad, g.l, g.R);
   });
   if (st) return st;
 
@@ -533,8 +630,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   const bool sec_final = L->pattern == SA_COLUMN;
   a.BH = g.BH;
   const int n_sm = sm_count();
-  // Tables whose items average many steps take the LONG shape of the kernel.
-  auto run = [&](int kind, const DevTable& t) -> int {
+  // Tables whose items average many steps take the LONG shape of the kernel;
+  // for D = 64 that is the wide-step kernel on the 128-query-step table.
+  auto run = [&](int kind, const DevTable& t, const DevTable& tw) -> int {
     EpiMaps em;
     const int mst = make_epi_maps(&em, dk, dv, dk_part, dv_part, g, a.key_view);
     if (mst) return mst;
@@ -543,9 +641,23 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     const bool long_items = D <= 64 && t.nnz >= kBwdLongSteps * static_cast<long long>(t.n_rows);
     const bool final_t = sec_final && a.key_view == SRC_T;
     auto go = [&](auto kernel, int threads, int smem) {
-      kernel<<<grid, threads, smem, s>>>(mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat, mv.col,
-                                         mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v, em.part_k, em.part_v, a);
+      launch_kernel(kernel, grid, threads, smem, s, mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
+                    mv.col, mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v, em.part_k, em.part_v, a);
     };
+    if constexpr (D == 64) {
+      if (long_items) {
+        BwdArgs aw = a;
+        aw.sched = tw.sched;
+        aw.ent = tw.ent;
+        aw.n_slots = tw.n_rows;
+        return launch(kind, s, [&] {
+          auto kernel = final_t ? sa_bwd_wide_kernel<true> : sa_bwd_wide_kernel<false>;
+          launch_kernel(kernel, grid, WideCfg::THREADS, WideCfg::SMEM, s, mq_w.nat, mq_w.col, mdo_w.nat, mdo_w.col,
+                        mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v,
+                        em.part_k, em.part_v, aw);
+        });
+      }
+    }
     return launch(kind, s, [&] {
       if constexpr (D <= 64) {
         if (long_items) {
@@ -566,7 +678,19 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_sec.n_rows;
     a.key_view = (L->pattern == SA_FIXED) ? SRC_S : SRC_T;
     a.add_part = 0;
-    if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec))) return st;
+    if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec, dc.bwd_sec_w))) return st;
+  }
+  const int r_tail = (L->pattern == SA_STRIDED && L->R > 0) ? N - L->R * L->l : 0;
+  if (r_tail > 0) {  // the partial last row's column part (after the column view's pass)
+    const long long warps = static_cast<long long>(g.BH) * r_tail;
+    st = launch(K_BWD_TAIL * K_PATTERNS + L->pattern, s, [&] {
+      launch_kernel(sa_tail_bwd_kernel<D>, static_cast<unsigned>((warps + 3) / 4), 128, 0, s,
+                    static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                    static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(dO),
+                    static_cast<const float*>(ld_nat), dq_acc, dk_part, dv_part, g.BH, N, L->l, L->R, w.n_pad, scale,
+                    a.scale_log2);
+    });
+    if (st) return st;
   }
   if (dc.bwd_main.n_rows > 0) {
     a.sched = dc.bwd_main.sched;
@@ -574,11 +698,12 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_main.n_rows;
     a.key_view = SRC_N;
     a.add_part = (sec && !sec_final) ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
-    if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main))) return st;
+    if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main, dc.bwd_main_w))) return st;
   }
   const long long n8 = rows * D / 8;
   return launch(K_BWD_FINAL * K_PATTERNS + L->pattern, s, [&] {
-    sa_bwd_final_kernel<<<grid_for(n8, 256), 256, 0, s>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+    launch_kernel(sa_bwd_final_kernel, grid_for(n8, 256), 256, 0, s, static_cast<const float*>(dq_acc),
+                  static_cast<__nv_bfloat16*>(dq), n8);
   });
 }
 
@@ -619,8 +744,14 @@ int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** 
   if (pattern != SA_ALL && l < 1) return SA_ERR_INVALID_ARG;
   if (pattern == SA_FIXED && (c < 1 || c > l)) return SA_ERR_INVALID_ARG;
   if (N % block != 0) return SA_ERR_UNSUPPORTED;
-  const bool grid2d = pattern == SA_STRIDED || pattern == SA_FIXED || pattern == SA_COLUMN;  // R = N / l rows
-  if (grid2d && N % l != 0) return SA_ERR_UNSUPPORTED;
+  // R = N / l whole rows of the 2-D view.  With N not a multiple of l, the
+  // fixed pattern's summary view keeps the whole blocks (the keys of a
+  // partial last block are seen by no later block), and the strided
+  // pattern's column view covers the whole rows while the partial row's
+  // column part runs in its own kernels.  The single column head (SA_COLUMN)
+  // needs whole rows.
+  const bool grid2d = pattern == SA_STRIDED || pattern == SA_FIXED || pattern == SA_COLUMN;
+  if (pattern == SA_COLUMN && N % l != 0) return SA_ERR_UNSUPPORTED;
   sa_layout* L = new (std::nothrow) sa_layout();
   if (!L) return SA_ERR_INVALID_ARG;
   L->pattern = pattern;
@@ -858,3 +989,25 @@ extern "C" int sparse_attn_bwd_noalloc(const void* q, const void* k, const void*
   return sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, D, L, scratch, SA_NOALLOC_SCRATCH_BYTES,
                          stream);
 }
+
+#ifdef SA_TEST_HOOKS
+// ==================================================================== test build only
+// Not part of the ABI (the header does not declare them): hooks of the
+// failure-detection tests, exported by libsparse_attn_test.so alone.
+extern "C" int sparse_attn_test_withhold(int on) {
+  return cudaMemcpyToSymbol(g_test_withhold, &on, sizeof(int)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+// Overwrites entry `index` of the forward natural-view tile table of the
+// layout's copy on the current device with `value` (a corrupted table).
+extern "C" int sparse_attn_test_corrupt_entry(const sa_layout* L, int index, int value) {
+  DeviceCopy dc;
+  const int st = to_device(L, &dc);
+  if (st) return st;
+  if (index < 0 || index >= dc.fwd_main.nnz) return SA_ERR_INVALID_ARG;
+  return cudaMemcpy(const_cast<int32_t*>(dc.fwd_main.ent) + index, &value, sizeof(int), cudaMemcpyHostToDevice) ==
+                 cudaSuccess
+             ? SA_OK
+             : SA_ERR_CUDA;
+}
+#endif

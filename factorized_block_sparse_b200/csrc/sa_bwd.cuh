@@ -174,7 +174,7 @@ template <int D, bool T_DIAG>
 __device__ __forceinline__ KeyRow key_row(const BwdArgs& a, int kt, int row) {
   KeyRow k;
   k.y = kt * BwdCfg<D>::TK + row;
-  const int nkeys = (a.key_view == SRC_S) ? a.R * a.c : a.N;
+  const int nkeys = (a.key_view == SRC_S) ? a.R * a.c : (a.key_view == SRC_T ? a.R * a.l : a.N);
   k.kvalid = k.y < nkeys;
   if (a.key_view == SRC_T) k.knat = (k.y % a.R) * a.l + k.y / a.R;
   else if (a.key_view == SRC_S) k.knat = (k.y / a.c) * a.l + (a.l - a.c) + k.y % a.c;
@@ -246,6 +246,10 @@ __global__ void __launch_bounds__(480, 1)
                   const __grid_constant__ CUtensorMap mdk_part, const __grid_constant__ CUtensorMap mdv_part,
                   const BwdArgs a) {
   using C = BwdCfg<D, LONG>;
+#ifdef SA_TEST_HOOKS
+  pdl_wait();  // the range check of the tables (previous kernel) has completed
+  if (*(volatile int*)&g_status == kStatusLut) return;  // a table failed it: touch nothing
+#endif
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + C::OFF_K;
@@ -320,6 +324,8 @@ __global__ void __launch_bounds__(480, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -683,7 +689,7 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
               for (int bx = 0; bx < D / 32; ++bx) {
                 if (q_src == SRC_T) {
-                  const int rb = a.R < 32 ? a.R : 32;
+                  const int rb = gcd_int(a.R, 32);
                   for (int s0 = 0; s0 < 32; s0 += rb) {
                     const int t = xw + s0;
                     tma_reduce_add_4d(&mdq_col, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
@@ -732,8 +738,8 @@ __global__ void __launch_bounds__(480, 1)
         const int y0 = it.kt * C::TK + quarter * 32;  // first view key of the warp
         const bool nat_out = a.key_view == SRC_N || FINAL_T;  // bf16 rows (else fp32 partials)
         bool row_add = false;
-        if (nat_out && a.add_part == 1) row_add = kr.kvalid;
-        else if (nat_out && a.add_part == 2) row_add = kr.kvalid && (kr.knat % a.l) >= (a.l - a.c);
+        if (nat_out && a.add_part == 1) row_add = kr.kvalid && kr.knat < a.R * a.l;  // keys of whole rows
+        else if (nat_out && a.add_part == 2) row_add = kr.kvalid && (kr.knat % a.l) >= (a.l - a.c) && kr.knat < a.R * a.l;
         const bool warp_add = __any_sync(0xffffffffu, row_add);
 #pragma unroll 1
         for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
@@ -801,7 +807,7 @@ __global__ void __launch_bounds__(480, 1)
           __syncwarp();
           if (lane == 0) {
             if constexpr (FINAL_T) {  // rows of the column runs
-              const int rb = a.R < 32 ? a.R : 32;
+              const int rb = gcd_int(a.R, 32);
               for (int s0 = 0; s0 < 32; s0 += rb) {
                 const int t = y0 + s0;
                 tma_store_4d(which ? &mdk_out : &mdv_out, stg + s0 * (D * 2), 0, t / a.R, t % a.R, it.bh);
@@ -813,15 +819,22 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
               for (int bx = 0; bx < D / 32; ++bx) {
                 if (a.key_view == SRC_T) {
-                  const int rb = a.R < 32 ? a.R : 32;
+                  const int rb = gcd_int(a.R, 32);
                   for (int s0 = 0; s0 < 32; s0 += rb) {
                     const int t = y0 + s0;
                     tma_store_4d(mp, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
                   }
-                } else if (a.c >= 32) {
-                  tma_store_4d(mp, stg + bx * 4096, bx * 32, a.l - a.c + y0 % a.c, y0 / a.c, it.bh);
                 } else {
-                  tma_store_4d(mp, stg + bx * 4096, bx * 32, a.l - a.c, y0 / a.c, it.bh);
+                  int cb, gb;
+                  summary_box(a.c, 32, &cb, &gb);
+                  if (gb > 1 || cb == a.c) {  // whole blocks
+                    tma_store_4d(mp, stg + bx * 4096, bx * 32, a.l - a.c, y0 / a.c, it.bh);
+                  } else {  // runs of cb keys inside one block
+                    for (int s0 = 0; s0 < 32; s0 += cb) {
+                      const int y = y0 + s0;
+                      tma_store_4d(mp, stg + bx * 4096 + s0 * 128, bx * 32, a.l - a.c + y % a.c, y / a.c, it.bh);
+                    }
+                  }
                 }
               }
             }
@@ -832,8 +845,8 @@ __global__ void __launch_bounds__(480, 1)
       } else {
       const size_t off = (static_cast<size_t>(it.bh) * a.N + (kr.kvalid ? kr.knat : 0)) * D;
       bool add = false;
-      if (a.add_part == 1) add = true;
-      else if (a.add_part == 2) add = (kr.knat % a.l) >= (a.l - a.c);
+      if (a.add_part == 1) add = kr.knat < a.R * a.l;
+      else if (a.add_part == 2) add = (kr.knat % a.l) >= (a.l - a.c) && kr.knat < a.R * a.l;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
         const uint32_t col = (which ? C::COL_DK : C::COL_DV) + (ne % C::DKVB) * 2 * D;
@@ -889,6 +902,8 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
                                                          int l, int R) {
   constexpr int TPR = D / 8;         // threads per row
   constexpr int RPW = 32 / TPR;      // rows per warp per step
+  pdl_wait();
+  pdl_trigger();
   const long long rows = static_cast<long long>(BH) * N;
   const int lane = threadIdx.x & 31;
   const int sub = lane % TPR;
@@ -923,7 +938,7 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
         const long long o = bh * n_pad * 2;
         ld_nat[o + (i / 64) * 128 + (i % 64)] = nl;
         ld_nat[o + (i / 64) * 128 + 64 + (i % 64)] = -acc;
-        if (ld_col) {
+        if (ld_col && i < R * l) {  // rows of a partial last row are not in the column view
           const int t = (i % l) * R + i / l;
           ld_col[o + (t / 64) * 128 + (t % 64)] = nl;
           ld_col[o + (t / 64) * 128 + 64 + (t % 64)] = -acc;
@@ -941,7 +956,13 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
     const long long o = bh * n_pad * 2 + (i / 64) * 128 + (i % 64);
     ld_nat[o] = -INFINITY;
     ld_nat[o + 64] = 0.f;
-    if (ld_col) {
+  }
+  if (ld_col) {  // the column view covers the R l positions of whole rows
+    const int pad_c = n_pad - R * l;
+    for (long long k = tid; k < static_cast<long long>(BH) * pad_c; k += nthr) {
+      const long long bh = k / pad_c;
+      const long long i = static_cast<long long>(R) * l + (k - bh * pad_c);
+      const long long o = bh * n_pad * 2 + (i / 64) * 128 + (i % 64);
       ld_col[o] = -INFINITY;
       ld_col[o + 64] = 0.f;
     }
@@ -952,6 +973,8 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
 __global__ void __launch_bounds__(256) sa_bwd_final_kernel(const float* __restrict__ acc,
                                                            __nv_bfloat16* __restrict__ dq,
                                                            long long n8) {
+  pdl_wait();
+  pdl_trigger();
   const long long nthreads = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += nthreads) {
     const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];

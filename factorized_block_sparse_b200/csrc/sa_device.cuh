@@ -19,6 +19,42 @@ namespace sa {
 __device__ int g_status = 0;
 
 constexpr int kStatusTimeout = 5;  // == SA_ERR_TIMEOUT
+constexpr int kStatusLut = 4;      // == SA_ERR_LUT
+
+#ifdef SA_TEST_HOOKS
+// Test build (libsparse_attn_test.so, for the failure-detection tests only):
+// device-side waits give up after about 2^22 cycles (a few milliseconds), a
+// flag makes the backward producer withhold one load so that a wait runs
+// out, and the device tables are range-checked before the kernels use them.
+constexpr long long kWaitCycles = 1LL << 22;
+__device__ int g_test_withhold = 0;
+#else
+constexpr long long kWaitCycles = 1LL << 31;
+#endif
+
+// Rows per TMA box of the column-major view (runs of R rows) and the summary
+// view (runs of c keys per block) for a tile of `rows` view positions that
+// starts at a multiple of `rows`: every box stays inside one run.
+__host__ __device__ __forceinline__ int gcd_int(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+// Summary-view box for a tile of `rows` keys: {cb rows of a block, gb blocks}.
+// Whole blocks when c divides rows, part of one block when rows divides c,
+// else boxes of gcd(c, rows) rows.
+__host__ __device__ __forceinline__ void summary_box(int c, int rows, int* cb, int* gb) {
+  if (rows % c == 0) {
+    *cb = c;
+    *gb = rows / c;
+  } else {
+    *cb = gcd_int(c, rows);
+    *gb = 1;
+  }
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -76,7 +112,7 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 }
 
 // Bounded wait for the phase with the given parity.  After about 2^31 SM
-// cycles without completion (or once any CTA has already recorded a
+// cycles (2^22 in the test build) without completion (or once any CTA has already recorded a
 // timeout) it records SA_ERR_TIMEOUT in the status word, sets *abort and
 // returns false; callers then skip the remaining work and drain.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* abort) {
@@ -90,7 +126,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* a
         *(volatile int*)abort = 1;
         return false;
       }
-      if (clock64() - t0 > (1LL << 31)) {
+      if (clock64() - t0 > kWaitCycles) {
         atomicExch(&g_status, kStatusTimeout);
         *(volatile int*)abort = 1;
         return false;
@@ -99,6 +135,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* a
   }
   return true;
 }
+
+// ------------------------------------------------ programmatic dependent launch
+// The library launches its kernels with programmatic stream serialisation:
+// a kernel may start (barrier set-up, TMEM allocation, static table reads)
+// while the previous kernel in the stream drains.  pdl_wait() blocks until
+// that kernel has completed and its writes are visible; every kernel calls it
+// before its first access to data another kernel may write or read.  It
+// returns at once for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel in the stream begin launching; its CTAs start once
+// every CTA of this grid has called this or exited.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {

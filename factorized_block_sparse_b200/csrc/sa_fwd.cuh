@@ -75,9 +75,9 @@ struct FwdCfg {
 // `dst` (PANELS panels of rows x ROWB bytes).
 //   src N: natural order, 3-D map {D, N, BH}, box {BOXW, rows, 1}
 //   src T: column-major order, 4-D map {D, l, R, BH}, box {BOXW, 1, RB, 1}
-//          with RB = min(R, rows): one load per column segment
-//   src S: summary order, 4-D map {D, l, R, BH}, box {BOXW, CB, GB, 1} with
-//          CB = min(c, rows), GB = max(1, rows / c)
+//          with RB = gcd(R, rows): one load per RB rows of a column
+//   src S: summary order, 4-D map {D, l, R, BH}, box {BOXW, CB, GB, 1} from
+//          summary_box(c, rows): whole blocks, or runs inside one block
 template <int D>
 __device__ __forceinline__ void load_rows(uint8_t* dst, int src, int pos0, int rows, int bh,
                                           const CUtensorMap* m_nat, const CUtensorMap* m_col,
@@ -92,16 +92,21 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, int src, int pos0, int r
     if (src == SRC_N) {
       tma_load_3d(d, m_nat, bar, x, pos0, bh);
     } else if (src == SRC_T) {
-      const int rb = R < rows ? R : rows;
+      const int rb = gcd_int(R, rows);
       for (int s = 0; s < rows; s += rb) {
         const int t = pos0 + s;
         tma_load_4d(d + s * C::ROWB, m_col, bar, x, t / R, t % R, bh);
       }
     } else {
-      if (c >= rows) {
-        tma_load_4d(d, m_sum, bar, x, l - c + (pos0 % c), pos0 / c, bh);
-      } else {
+      int cb, gb;
+      summary_box(c, rows, &cb, &gb);
+      if (gb > 1 || cb == c) {  // whole blocks
         tma_load_4d(d, m_sum, bar, x, l - c, pos0 / c, bh);
+      } else {  // runs of cb keys inside one block
+        for (int s = 0; s < rows; s += cb) {
+          const int y = pos0 + s;
+          tma_load_4d(d + s * C::ROWB, m_sum, bar, x, l - c + y % c, y / c, bh);
+        }
       }
     }
   }
@@ -135,6 +140,10 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
                   const __grid_constant__ CUtensorMap mo_nat, const __grid_constant__ CUtensorMap mo_col,
                   const FwdArgs a) {
   using C = FwdCfg<D>;
+#ifdef SA_TEST_HOOKS
+  pdl_wait();  // the range check of the tables (previous kernel) has completed
+  if (*(volatile int*)&g_status == kStatusLut) return;  // a table failed it: touch nothing
+#endif
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -185,6 +194,8 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0 && n > 0) {
@@ -259,7 +270,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int x = qt * C::TQ + row;  // view position of this query
-    const bool valid = x < a.N;
+    const bool valid = x < (a.q_col ? a.R * a.l : a.N);  // the column view covers whole rows
     const int nat = a.q_col ? (x % a.R) * a.l + x / a.R : x;
     // key intervals by source view (inclusive)
     int lo_n, hi_n;
@@ -436,7 +447,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
 #pragma unroll
       for (int p = 0; p < C::PANELS; ++p) {
         if (a.q_col) {
-          const int rb = a.R < 32 ? a.R : 32;
+          const int rb = gcd_int(a.R, 32);
           for (int s0 = 0; s0 < 32; s0 += rb) {
             const int t = xw + s0;
             tma_store_4d(&mo_col, stg + p * PB + s0 * C::ROWB, p * 64, t / a.R, t % a.R, bh);

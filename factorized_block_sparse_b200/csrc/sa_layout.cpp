@@ -42,8 +42,20 @@ Interval key_interval(const sa_layout* L, int view, long long x) {
         return {(x / l) * l, x};
     }
   }
-  if (view == SA_VIEW_COLUMN) {  // inside the column run of length R; strict unless the
-    return {(x / R) * R, L->pattern == SA_COLUMN ? x : x - 1};  // view stands alone
+  if (view == SA_VIEW_COLUMN) {
+    // Inside the run of x's column, strict unless the view stands alone.
+    // Column-major order: columns 0 .. r-1 hold R + 1 positions when N is not
+    // a multiple of l (r = N - R l, the length of the partial last row), the
+    // others R.
+    const long long r = L->N - R * l;
+    long long start;
+    if (x < r * (R + 1)) {
+      start = (x / (R + 1)) * (R + 1);
+    } else {
+      const long long c = r + (x - r * (R + 1)) / R;
+      start = r * (R + 1) + (c - r) * R;
+    }
+    return {start, L->pattern == SA_COLUMN ? x : x - 1};
   }
   // SA_VIEW_SUMMARY: summary keys of strictly earlier blocks
   return {0, (x / l) * c - 1};
@@ -54,7 +66,7 @@ Csr build_public(const sa_layout* L, int view) {
   const int b = L->block;
   const long long nq = L->N;
   const long long nk = view_keys(L, view);
-  t.n_rows = static_cast<int>(nq / b);
+  t.n_rows = static_cast<int>((nq + b - 1) / b);
   t.n_cols = static_cast<int>((nk + b - 1) / b);
   t.row_ptr.assign(1, 0);
   std::vector<Interval> iv(b);
@@ -184,10 +196,43 @@ void finish_table(TileTable& tt, const std::vector<std::vector<int32_t>>& rows) 
   }
 }
 
+// The same key tiles with 128-query steps: query tile t of a 64-query table
+// becomes step t / 2.  A step is FULL only when both of its 64-query halves
+// are listed and FULL; a half that is missing (outside the key tile's
+// queries, or past the end of the view) is masked like any PARTIAL part.
+void widen(const TileTable& t64, TileTable& out) {
+  std::vector<std::vector<int32_t>> rows(t64.n_rows);
+  for (int r = 0; r < t64.n_rows; ++r) {
+    int cur = -1, src = 0, halves = 0, part = 0;
+    auto flush = [&] {
+      if (cur >= 0) rows[r].push_back(pack_entry(cur, src, (part || halves != 2) ? 1 : 0));
+    };
+    for (int e = t64.row_ptr[r]; e < t64.row_ptr[r + 1]; ++e) {
+      const int32_t v = t64.ent[e];
+      const int w = (v >> 3) / 2;
+      if (w != cur) {
+        flush();
+        cur = w;
+        src = (v >> 1) & 3;
+        halves = 0;
+        part = 0;
+      }
+      ++halves;
+      part |= v & 1;
+    }
+    flush();
+  }
+  finish_table(out, rows);
+}
+
 }  // namespace
 
 int view_keys(const sa_layout* L, int view) {
-  if (view == SA_VIEW_SUMMARY) return L->R * L->c;
+  if (view == SA_VIEW_SUMMARY) {
+    // the last c offsets of every block, the last (partial) block included
+    const int tail = L->N - L->R * L->l;
+    return L->R * L->c + std::max(0, tail - (L->l - L->c));
+  }
   return L->N;
 }
 
@@ -214,9 +259,32 @@ void build_kernel_tables(sa_layout* L) {
   } else {
     finish_table(L->fwd_main, {});
   }
+  // The column view's kernel passes cover the whole rows of the 2-D view
+  // (Ng = R l positions in column-major order); the positions of a partial
+  // last row, if any, get their column part from the tail kernels.  With
+  // whole rows only this is the public column table itself.
+  const long long Ng = static_cast<long long>(L->R) * L->l;
+  Csr colg, colgT;
+  int bg = b;
+  if (L->has[SA_VIEW_COLUMN]) {
+    if (Ng == N) {
+      colg = L->view[SA_VIEW_COLUMN];
+      colgT = L->viewT[SA_VIEW_COLUMN];
+    } else {
+      sa_layout G;
+      G.pattern = L->pattern;
+      G.N = static_cast<int>(Ng);
+      G.l = L->l;
+      G.c = L->c;
+      G.R = L->R;
+      G.block = bg = kBwdTQ;  // a granularity of every kernel tile
+      colg = build_public(&G, SA_VIEW_COLUMN);
+      colgT = transpose(colg);
+    }
+  }
   // Forward, column-order query tiles (strided).
   if (L->has[SA_VIEW_COLUMN]) {
-    auto col = coarsen(L->view[SA_VIEW_COLUMN], b, kFwdTQ, kFwdTK, N, N);
+    auto col = coarsen(colg, bg, kFwdTQ, kFwdTK, Ng, Ng);
     std::vector<std::vector<int32_t>> rows(col.size());
     for (size_t r = 0; r < col.size(); ++r)
       for (auto& e : col[r].ent) rows[r].push_back(pack_entry(e.first, SRC_T, e.second));
@@ -238,7 +306,8 @@ void build_kernel_tables(sa_layout* L) {
   if (L->has[SA_VIEW_COLUMN] || L->has[SA_VIEW_SUMMARY]) {
     const int v = L->has[SA_VIEW_COLUMN] ? SA_VIEW_COLUMN : SA_VIEW_SUMMARY;
     const int src = (v == SA_VIEW_COLUMN) ? SRC_T : SRC_S;
-    auto kt = coarsen(L->viewT[v], b, kBwdTK, kBwdTQ, view_keys(L, v), N);
+    auto kt = (v == SA_VIEW_COLUMN) ? coarsen(colgT, bg, kBwdTK, kBwdTQ, Ng, Ng)
+                                    : coarsen(L->viewT[v], b, kBwdTK, kBwdTQ, view_keys(L, v), N);
     std::vector<std::vector<int32_t>> rows(kt.size());
     for (size_t r = 0; r < kt.size(); ++r)
       for (auto& e : kt[r].ent) rows[r].push_back(pack_entry(e.first, src, e.second));
@@ -246,6 +315,8 @@ void build_kernel_tables(sa_layout* L) {
   } else {
     finish_table(L->bwd_sec, {});
   }
+  widen(L->bwd_main, L->bwd_main_w);
+  widen(L->bwd_sec, L->bwd_sec_w);
 }
 
 }  // namespace

@@ -38,11 +38,14 @@ class SparseAttnError(RuntimeError):
         super().__init__(f"{what}: {strerror(status)} (status {status})")
 
 
-def _load():
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+def load_library(path=None):
+    """ctypes handle of the library at ``path`` (default: the product build)
+    with the argument types of every entry point set."""
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m factorized_block_sparse_b200.build` (no CPU fallback exists)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     P, I, F, VP = ctypes.POINTER, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
     lib.sparse_attn_layout.argtypes = [I, I, I, I, I, P(VP)]
     lib.sparse_attn_layout.restype = I
@@ -86,7 +89,7 @@ def _load():
     return lib
 
 
-lib = _load()
+lib = load_library()
 
 
 def strerror(status):

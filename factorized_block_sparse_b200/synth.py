@@ -34,6 +34,9 @@ WORKLOADS = {
     # the image64 strided pattern in its two-head form: row head and column head
     "image64-local": dict(mode="local", B=1, H=16, N=12288, D=64, l=192, c=0, block=64),
     "image64-column": dict(mode="column", B=1, H=16, N=12288, D=64, l=192, c=0, block=64),
+    # longer sequences, the strided pattern with l = sqrt(N): 2^18 and 2^20 positions
+    "long-strided-262144": dict(mode="strided", B=1, H=4, N=1 << 18, D=64, l=512, c=0, block=64),
+    "long-strided-1048576": dict(mode="strided", B=1, H=4, N=1 << 20, D=64, l=1024, c=0, block=64),
 }
 
 

@@ -61,7 +61,10 @@ def test_argument_errors(sa):
     assert L(3, 64, 8, 9, 16, ctypes.byref(h)) == sa.SA_ERR_INVALID_ARG   # c <= l
     assert L(0, 64, 1, 0, 0, ctypes.byref(h)) == sa.SA_ERR_INVALID_ARG
     assert L(0, 60, 1, 0, 16, ctypes.byref(h)) == sa.SA_ERR_UNSUPPORTED   # N % block
-    assert L(2, 64, 12, 0, 16, ctypes.byref(h)) == sa.SA_ERR_UNSUPPORTED  # N % l
+    assert L(4, 64, 12, 0, 16, ctypes.byref(h)) == sa.SA_ERR_UNSUPPORTED  # column head: N % l
+    for pat in (2, 3):                                                    # strided, fixed: any N % l
+        assert L(pat, 64, 12, 4, 16, ctypes.byref(h)) == sa.SA_OK
+        sa.lib.sparse_attn_layout_free(h)
     assert L(4, 64, 12, 0, 16, ctypes.byref(h)) == sa.SA_ERR_UNSUPPORTED  # column: N % l
     assert L(6, 64, 8, 0, 16, ctypes.byref(h)) == sa.SA_ERR_INVALID_ARG   # no pattern 6
     assert L(5, 64, 12, 0, 16, ctypes.byref(h)) == sa.SA_OK               # block: any l
@@ -87,8 +90,16 @@ def test_argument_errors(sa):
             == sa.SA_ERR_INVALID_ARG
         assert sa.lib.sparse_attn_bwd_ex(*([fake] * 9), 1, 1, 256, 32, bad, lay.handle, fake, 1 << 20, None) \
             == sa.SA_ERR_INVALID_ARG
+    # D = 32 rows are 64 bytes: runs of an odd number of rows cannot be moved
+    # by TMA (128-byte shared-memory boundaries), so odd R or odd c > 1 is refused
+    for mode, N, l, c in (("strided", 1344, 64, 0), ("column", 320, 64, 0), ("fixed", 1024, 128, 5)):
+        odd = sa.Layout(mode, N, l, c, 64)
+        assert sa.lib.sparse_attn_fwd(fake, fake, fake, fake, fake, 1, 1, N, 32, odd.handle, None) \
+            == sa.SA_ERR_UNSUPPORTED, mode
+        assert sa.lib.sparse_attn_bwd(*([fake] * 9), 1, 1, N, 32, odd.handle, fake, 1 << 30, None) \
+            == sa.SA_ERR_UNSUPPORTED, mode
     assert sa.strerror(sa.SA_ERR_TIMEOUT) == "device-side wait timed out"
-    assert sa.lib.sparse_attn_kernel_kinds() == 42  # 6 kernels x 7 patterns
+    assert sa.lib.sparse_attn_kernel_kinds() == 56  # 8 kernels x 7 patterns
 
 
 def _compare(sa, mode, N, l, c, b, rows=None):
@@ -143,6 +154,10 @@ def test_layout_bit_exact_audio_sampled_rows(sa):
     ("strided", 64, 8, 0, 3 * 0 + 4), ("strided", 96, 6, 0, 48),
     ("fixed", 128, 16, 16, 16), ("fixed", 128, 16, 1, 8), ("fixed", 144, 12, 5, 16),
     ("fixed", 96, 24, 3, 48), ("fixed", 64, 64, 8, 16),
+    # N not a multiple of l: a partial last block, with and without summary offsets of its own
+    ("fixed", 136, 16, 4, 8), ("fixed", 140, 16, 6, 4), ("fixed", 1136, 128, 32, 16), ("fixed", 100, 24, 24, 4),
+    ("strided", 100, 12, 0, 4), ("strided", 130, 16, 0, 2), ("strided", 1000, 64, 0, 8), ("strided", 40, 64, 0, 8),
+    ("strided", 1216, 96, 0, 64),
     ("column", 128, 16, 0, 16), ("column", 144, 12, 0, 8), ("column", 128, 1, 0, 16),
     ("column", 128, 128, 0, 16), ("column", 96, 6, 0, 48),
     ("block", 128, 16, 0, 16), ("block", 120, 7, 0, 8), ("block", 64, 64, 0, 16), ("block", 96, 1, 0, 8),

@@ -47,6 +47,25 @@ SMALL = [
     # 64-query steps each, so its backward takes the LONG shape element by element
     ("strided", 1, 1, 3072, 64, 192, 0, 64),
     ("strided", 1, 2, 6144, 64, 192, 0, 64),    # R = 32, image64's row length
+    # column and summary geometries that need TMA boxes of gcd(R, rows) or
+    # gcd(c, rows) rows: R neither dividing nor divisible by 128, R odd, c
+    # neither dividing 64 nor a multiple of 128
+    ("strided", 1, 1, 1536, 64, 64, 0, 64),     # R = 24
+    ("strided", 1, 2, 1280, 64, 256, 0, 64),    # R = 5
+    ("column", 1, 1, 768, 64, 64, 0, 64),       # R = 12
+    ("column", 1, 1, 1344, 64, 64, 0, 64),      # R = 21
+    ("fixed", 1, 1, 2048, 64, 128, 48, 64),     # c = 48
+    ("fixed", 1, 1, 1536, 32, 96, 24, 32),      # c = 24, D = 32
+    ("fixed", 1, 2, 1024, 128, 128, 96, 64),    # c = 96, D = 128
+    # N not a multiple of l (a partial last block)
+    ("fixed", 1, 2, 1136, 64, 128, 32, 16),     # the partial block holds summary offsets of its own
+    ("fixed", 2, 1, 1088, 32, 128, 16, 64),     # ... and here it does not
+    ("fixed", 1, 1, 3000, 64, 128, 32, 8),      # summary view long enough for the LONG shape
+    ("strided", 1, 2, 1000, 64, 64, 0, 8),      # R = 15 whole rows + a partial row of 40
+    ("strided", 2, 1, 1216, 32, 96, 0, 64),     # R = 12 + 64, D = 32
+    ("strided", 1, 1, 1152 + 80, 128, 96, 0, 16),  # R = 12 + 80, D = 128
+    ("strided", 1, 1, 200, 64, 256, 0, 8),      # N < l: no whole row, no column part
+    ("strided", 1, 1, 3000, 64, 192, 0, 8),     # R = 15 + 120, the natural view in the LONG shape
 ]
 
 
