@@ -21,7 +21,7 @@ TEST_LIB = os.path.join(HERE, "libsparse_attn_test.so")
 SOURCES = [os.path.join(HERE, "csrc", "sa_api.cu"), os.path.join(HERE, "csrc", "sa_layout.cpp")]
 HEADERS = [os.path.join(ROOT, "include", "sparse_attn.h")] + [
     os.path.join(HERE, "csrc", f) for f in ("sa_internal.h", "sa_device.cuh", "sa_fwd.cuh", "sa_bwd.cuh",
-                                            "sa_bwd_wide.cuh", "sa_tail.cuh")]
+                                            "sa_tail.cuh")]
 
 
 def nvcc_path():

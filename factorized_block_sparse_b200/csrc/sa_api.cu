@@ -18,7 +18,6 @@
 #include <vector>
 
 #include "sa_bwd.cuh"
-#include "sa_bwd_wide.cuh"
 #include "sa_device.cuh"
 #include "sa_fwd.cuh"
 #include "sa_internal.h"
@@ -166,7 +165,7 @@ __global__ void sa_check_table_kernel(DevTable t, int max_tile) {
 }
 
 int check_tables(const DeviceCopy& dc, int N, cudaStream_t s) {
-  const DevTable* ts[6] = {&dc.fwd_main, &dc.fwd_col, &dc.bwd_main, &dc.bwd_sec, &dc.bwd_main_w, &dc.bwd_sec_w};
+  const DevTable* ts[4] = {&dc.fwd_main, &dc.fwd_col, &dc.bwd_main, &dc.bwd_sec};
   for (const DevTable* t : ts) {
     if (t->n_rows == 0) continue;
     sa_check_table_kernel<<<8, 256, 0, s>>>(*t, N / 64 + 2);
@@ -351,8 +350,8 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
       *out = d;
       return SA_OK;
     }
-  constexpr int NT = 6;
-  const TileTable* tabs[NT] = {&L->fwd_main, &L->fwd_col, &L->bwd_main, &L->bwd_sec, &L->bwd_main_w, &L->bwd_sec_w};
+  constexpr int NT = 4;
+  const TileTable* tabs[NT] = {&L->fwd_main, &L->fwd_col, &L->bwd_main, &L->bwd_sec};
   std::vector<int32_t> blob;
   size_t offs[NT][4];
   for (int t = 0; t < NT; ++t) {
@@ -379,7 +378,7 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
   DeviceCopy d;
   d.device = dev;
   d.blob = dptr;
-  DevTable* dts[NT] = {&d.fwd_main, &d.fwd_col, &d.bwd_main, &d.bwd_sec, &d.bwd_main_w, &d.bwd_sec_w};
+  DevTable* dts[NT] = {&d.fwd_main, &d.fwd_col, &d.bwd_main, &d.bwd_sec};
   const int32_t* base = static_cast<const int32_t*>(dptr);
   for (int t = 0; t < NT; ++t) {
     dts[t]->row_ptr = base + offs[t][0];
@@ -475,6 +474,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.R = g.R;
   a.pattern = kernel_pattern(L->pattern);
   a.t_open = (L->pattern == SA_COLUMN) ? 0 : 1;
+  a.box = make_boxes(g.R, g.c);
   a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   // Column view first (SA_STRIDED, SA_COLUMN); the natural view then merges
   // into its result (SA_STRIDED) or runs alone (the other patterns).
@@ -541,7 +541,7 @@ WsLayout ws_layout(int B, int H, int N, int D, const sa_layout* L) {
   const size_t BH = static_cast<size_t>(B) * H;
   const size_t rows = BH * N;
   WsLayout w;
-  w.n_pad = (N + kBwdWideTQ - 1) / kBwdWideTQ * kBwdWideTQ;  // whole steps of either kernel shape
+  w.n_pad = (N + BwdCfg<64>::TQ - 1) / BwdCfg<64>::TQ * BwdCfg<64>::TQ;
   const size_t ld_bytes = align256(BH * w.n_pad * 8);  // two floats per query position
   w.ld_nat = 0;
   w.ld_col = ld_bytes;
@@ -582,14 +582,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     if ((st = set_smem(sa_bwd_kernel<D, true, false>, BwdCfg<D, true>::SMEM))) return st;
     if ((st = set_smem(sa_bwd_kernel<D, true, true>, BwdCfg<D, true>::SMEM))) return st;
   }
-  // Q / dO maps with 128-row boxes for the wide-step shape (D = 64)
-  MapSet mq_w, mdo_w;
-  if constexpr (D == 64) {
-    if ((st = set_smem(sa_bwd_wide_kernel<false>, WideCfg::SMEM))) return st;
-    if ((st = set_smem(sa_bwd_wide_kernel<true>, WideCfg::SMEM))) return st;
-    if ((st = make_maps(&mq_w, q, g, L->pattern, WideCfg::TQ))) return st;
-    if ((st = make_maps(&mdo_w, dO, g, L->pattern, WideCfg::TQ))) return st;
-  }
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* ld_nat = reinterpret_cast<float*>(wsb + w.ld_nat);
@@ -625,14 +617,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.pattern = kernel_pattern(L->pattern);
   a.scale = scale;
   a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
+  a.box = make_boxes(g.R, g.c);
   const bool sec = dc.bwd_sec.n_rows > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN
   // SA_COLUMN has no natural view: its column-view pass writes the final dK/dV.
   const bool sec_final = L->pattern == SA_COLUMN;
   a.BH = g.BH;
   const int n_sm = sm_count();
-  // Tables whose items average many steps take the LONG shape of the kernel;
-  // for D = 64 that is the wide-step kernel on the 128-query-step table.
-  auto run = [&](int kind, const DevTable& t, const DevTable& tw) -> int {
+  // Tables whose items average many steps take the LONG shape of the kernel.
+  auto run = [&](int kind, const DevTable& t) -> int {
     EpiMaps em;
     const int mst = make_epi_maps(&em, dk, dv, dk_part, dv_part, g, a.key_view);
     if (mst) return mst;
@@ -644,20 +636,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
       launch_kernel(kernel, grid, threads, smem, s, mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                     mv.col, mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v, em.part_k, em.part_v, a);
     };
-    if constexpr (D == 64) {
-      if (long_items) {
-        BwdArgs aw = a;
-        aw.sched = tw.sched;
-        aw.ent = tw.ent;
-        aw.n_slots = tw.n_rows;
-        return launch(kind, s, [&] {
-          auto kernel = final_t ? sa_bwd_wide_kernel<true> : sa_bwd_wide_kernel<false>;
-          launch_kernel(kernel, grid, WideCfg::THREADS, WideCfg::SMEM, s, mq_w.nat, mq_w.col, mdo_w.nat, mdo_w.col,
-                        mk.nat, mk.col, mk.sum, mv.nat, mv.col, mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v,
-                        em.part_k, em.part_v, aw);
-        });
-      }
-    }
     return launch(kind, s, [&] {
       if constexpr (D <= 64) {
         if (long_items) {
@@ -678,7 +656,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_sec.n_rows;
     a.key_view = (L->pattern == SA_FIXED) ? SRC_S : SRC_T;
     a.add_part = 0;
-    if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec, dc.bwd_sec_w))) return st;
+    if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec))) return st;
   }
   const int r_tail = (L->pattern == SA_STRIDED && L->R > 0) ? N - L->R * L->l : 0;
   if (r_tail > 0) {  // the partial last row's column part (after the column view's pass)
@@ -698,7 +676,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_main.n_rows;
     a.key_view = SRC_N;
     a.add_part = (sec && !sec_final) ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
-    if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main, dc.bwd_main_w))) return st;
+    if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main))) return st;
   }
   const long long n8 = rows * D / 8;
   return launch(K_BWD_FINAL * K_PATTERNS + L->pattern, s, [&] {

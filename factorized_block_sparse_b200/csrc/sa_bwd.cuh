@@ -61,6 +61,7 @@ struct BwdArgs {
   int add_part;  // main pass: add secondary partials (1 strided: all keys; 2 fixed: summary keys)
   float scale;       // 1/sqrt(D)
   float scale_log2;  // log2(e)/sqrt(D)
+  BoxSet box;        // column / summary TMA boxes per tile height
 };
 
 // Two shapes of the same kernel.  LONG is for tables whose items run many
@@ -109,7 +110,7 @@ struct BwdCfg {
   // 4 x DQS_WARP_BYTES; 1 KiB aligned (the 128-byte swizzle pattern is address based)
   static constexpr int OFF_DQS = (OFF_LD + STAGES * LD_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = OFF_DQS + 4 * DQS_WARP_BYTES;
-  static constexpr int N_BARS = 2 * KVB + 2 * STAGES + 2 * 7 + DST_BUFS + 2 * DQBUF + 2 * DKVB + 4;
+  static constexpr int N_BARS = 2 * KVB + 2 * STAGES + 2 * 7 + DST_BUFS + 2 * DQBUF + 2 * DKVB + 4 + 2;
   static constexpr int OFF_MISC = OFF_BAR + 8 * N_BARS;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
@@ -279,6 +280,7 @@ __global__ void __launch_bounds__(480, 1)
   uint64_t* bar_dkv_full = bar_dq_free + C::DQBUF;       // [DKVB] per non-empty item
   uint64_t* bar_dkv_free = bar_dkv_full + C::DKVB;       // [DKVB]
   uint64_t* bar_epi = bar_dkv_free + C::DKVB;            // [4] partial rows landed (epilogue warp)
+  uint64_t* bar_drain = bar_epi + 4;                     // [2] each issuer's last commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
 
@@ -316,6 +318,8 @@ __global__ void __launch_bounds__(480, 1)
       mbar_init(bar_dkv_free + b, 128);
     }
     for (int w = 0; w < 4; ++w) mbar_init(bar_epi + w, 1);
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_drain + 1, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(480, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
-      int gs = 0, ne = 0;
+      int gs = 0, ne = 0, issued = 0, kv_issued = 0;
       BwdItem nxt = (cta < n_items) ? bwd_item(a, cta) : BwdItem{0, 0, 0, 0};
       for (int k = 0, item = cta; ok && item < n_items;) {
         const BwdItem it = nxt;
@@ -340,11 +344,12 @@ __global__ void __launch_bounds__(480, 1)
         if (it.n == 0) continue;
         const int kb = ne % C::KVB;
         if (ne >= C::KVB && !mbar_wait(bar_kv_empty + kb, ((ne / C::KVB) - 1) & 1, abort_flag)) break;
+        ++kv_issued;
         mbar_arrive_expect_tx(bar_kv_full + kb, 2 * C::KV_BYTES);
         load_rows<D>(sK + kb * C::KV_BYTES, a.key_view, it.kt * C::TK, C::TK, it.bh, &mk_nat, &mk_col, &mk_sum,
-                     bar_kv_full + kb, a.R, a.l, a.c);
+                     bar_kv_full + kb, a.R, a.l, a.c, a.box.b[box_index(C::TK)]);
         load_rows<D>(sV + kb * C::KV_BYTES, a.key_view, it.kt * C::TK, C::TK, it.bh, &mv_nat, &mv_col, &mv_sum,
-                     bar_kv_full + kb, a.R, a.l, a.c);
+                     bar_kv_full + kb, a.R, a.l, a.c, a.box.b[box_index(C::TK)]);
         const float* ld = (q_src == SRC_T ? a.ld_col : a.ld_nat) + static_cast<size_t>(it.bh) * a.n_pad * 2;
         int e_next = a.ent[it.e0];
         for (int j = 0; j < it.n; ++j) {
@@ -356,16 +361,28 @@ __global__ void __launch_bounds__(480, 1)
             ok = false;
             break;
           }
+          ++issued;
+#ifdef SA_TEST_HOOKS
+          if (g == 0 && *(volatile int*)&g_test_withhold) continue;  // the first step's tiles never arrive
+#endif
           const int qpos = (e >> 3) * C::TQ;
           mbar_arrive_expect_tx(bar_qdo_full + st, 2 * C::QS_BYTES + C::LD_BYTES);
           load_rows<D>(sQ + st * C::QS_BYTES, q_src, qpos, C::TQ, it.bh, &mq_nat, &mq_col, &mq_col,
-                       bar_qdo_full + st, a.R, a.l, a.c);
+                       bar_qdo_full + st, a.R, a.l, a.c, a.box.b[box_index(C::TQ)]);
           load_rows<D>(sDO + st * C::QS_BYTES, q_src, qpos, C::TQ, it.bh, &mdo_nat, &mdo_col, &mdo_col,
-                       bar_qdo_full + st, a.R, a.l, a.c);
+                       bar_qdo_full + st, a.R, a.l, a.c, a.box.b[box_index(C::TQ)]);
           bulk_load(sLD + st * 2 * C::TQ, ld + 2 * qpos, C::LD_BYTES, bar_qdo_full + st);
         }
         gs += it.n;
         ++ne;
+      }
+      // After an abort, wait (bounded) for the loads still in flight, so that
+      // no copy lands in shared memory after the CTA has exited.
+      if (*(volatile int*)abort_flag) {
+        for (int h = kv_issued > C::KVB ? kv_issued - C::KVB : 0; h < kv_issued; ++h)
+          mbar_wait_drain(bar_kv_full + h % C::KVB, (h / C::KVB) & 1);
+        for (int h = issued > C::STAGES ? issued - C::STAGES : 0; h < issued; ++h)
+          mbar_wait_drain(bar_qdo_full + h % C::STAGES, (h / C::STAGES) & 1);
       }
     }
   } else if (warp == 1) {
@@ -418,6 +435,9 @@ __global__ void __launch_bounds__(480, 1)
         gs += it.n;
         ++ne;
       }
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0);
     }
   } else if (warp == 14) {
     // ------------------------------------------------------------ G issuer: dV, dK, dQ
@@ -496,6 +516,9 @@ __global__ void __launch_bounds__(480, 1)
         gs += it.n;
         ++ne;
       }
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(bar_drain + 1);
+      mbar_wait_drain(bar_drain + 1, 0);
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------ elementwise
@@ -689,7 +712,7 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
               for (int bx = 0; bx < D / 32; ++bx) {
                 if (q_src == SRC_T) {
-                  const int rb = gcd_int(a.R, 32);
+                  const int rb = a.box.b[0].rb_t;
                   for (int s0 = 0; s0 < 32; s0 += rb) {
                     const int t = xw + s0;
                     tma_reduce_add_4d(&mdq_col, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
@@ -807,7 +830,7 @@ __global__ void __launch_bounds__(480, 1)
           __syncwarp();
           if (lane == 0) {
             if constexpr (FINAL_T) {  // rows of the column runs
-              const int rb = gcd_int(a.R, 32);
+              const int rb = a.box.b[0].rb_t;
               for (int s0 = 0; s0 < 32; s0 += rb) {
                 const int t = y0 + s0;
                 tma_store_4d(which ? &mdk_out : &mdv_out, stg + s0 * (D * 2), 0, t / a.R, t % a.R, it.bh);
@@ -819,15 +842,14 @@ __global__ void __launch_bounds__(480, 1)
 #pragma unroll
               for (int bx = 0; bx < D / 32; ++bx) {
                 if (a.key_view == SRC_T) {
-                  const int rb = gcd_int(a.R, 32);
+                  const int rb = a.box.b[0].rb_t;
                   for (int s0 = 0; s0 < 32; s0 += rb) {
                     const int t = y0 + s0;
                     tma_store_4d(mp, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
                   }
                 } else {
-                  int cb, gb;
-                  summary_box(a.c, 32, &cb, &gb);
-                  if (gb > 1 || cb == a.c) {  // whole blocks
+                  const int cb = a.box.b[0].cb_s;
+                  if (a.box.b[0].gb_s > 1 || cb == a.c) {  // whole blocks
                     tma_store_4d(mp, stg + bx * 4096, bx * 32, a.l - a.c, y0 / a.c, it.bh);
                   } else {  // runs of cb keys inside one block
                     for (int s0 = 0; s0 < 32; s0 += cb) {

@@ -56,6 +56,27 @@ __host__ __device__ __forceinline__ void summary_box(int c, int rows, int* cb, i
   }
 }
 
+// TMA box geometry of the column and summary views for tiles of 32, 64 and
+// 128 rows (index 0, 1, 2), computed on the host: rb_t rows per box of the
+// column view; the summary view moves whole blocks when cb_s == c (gb_s
+// blocks per box), else runs of cb_s keys inside one block.
+struct BoxGeo {
+  int rb_t, cb_s, gb_s;
+};
+struct BoxSet {
+  BoxGeo b[3];
+};
+__host__ __device__ constexpr int box_index(int rows) { return rows == 32 ? 0 : (rows == 64 ? 1 : 2); }
+inline BoxSet make_boxes(int R, int c) {
+  BoxSet s;
+  for (int i = 0; i < 3; ++i) {
+    const int rows = 32 << i;
+    s.b[i].rb_t = gcd_int(R, rows);
+    summary_box(c, rows, &s.b[i].cb_s, &s.b[i].gb_s);
+  }
+  return s;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -147,6 +168,16 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // Lets the next kernel in the stream begin launching; its CTAs start once
 // every CTA of this grid has called this or exited.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Bounded wait used only to drain in-flight asynchronous work (loads, MMAs)
+// after an abort: it ignores the abort flag and gives up after about 2^26
+// cycles.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > (1LL << 26)) return;
+  }
+}
 
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -43,6 +43,7 @@ struct FwdArgs {
   int merge;    // 1: combine with the partial (o, lse) already stored
   int t_open;   // column view: 1 when it excludes the diagonal (SA_STRIDED), 0 when it stands alone
   float scale_log2;
+  BoxSet box;  // column / summary TMA boxes per tile height
 };
 
 template <int D>
@@ -82,7 +83,7 @@ template <int D>
 __device__ __forceinline__ void load_rows(uint8_t* dst, int src, int pos0, int rows, int bh,
                                           const CUtensorMap* m_nat, const CUtensorMap* m_col,
                                           const CUtensorMap* m_sum, uint64_t* bar, int R, int l,
-                                          int c) {
+                                          int c, const BoxGeo& bg) {
   using C = FwdCfg<D>;
   const int panel_bytes = rows * C::ROWB;
 #pragma unroll
@@ -92,15 +93,14 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, int src, int pos0, int r
     if (src == SRC_N) {
       tma_load_3d(d, m_nat, bar, x, pos0, bh);
     } else if (src == SRC_T) {
-      const int rb = gcd_int(R, rows);
+      const int rb = bg.rb_t;
       for (int s = 0; s < rows; s += rb) {
         const int t = pos0 + s;
         tma_load_4d(d + s * C::ROWB, m_col, bar, x, t / R, t % R, bh);
       }
     } else {
-      int cb, gb;
-      summary_box(c, rows, &cb, &gb);
-      if (gb > 1 || cb == c) {  // whole blocks
+      const int cb = bg.cb_s;
+      if (bg.gb_s > 1 || cb == c) {  // whole blocks
         tma_load_4d(d, m_sum, bar, x, l - c, pos0 / c, bh);
       } else {  // runs of cb keys inside one block
         for (int s = 0; s < rows; s += cb) {
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
       const CUtensorMap* mq = a.q_col ? &mq_col : &mq_nat;
       mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
       load_rows<D>(sQ, a.q_col ? SRC_T : SRC_N, qt * C::TQ, C::TQ, bh, mq, mq, mq, bar_q, a.R,
-                   a.l, a.c);
+                   a.l, a.c, a.box.b[box_index(C::TQ)]);
       for (int j = 0; j < n; ++j) {
         const int st = j % C::STAGES;
         if (j >= C::STAGES && !mbar_wait(bar_kv_empty + st, ((j / C::STAGES) - 1) & 1, abort_flag))
@@ -213,10 +213,10 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
         const int kpos = (e >> 3) * C::TK;
         mbar_arrive_expect_tx(bar_k_full + st, C::KV_BYTES);
         load_rows<D>(sK + st * C::KV_BYTES, src, kpos, C::TK, bh, &mk_nat, &mk_col, &mk_sum,
-                     bar_k_full + st, a.R, a.l, a.c);
+                     bar_k_full + st, a.R, a.l, a.c, a.box.b[box_index(C::TK)]);
         mbar_arrive_expect_tx(bar_v_full + st, C::KV_BYTES);
         load_rows<D>(sV + st * C::KV_BYTES, src, kpos, C::TK, bh, &mv_nat, &mv_col, &mv_sum,
-                     bar_v_full + st, a.R, a.l, a.c);
+                     bar_v_full + st, a.R, a.l, a.c, a.box.b[box_index(C::TK)]);
       }
     }
   } else if (warp == 1) {
@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
 #pragma unroll
       for (int p = 0; p < C::PANELS; ++p) {
         if (a.q_col) {
-          const int rb = gcd_int(a.R, 32);
+          const int rb = a.box.b[0].rb_t;
           for (int s0 = 0; s0 < 32; s0 += rb) {
             const int t = xw + s0;
             tma_store_4d(&mo_col, stg + p * PB + s0 * C::ROWB, p * 64, t / a.R, t % a.R, bh);

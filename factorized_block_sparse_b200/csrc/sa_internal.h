@@ -21,9 +21,6 @@ constexpr int kBwdTQ = 64;   // backward: queries per step
 // Backward tables whose items average at least this many steps run the
 // kernel shape with the deeper Q/dO ring (P^T in TMEM).
 constexpr int kBwdLongSteps = 4;
-// The wide-step shape of the long-item backward (D = 64) walks 128-query
-// steps: its tables pair the 64-query tiles of the backward tables.
-constexpr int kBwdWideTQ = 128;
 
 enum Src : int { SRC_N = 0, SRC_T = 1, SRC_S = 2 };
 
@@ -58,7 +55,7 @@ struct DevTable {
 struct DeviceCopy {
   int device = -1;
   void* blob = nullptr;
-  DevTable fwd_main, fwd_col, bwd_main, bwd_sec, bwd_main_w, bwd_sec_w;
+  DevTable fwd_main, fwd_col, bwd_main, bwd_sec;
 };
 
 }  // namespace sa
@@ -73,7 +70,6 @@ struct sa_layout {
   sa::TileTable fwd_col;   // column-order query tiles: T-view keys (strided)
   sa::TileTable bwd_main;  // natural key tiles: N-view query tiles
   sa::TileTable bwd_sec;   // T-order (strided) or summary-order (fixed) key tiles
-  sa::TileTable bwd_main_w, bwd_sec_w;  // the same key tiles with 128-query steps
   mutable std::mutex mu;
   mutable std::vector<sa::DeviceCopy> dev;
 };

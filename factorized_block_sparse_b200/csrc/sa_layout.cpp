@@ -196,35 +196,6 @@ void finish_table(TileTable& tt, const std::vector<std::vector<int32_t>>& rows) 
   }
 }
 
-// The same key tiles with 128-query steps: query tile t of a 64-query table
-// becomes step t / 2.  A step is FULL only when both of its 64-query halves
-// are listed and FULL; a half that is missing (outside the key tile's
-// queries, or past the end of the view) is masked like any PARTIAL part.
-void widen(const TileTable& t64, TileTable& out) {
-  std::vector<std::vector<int32_t>> rows(t64.n_rows);
-  for (int r = 0; r < t64.n_rows; ++r) {
-    int cur = -1, src = 0, halves = 0, part = 0;
-    auto flush = [&] {
-      if (cur >= 0) rows[r].push_back(pack_entry(cur, src, (part || halves != 2) ? 1 : 0));
-    };
-    for (int e = t64.row_ptr[r]; e < t64.row_ptr[r + 1]; ++e) {
-      const int32_t v = t64.ent[e];
-      const int w = (v >> 3) / 2;
-      if (w != cur) {
-        flush();
-        cur = w;
-        src = (v >> 1) & 3;
-        halves = 0;
-        part = 0;
-      }
-      ++halves;
-      part |= v & 1;
-    }
-    flush();
-  }
-  finish_table(out, rows);
-}
-
 }  // namespace
 
 int view_keys(const sa_layout* L, int view) {
@@ -315,8 +286,6 @@ void build_kernel_tables(sa_layout* L) {
   } else {
     finish_table(L->bwd_sec, {});
   }
-  widen(L->bwd_main, L->bwd_main_w);
-  widen(L->bwd_sec, L->bwd_sec_w);
 }
 
 }  // namespace
