@@ -243,7 +243,7 @@ int make_dq_maps(CUtensorMap* nat, CUtensorMap* col, const float* base, const Ge
                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return SA_ERR_CUDA;
   }
-  if (pattern == SA_STRIDED || pattern == SA_COLUMN) {
+  if ((pattern == SA_STRIDED || pattern == SA_COLUMN) && g.R > 0) {  // R = 0: no whole row, no column view
     const cuuint64_t dims[4] = {(cuuint64_t)g.D, (cuuint64_t)g.l, (cuuint64_t)g.R, (cuuint64_t)g.BH};
     const cuuint64_t strides[3] = {(cuuint64_t)g.D * 4, (cuuint64_t)g.l * g.D * 4, (cuuint64_t)g.N * g.D * 4};
     const cuuint32_t box[4] = {32, 1, (cuuint32_t)gcd_int(g.R, 32), 1};
@@ -327,11 +327,11 @@ int make_maps(MapSet* ms, const void* base, const Geo& g, int pattern, int rows)
   std::memset(ms, 0, sizeof(*ms));
   int st = map_nat(&ms->nat, base, g, rows);
   if (st) return st;
-  if (pattern == SA_STRIDED || pattern == SA_COLUMN) {
+  if ((pattern == SA_STRIDED || pattern == SA_COLUMN) && g.R > 0) {  // R = 0: no whole row, no column view
     st = map_grid(&ms->col, base, g, 1, (uint32_t)gcd_int(g.R, rows));
     if (st) return st;
   }
-  if (pattern == SA_FIXED) {
+  if (pattern == SA_FIXED && g.R > 0) {  // R = 0: no whole block, no summary view
     int cb = 1, gb = 1;
     summary_box(g.c, rows, &cb, &gb);
     st = map_grid(&ms->sum, base, g, (uint32_t)cb, (uint32_t)gb);
@@ -455,7 +455,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   CUtensorMap mo_nat, mo_col;
   std::memset(&mo_col, 0, sizeof(mo_col));
   if ((st = map_nat(&mo_nat, o, g, 32))) return st;
-  if ((L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) &&
+  if ((L->pattern == SA_STRIDED || L->pattern == SA_COLUMN) && g.R > 0 &&
       (st = map_grid(&mo_col, o, g, 1, static_cast<uint32_t>(gcd_int(g.R, 32)))))
     return st;
   DeviceCopy dc;
@@ -618,7 +618,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.scale = scale;
   a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   a.box = make_boxes(g.R, g.c);
-  const bool sec = dc.bwd_sec.n_rows > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN
+  const bool sec = dc.bwd_sec.n_rows > 0 && g.R > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN with a whole row
   // SA_COLUMN has no natural view: its column-view pass writes the final dK/dV.
   const bool sec_final = L->pattern == SA_COLUMN;
   a.BH = g.BH;

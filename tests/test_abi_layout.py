@@ -157,7 +157,7 @@ def test_layout_bit_exact_audio_sampled_rows(sa):
     # N not a multiple of l: a partial last block, with and without summary offsets of its own
     ("fixed", 136, 16, 4, 8), ("fixed", 140, 16, 6, 4), ("fixed", 1136, 128, 32, 16), ("fixed", 100, 24, 24, 4),
     ("strided", 100, 12, 0, 4), ("strided", 130, 16, 0, 2), ("strided", 1000, 64, 0, 8), ("strided", 40, 64, 0, 8),
-    ("strided", 1216, 96, 0, 64),
+    ("strided", 1216, 96, 0, 64), ("fixed", 40, 64, 8, 4), ("fixed", 200, 256, 64, 8),
     ("column", 128, 16, 0, 16), ("column", 144, 12, 0, 8), ("column", 128, 1, 0, 16),
     ("column", 128, 128, 0, 16), ("column", 96, 6, 0, 48),
     ("block", 128, 16, 0, 16), ("block", 120, 7, 0, 8), ("block", 64, 64, 0, 16), ("block", 96, 1, 0, 8),

@@ -65,6 +65,7 @@ SMALL = [
     ("strided", 2, 1, 1216, 32, 96, 0, 64),     # R = 12 + 64, D = 32
     ("strided", 1, 1, 1152 + 80, 128, 96, 0, 16),  # R = 12 + 80, D = 128
     ("strided", 1, 1, 200, 64, 256, 0, 8),      # N < l: no whole row, no column part
+    ("fixed", 1, 1, 200, 64, 256, 64, 8),       # N < l: one partial block, no summary view
     ("strided", 1, 1, 3000, 64, 192, 0, 8),     # R = 15 + 120, the natural view in the LONG shape
 ]
 
