@@ -358,6 +358,7 @@ def config_dict(names, args):
         "seq_len": ws[0]["N"],
         "parallelism": f"replicas x{max(1, args.gpus)} (independent (batch, head) work per GPU, no collective)",
         "l2": "flushed between timed steps (256 MiB write outside the events)",
+        "streams": getattr(args, "streams", 1),
     }
 
 
@@ -373,6 +374,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--configs", type=int, default=1, help="1: also time every other named configuration")
+    ap.add_argument("--streams", type=int, default=2, help="streams the step's independent workloads use")
     args = ap.parse_args()
     names = STEPS[args.workload]
     if args.warmup < 3:
@@ -410,12 +412,32 @@ def main():
                           dk=dk, dv=dv, ws=ws))
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
+    # The step's workloads are independent problems: with --streams 2 the
+    # second one is issued on its own stream (forked from and joined back to
+    # the launching stream inside the step), so their kernels can overlap.
+    streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(min(args.streams, len(state)) - 1)]
 
-    def step():
-        for s in state:
-            sa.sparse_attn_fwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["lay"], sptr)
-            sa.sparse_attn_bwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["dO"], s["dq"], s["dk"], s["dv"],
-                               s["lay"], s["ws"], sptr)
+    def run_one(s, strm):
+        p = strm.cuda_stream
+        sa.sparse_attn_fwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["lay"], p)
+        sa.sparse_attn_bwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["dO"], s["dq"], s["dk"], s["dv"],
+                           s["lay"], s["ws"], p)
+
+    def step(serial=False):
+        if serial or len(streams) == 1:
+            for s in state:
+                run_one(s, stream)
+            return
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        for strm in streams[1:]:
+            strm.wait_event(fork)
+        for i, s in enumerate(state):
+            run_one(s, streams[i % len(streams)])
+        for strm in streams[1:]:
+            join = torch.cuda.Event()
+            join.record(strm)
+            stream.wait_event(join)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
@@ -438,7 +460,7 @@ def main():
         for i in range(args.steps):
             flush.zero_()
             evs[i][0].record(stream)
-            step()
+            step(serial=per_kernel)  # per-launch events: one stream, so each launch's events bracket it alone
             evs[i][1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -507,8 +529,9 @@ def main():
                      "peak_kind": "burst (of measured)" if pk["source"] == "measured" else "fallback"},
         "kernels": kernels,
         "kernel_pass": {"ms_per_step": round(max_over_ranks(kernel_pass_ms, world, dev) / args.steps, 4),
-                        "note": "per-kernel events are taken in a second pass of K steps with every launch "
-                                "bracketed by events; the headline steps run without them"},
+                        "note": "per-kernel events are taken in a second pass of K steps on one stream with "
+                                "every launch bracketed by events; the headline steps run without them, the "
+                                "step's workloads on their own streams"},
         "workloads": workload_lines(state, ktimes, pk),
         "configs": configs,
         "gpu_launches": launches,

@@ -353,7 +353,7 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
   constexpr int NT = 4;
   const TileTable* tabs[NT] = {&L->fwd_main, &L->fwd_col, &L->bwd_main, &L->bwd_sec};
   std::vector<int32_t> blob;
-  size_t offs[NT][4];
+  size_t offs[NT][5];
   for (int t = 0; t < NT; ++t) {
     const TileTable& tt = *tabs[t];
     offs[t][3] = blob.size();  // 16-byte aligned: every section is padded to 4 ints
@@ -366,6 +366,9 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
     while (blob.size() % 4) blob.push_back(0);
     offs[t][2] = blob.size();
     blob.insert(blob.end(), tt.order.begin(), tt.order.end());
+    while (blob.size() % 4) blob.push_back(0);
+    offs[t][4] = blob.size();
+    blob.insert(blob.end(), tt.bits.begin(), tt.bits.end());
     while (blob.size() % 4) blob.push_back(0);
   }
   if (blob.empty()) blob.push_back(0);
@@ -385,6 +388,7 @@ int to_device(const sa_layout* L, DeviceCopy* out) {
     dts[t]->ent = base + offs[t][1];
     dts[t]->order = base + offs[t][2];
     dts[t]->sched = base + offs[t][3];
+    dts[t]->bits = tabs[t]->bits.empty() ? nullptr : reinterpret_cast<const uint32_t*>(base + offs[t][4]);
     dts[t]->n_rows = tabs[t]->n_rows;
     dts[t]->nnz = static_cast<int>(tabs[t]->ent.size());
   }
@@ -463,9 +467,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 #ifdef SA_TEST_HOOKS
   if ((st = check_tables(dc, N, s))) return st;
 #endif
-  auto kern = sa_fwd_kernel<D>;
+  // a caller block mask with blocks below a tile: the variant that applies sub-block bits
+  const bool blk = L->pattern == SA_BLOCKS && L->block < kFwdTQ;
+  auto kern = blk ? sa_fwd_kernel<D, true> : sa_fwd_kernel<D, false>;
   if ((st = set_smem(kern, FwdCfg<D>::SMEM))) return st;
   FwdArgs a;
+  a.bits = blk ? dc.fwd_main.bits : nullptr;
+  a.blk = blk ? L->block : 0;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.N = N;
@@ -578,9 +586,11 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
 #endif
   if ((st = set_smem(sa_bwd_kernel<D, false, false>, BwdCfg<D, false>::SMEM))) return st;
   if ((st = set_smem(sa_bwd_kernel<D, false, true>, BwdCfg<D, false>::SMEM))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, false, false, true>, BwdCfg<D, false>::SMEM))) return st;
   if constexpr (D <= 64) {
     if ((st = set_smem(sa_bwd_kernel<D, true, false>, BwdCfg<D, true>::SMEM))) return st;
     if ((st = set_smem(sa_bwd_kernel<D, true, true>, BwdCfg<D, true>::SMEM))) return st;
+    if ((st = set_smem(sa_bwd_kernel<D, true, false, true>, BwdCfg<D, true>::SMEM))) return st;
   }
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -618,6 +628,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.scale = scale;
   a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   a.box = make_boxes(g.R, g.c);
+  a.bits = nullptr;
+  a.blk = 0;
   const bool sec = dc.bwd_sec.n_rows > 0 && g.R > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN with a whole row
   // SA_COLUMN has no natural view: its column-view pass writes the final dK/dV.
   const bool sec_final = L->pattern == SA_COLUMN;
@@ -632,6 +644,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     dim3 grid(static_cast<unsigned>(std::min<long long>(items, n_sm)));
     const bool long_items = D <= 64 && t.nnz >= kBwdLongSteps * static_cast<long long>(t.n_rows);
     const bool final_t = sec_final && a.key_view == SRC_T;
+    const bool blk = a.blk > 0;  // caller block mask with blocks below a tile (natural view only)
     auto go = [&](auto kernel, int threads, int smem) {
       launch_kernel(kernel, grid, threads, smem, s, mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                     mv.col, mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v, em.part_k, em.part_v, a);
@@ -641,12 +654,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
         if (long_items) {
           using CL = BwdCfg<D, true>;
           if (final_t) go(sa_bwd_kernel<D, true, true>, CL::THREADS, CL::SMEM);
+          else if (blk) go(sa_bwd_kernel<D, true, false, true>, CL::THREADS, CL::SMEM);
           else go(sa_bwd_kernel<D, true, false>, CL::THREADS, CL::SMEM);
           return;
         }
       }
       using CS = BwdCfg<D, false>;
       if (final_t) go(sa_bwd_kernel<D, false, true>, CS::THREADS, CS::SMEM);
+      else if (blk) go(sa_bwd_kernel<D, false, false, true>, CS::THREADS, CS::SMEM);
       else go(sa_bwd_kernel<D, false, false>, CS::THREADS, CS::SMEM);
     });
   };
@@ -671,6 +686,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     if (st) return st;
   }
   if (dc.bwd_main.n_rows > 0) {
+    a.bits = dc.bwd_main.bits;
+    a.blk = (L->pattern == SA_BLOCKS && L->block < kBwdTK) ? L->block : 0;
     a.sched = dc.bwd_main.sched;
     a.ent = dc.bwd_main.ent;
     a.n_slots = dc.bwd_main.n_rows;
@@ -697,7 +714,10 @@ int sparse_attn_layout_blocks(int N, int block, const int32_t* row_ptr, const in
   if (!out) return SA_ERR_INVALID_ARG;
   *out = nullptr;
   if (!row_ptr || !col_idx || N < 1 || block < 1) return SA_ERR_INVALID_ARG;
-  if (block % kFwdTQ != 0 || block % kBwdTK != 0 || N % block != 0) return SA_ERR_UNSUPPORTED;
+  // blocks of a multiple of 128 (every kernel tile inside one block), or of
+  // 16, 32 or 64 positions (tiles carry which of their blocks are listed)
+  const bool whole = block % kFwdTQ == 0 && block % kBwdTK == 0;
+  if (!(whole || block == 16 || block == 32 || block == 64) || N % block != 0) return SA_ERR_UNSUPPORTED;
   sa_layout* L = new (std::nothrow) sa_layout();
   if (!L) return SA_ERR_INVALID_ARG;
   L->pattern = SA_BLOCKS;

@@ -62,6 +62,8 @@ struct BwdArgs {
   float scale;       // 1/sqrt(D)
   float scale_log2;  // log2(e)/sqrt(D)
   BoxSet box;        // column / summary TMA boxes per tile height
+  const uint32_t* bits;  // sub-block bits per entry (caller block masks with blocks below a tile)
+  int blk;               // their block size (16, 32 or 64), else 0
 };
 
 // Two shapes of the same kernel.  LONG is for tables whose items run many
@@ -235,7 +237,9 @@ __device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size
 
 // FINAL_T: the pass writes final bf16 dK/dV in column-major order (the
 // column view of SA_COLUMN, which has no natural view).
-template <int D, bool LONG, bool FINAL_T>
+// BLK: a caller block mask whose blocks are smaller than a tile (the
+// entries' sub-block bits are applied on PARTIAL steps).
+template <int D, bool LONG, bool FINAL_T, bool BLK = false>
 __global__ void __launch_bounds__(480, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mdo_nat, const __grid_constant__ CUtensorMap mdo_col,
@@ -579,7 +583,11 @@ __global__ void __launch_bounds__(480, 1)
           sv[4 * i + 3] = ex2(x23.y);
         }
         if (partial) {
-          if constexpr (C::PT_TMEM) {
+          if constexpr (BLK) {
+            const int nj = C::TQ / a.blk;
+            const uint32_t nib = (a.bits[it.e0 + j] >> ((row / a.blk) * nj)) & ((1u << nj) - 1u);
+            mask_bits64(sv, interval_bits64(kr.qlo - x0, kr.qhi - x0) & sub_block_cols(nib, a.blk), 0.f);
+          } else if constexpr (C::PT_TMEM) {
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
               const int x = x0 + i;

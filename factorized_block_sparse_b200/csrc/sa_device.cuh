@@ -474,6 +474,34 @@ __device__ __forceinline__ void mask_interval64(float* v, int lo, int hi, float 
   for (int i = 0; i < 32; ++i) v[32 + i] = ((m1 >> i) & 1u) ? v[32 + i] : fill;
 }
 
+// Caller block masks with blocks smaller than a tile: the 64-bit mask of the
+// columns whose sub-block is listed.  Bit j of `nib` covers columns
+// [j * blk, (j + 1) * blk) (blk = 16, 32 or 64).
+__device__ __forceinline__ uint64_t sub_block_cols(uint32_t nib, int blk) {
+  const uint64_t one = (blk >= 64) ? ~0ull : ((1ull << blk) - 1ull);
+  uint64_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (j * blk < 64 && ((nib >> j) & 1u)) m |= one << (j * blk);
+  return m;
+}
+
+// The interval [lo, hi] of a 64-column tile as a mask (empty when lo > hi).
+__device__ __forceinline__ uint64_t interval_bits64(int lo, int hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 63);
+  return (lo <= hi) ? ((~0ull << lo) & (~0ull >> (63 - hi))) : 0ull;
+}
+
+// Keeps v[i] where bit i of m is set, sets the others to `fill`.
+__device__ __forceinline__ void mask_bits64(float* v, uint64_t m, float fill) {
+  const uint32_t m0 = static_cast<uint32_t>(m), m1 = static_cast<uint32_t>(m >> 32);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = ((m0 >> i) & 1u) ? v[i] : fill;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[32 + i] = ((m1 >> i) & 1u) ? v[32 + i] : fill;
+}
+
 // Byte offset of 16-byte chunk `chunk` of row `row` in a K-major tile whose
 // rows are 128 bytes (64 bf16) wide, swizzled 128B (8-row atoms of 1 KiB).
 __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk) {

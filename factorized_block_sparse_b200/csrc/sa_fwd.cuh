@@ -44,6 +44,8 @@ struct FwdArgs {
   int t_open;   // column view: 1 when it excludes the diagonal (SA_STRIDED), 0 when it stands alone
   float scale_log2;
   BoxSet box;  // column / summary TMA boxes per tile height
+  const uint32_t* bits;  // sub-block bits per entry (caller block masks with blocks below a tile)
+  int blk;               // their block size (16, 32 or 64), else 0
 };
 
 template <int D>
@@ -131,7 +133,9 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int rows, int kk
   return make_desc(base + kk * 16 * C::ROWB, rows * C::ROWB, C::SBO, C::SWZ);
 }
 
-template <int D>
+// BLK: a caller block mask whose blocks are smaller than a tile (the
+// entries' sub-block bits are applied on PARTIAL tiles).
+template <int D, bool BLK = false>
 __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
     sa_fwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mk_nat, const __grid_constant__ CUtensorMap mk_col,
@@ -304,7 +308,13 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
         const int lo = src == SRC_N ? lo_n : (src == SRC_T ? lo_t : lo_s);
         const int hi = src == SRC_N ? hi_n : (src == SRC_T ? hi_t : hi_s);
         static_assert(C::TK == 64, "interval mask of 64 keys");
-        mask_interval64(s, lo - k0, hi - k0, -INFINITY);
+        if constexpr (BLK) {
+          const int nj = C::TK / a.blk;
+          const uint32_t nib = (a.bits[e0 + j] >> ((row / a.blk) * nj)) & ((1u << nj) - 1u);
+          mask_bits64(s, interval_bits64(lo - k0, hi - k0) & sub_block_cols(nib, a.blk), -INFINITY);
+        } else {
+          mask_interval64(s, lo - k0, hi - k0, -INFINITY);
+        }
       }
       // row max as a tree (short dependency chains)
       float mx8[8];

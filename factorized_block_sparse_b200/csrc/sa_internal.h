@@ -40,6 +40,10 @@ struct TileTable {
   std::vector<int32_t> ent;      // packed entries, ascending tile per source
   std::vector<int32_t> order;    // rows by descending entry count (launch order)
   std::vector<int32_t> sched;    // per launch slot s: {row order[s], its first entry, its count, 0}
+  // Caller block masks with blocks smaller than the kernel tiles: per entry,
+  // which (row block, column block) pairs of the tile are listed (see
+  // sub_block_bits in the layout builder); empty otherwise.
+  std::vector<int32_t> bits;
   int n_rows = 0;
 };
 
@@ -48,6 +52,7 @@ struct DevTable {
   const int32_t* ent = nullptr;
   const int32_t* order = nullptr;
   const int32_t* sched = nullptr;  // 16-byte aligned, 4 ints per slot
+  const uint32_t* bits = nullptr;  // per entry (caller block masks with blocks below a tile), or null
   int n_rows = 0;
   int nnz = 0;
 };
@@ -82,4 +87,6 @@ int build_layout(sa_layout* L);
 int build_layout_blocks(sa_layout* L, const int32_t* row_ptr, const int32_t* col_idx);
 // Number of key positions of a view (summary view: R * c).
 int view_keys(const sa_layout* L, int view);
+// Per-entry sub-block bits of a caller block mask with blocks below a tile.
+void sub_block_bits(sa_layout* L);
 }  // namespace sa

@@ -304,6 +304,45 @@ int build_layout(sa_layout* L) {
   return SA_OK;
 }
 
+namespace {
+
+// Blocks smaller than the kernel tiles (16, 32 or 64 positions): a tile holds
+// several blocks, some of which may be unlisted.  Per entry, bit
+// (i * nj + j) says whether the i-th block along the tile's rows and the j-th
+// along its columns is listed: forward tiles are 128 queries x 64 keys
+// (i: query block, j: key block), backward tiles 128 keys x 64 queries
+// (i: key block, j: query block).
+bool listed(const Csr& t, int qb, int kb) {
+  if (qb < 0 || qb >= t.n_rows) return false;
+  const auto b = t.col_idx.begin() + t.row_ptr[qb], e = t.col_idx.begin() + t.row_ptr[qb + 1];
+  return std::binary_search(b, e, kb);
+}
+
+void table_bits(TileTable& tt, const Csr& mask, int b, int tm, int tn, bool key_major) {
+  const int ni = tm / b, nj = tn / b;
+  tt.bits.assign(tt.ent.size(), 0);
+  for (int r = 0; r < tt.n_rows; ++r) {
+    for (int e = tt.row_ptr[r]; e < tt.row_ptr[r + 1]; ++e) {
+      const int tile = tt.ent[e] >> 3;
+      uint32_t m = 0;
+      for (int i = 0; i < ni; ++i)
+        for (int j = 0; j < nj; ++j) {
+          const int rb = r * ni + i, cb = tile * nj + j;  // blocks along the tile's rows / columns
+          if (key_major ? listed(mask, cb, rb) : listed(mask, rb, cb)) m |= 1u << (i * nj + j);
+        }
+      tt.bits[e] = static_cast<int32_t>(m);
+    }
+  }
+}
+
+}  // namespace
+
+void sub_block_bits(sa_layout* L) {
+  const Csr& m = L->view[SA_VIEW_NATURAL];
+  table_bits(L->fwd_main, m, L->block, kFwdTQ, kFwdTK, false);
+  table_bits(L->bwd_main, m, L->block, kBwdTK, kBwdTQ, true);
+}
+
 int build_layout_blocks(sa_layout* L, const int32_t* row_ptr, const int32_t* col_idx) {
   // The caller's table is the natural view: per query block, ascending key
   // blocks at or below the diagonal, the diagonal block last.  Diagonal
@@ -328,6 +367,7 @@ int build_layout_blocks(sa_layout* L, const int32_t* row_ptr, const int32_t* col
   L->view[SA_VIEW_NATURAL] = t;
   L->viewT[SA_VIEW_NATURAL] = transpose(t);
   build_kernel_tables(L);
+  if (L->block < kFwdTQ) sub_block_bits(L);
   return SA_OK;
 }
 

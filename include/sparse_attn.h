@@ -144,11 +144,12 @@ int sparse_attn_layout(int pattern, int N, int l, int c, int block, sa_layout** 
  * during the call only) list, per query block r, the key blocks s in the
  * mask, ascending, with 0 <= s <= r and the diagonal block s = r last (so
  * no row is empty).  Element (i, j) attends when its block is listed and
- * j <= i.  block must be a multiple of 128 (the kernels' tile: every tile
- * then lies inside one block) and divide N.
+ * j <= i.  block must divide N and be a multiple of 128 (every kernel tile
+ * then lies inside one block) or one of 16, 32, 64 (a kernel tile then
+ * holds several blocks and masks the unlisted ones element by element).
  * Errors: SA_ERR_INVALID_ARG (null pointer, N < 1, a row that is empty,
  * unsorted, above the diagonal or without its diagonal block),
- * SA_ERR_UNSUPPORTED (block not a multiple of 128, N % block not zero).
+ * SA_ERR_UNSUPPORTED (another block size, N % block not zero).
  */
 int sparse_attn_layout_blocks(int N, int block, const int32_t* row_ptr, const int32_t* col_idx,
                               sa_layout** out);

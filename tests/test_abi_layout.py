@@ -175,7 +175,8 @@ def _random_blocks(nb, seed, p=0.35):
     return rp, ci
 
 
-@pytest.mark.parametrize("N,b,seed", [(1024, 128, 0), (2048, 256, 1), (1536, 128, 2)])
+@pytest.mark.parametrize("N,b,seed", [(1024, 128, 0), (2048, 256, 1), (1536, 128, 2), (1024, 64, 3), (512, 32, 4),
+                                      (256, 16, 5)])
 def test_layout_blocks_bit_exact(sa, N, b, seed):
     from oracle import patterns
 
@@ -199,7 +200,7 @@ def test_layout_blocks_errors(sa):
         sa.Layout.from_blocks(384, 128, [0, 1, 3, 5], [0, 1, 0, 0, 2])  # unsorted row 1
     assert e.value.status == sa.SA_ERR_INVALID_ARG
     with pytest.raises(sa.SparseAttnError) as e:
-        sa.Layout.from_blocks(256, 64, [0, 1, 3, 4, 6], [0, 0, 1, 2, 2, 3])  # block not a multiple of 128
+        sa.Layout.from_blocks(288, 48, [0, 1, 3, 4, 6, 7, 8], [0, 0, 1, 2, 2, 3, 4, 5])  # block 48: not supported
     assert e.value.status == sa.SA_ERR_UNSUPPORTED
     with pytest.raises(sa.SparseAttnError) as e:
         sa.Layout.from_blocks(300, 128, [0, 1, 3], [0, 0, 1])        # N % block

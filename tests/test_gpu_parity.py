@@ -184,18 +184,28 @@ def test_parity_full_size_whole_head(cuda_device, name, sl):
         assert_close(f"{name} ({b},{h}) {n}", got[n][b:b + 1, h:h + 1], ref[n])
 
 
-def test_long_sequence_sampled(cuda_device):
-    """A strided head at N = 2^18 (l = 512, R = 512): sampled rows and key
-    columns against the oracle, and properties at every position."""
-    mode, B, H, N, D, l, c, block = "strided", 1, 1, 1 << 18, 64, 512, 0, 64
+@pytest.mark.parametrize("N,l,rows,cols", [
+    (1 << 18, 512, [0, 1, 777, 131071, 200000, (1 << 18) - 1], [5, 100003, (1 << 18) - 1]),
+    # 2^20 positions, l = 1024: whole 128-row tiles at the start, middle and end; key columns near the end
+    (1 << 20, 1024, list(range(128)) + list(range(524288, 524416)) + list(range((1 << 20) - 128, 1 << 20)),
+     list(range((1 << 20) - 300, (1 << 20) - 290)) + [(1 << 20) - 1]),
+])
+def test_long_sequence_sampled(cuda_device, N, l, rows, cols):
+    """A strided head at N = 2^18 (l = 512) and 2^20 (l = 1024): sampled rows and
+    key columns against the oracle, and properties at every position."""
+    mode, B, H, D, c, block = "strided", 1, 1, 64, 0, 64
     x, got, _ = run_library(mode, B, H, N, D, l, c, block)
     q, k, v, dO = (synth.to_f64(x[n]) for n in ("q", "k", "v", "dO"))
-    rows = np.array([0, 1, 777, 131071, 200000, N - 1])
-    Or, Lr = attention.forward_rows(q, k, v, mode, l, c, rows)
+    rows = np.array(rows)
+    # the oracle's rows in chunks of 16 (a row of scores at N = 2^20 is 8 MB in float64)
+    parts = [rows[i:i + 16] for i in range(0, len(rows), 16)]
+    Or = np.concatenate([attention.forward_rows(q, k, v, mode, l, c, p)[0] for p in parts], axis=2)
+    Lr = np.concatenate([attention.forward_rows(q, k, v, mode, l, c, p)[1] for p in parts], axis=2)
     assert_close("long o", got["o"][:, :, rows], Or)
     assert_close("long lse", got["lse"][:, :, rows], Lr)
-    assert_close("long dq", got["dq"][:, :, rows], attention.dq_rows(q, k, v, dO, mode, l, c, rows))
-    cols = np.array([5, 100003, N - 1])
+    dqr = np.concatenate([attention.dq_rows(q, k, v, dO, mode, l, c, p) for p in parts], axis=2)
+    assert_close("long dq", got["dq"][:, :, rows], dqr)
+    cols = np.array(cols)
     dkc, dvc = attention.dkv_cols(q, k, v, dO, mode, l, c, cols)
     assert_close("long dk", got["dk"][:, :, cols], dkc)
     assert_close("long dv", got["dv"][:, :, cols], dvc)
@@ -213,7 +223,11 @@ def _random_blocks(nb, seed, p=0.35):
 
 
 @pytest.mark.parametrize("B,H,N,D,b,seed", [(1, 2, 2048, 64, 128, 0), (2, 1, 1024, 32, 256, 1),
-                                            (1, 1, 1024, 128, 128, 2)])
+                                            (1, 1, 1024, 128, 128, 2),
+                                            # blocks smaller than a kernel tile: sub-block bits
+                                            (1, 2, 2048, 64, 64, 3), (1, 1, 1024, 32, 32, 4), (2, 1, 768, 64, 16, 5),
+                                            (1, 1, 1024, 128, 32, 6),
+                                            (1, 1, 4096, 64, 64, 7)])  # long rows: the LONG backward shape
 def test_parity_block_mask(cuda_device, B, H, N, D, b, seed):
     """A caller's block mask (sparse_attn_layout_blocks) against the oracle's BlockMask."""
     from factorized_block_sparse_b200 import sparse_attn as sa
