@@ -446,6 +446,16 @@ int kernel_pattern(int pattern) {
   return pattern;
 }
 
+int sm_count();
+
+// Persistent forward grid: every resident CTA slot (two per SM for D <= 64),
+// at most one CTA per item.
+unsigned fwd_grid(int n_rows, int BH, int D) {
+  const long long items = static_cast<long long>(n_rows) * BH;
+  const long long slots = static_cast<long long>(sm_count()) * (D <= 64 ? 2 : 1);
+  return static_cast<unsigned>(std::max(1LL, std::min(items, slots)));
+}
+
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
              float scale, const sa_layout* L, cudaStream_t s) {
@@ -482,6 +492,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.R = g.R;
   a.pattern = kernel_pattern(L->pattern);
   a.t_open = (L->pattern == SA_COLUMN) ? 0 : 1;
+  a.BH = g.BH;
   a.box = make_boxes(g.R, g.c);
   a.scale_log2 = static_cast<float>(1.4426950408889634 * static_cast<double>(scale));
   // Column view first (SA_STRIDED, SA_COLUMN); the natural view then merges
@@ -493,7 +504,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     a.order = dc.fwd_col.order;
     a.q_col = 1;
     a.merge = 0;
-    dim3 grid(g.BH, dc.fwd_col.n_rows);
+    a.n_rows = dc.fwd_col.n_rows;
+    dim3 grid(fwd_grid(a.n_rows, g.BH, D));
     st = launch(K_FWD_COL * K_PATTERNS + L->pattern, s, [&] {
       launch_kernel(kern, grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s, mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat,
                     mv.col, mv.sum, mo_nat, mo_col, a);
@@ -519,7 +531,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   a.q_col = 0;
   a.merge = (col_pass || r_tail > 0) ? 1 : 0;
   if (dc.fwd_main.n_rows == 0) return SA_OK;  // SA_COLUMN: no natural view
-  dim3 grid(g.BH, dc.fwd_main.n_rows);
+  a.n_rows = dc.fwd_main.n_rows;
+  dim3 grid(fwd_grid(a.n_rows, g.BH, D));
   return launch(K_FWD_MAIN * K_PATTERNS + L->pattern, s, [&] {
     launch_kernel(kern, grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM, s, mq.nat, mq.col, mk.nat, mk.col, mk.sum, mv.nat,
                   mv.col, mv.sum, mo_nat, mo_col, a);
@@ -527,6 +540,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
 
 // The default softmax scale 1/sqrt(D).
 float default_scale(int D) { return static_cast<float>(1.0 / std::sqrt(static_cast<double>(D > 0 ? D : 1))); }
