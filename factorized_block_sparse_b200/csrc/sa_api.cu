@@ -13,6 +13,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 #include <new>
 #include <vector>
@@ -583,6 +584,23 @@ int grid_for(long long work_items, int per_block) {
   return static_cast<int>(b);
 }
 
+// Every instantiation of the backward kernel that a launch below may pick:
+// (FINAL_T, BLK, DqMode) = the column view of SA_COLUMN (reduce or store),
+// a secondary or natural pass (reduce, store or final), a natural pass of a
+// caller mask with small blocks (reduce or final).
+template <int D, bool LONG>
+int set_bwd_smem() {
+  constexpr int sm = BwdCfg<D, LONG>::SMEM;
+  int st;
+  if ((st = set_smem(sa_bwd_kernel<D, LONG, false, false, kDqReduce>, sm))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, LONG, false, false, kDqStore>, sm))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, LONG, false, false, kDqFinal>, sm))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, LONG, true, false, kDqReduce>, sm))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, LONG, true, false, kDqStore>, sm))) return st;
+  if ((st = set_smem(sa_bwd_kernel<D, LONG, false, true, kDqReduce>, sm))) return st;
+  return set_smem(sa_bwd_kernel<D, LONG, false, true, kDqFinal>, sm);
+}
+
 template <int D>
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
              void* dq, void* dk, void* dv, int B, int H, int N, float scale, const sa_layout* L, void* ws, cudaStream_t s) {
@@ -598,13 +616,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
 #ifdef SA_TEST_HOOKS
   if ((st = check_tables(dc, N, s))) return st;
 #endif
-  if ((st = set_smem(sa_bwd_kernel<D, false, false>, BwdCfg<D, false>::SMEM))) return st;
-  if ((st = set_smem(sa_bwd_kernel<D, false, true>, BwdCfg<D, false>::SMEM))) return st;
-  if ((st = set_smem(sa_bwd_kernel<D, false, false, true>, BwdCfg<D, false>::SMEM))) return st;
+  if ((st = set_bwd_smem<D, false>())) return st;
   if constexpr (D <= 64) {
-    if ((st = set_smem(sa_bwd_kernel<D, true, false>, BwdCfg<D, true>::SMEM))) return st;
-    if ((st = set_smem(sa_bwd_kernel<D, true, true>, BwdCfg<D, true>::SMEM))) return st;
-    if ((st = set_smem(sa_bwd_kernel<D, true, false, true>, BwdCfg<D, true>::SMEM))) return st;
+    if ((st = set_bwd_smem<D, true>())) return st;
   }
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -618,10 +632,21 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   CUtensorMap mdq_nat, mdq_col;
   if ((st = make_dq_maps(&mdq_nat, &mdq_col, dq_acc, g, L->pattern))) return st;
 
+  const bool sec = dc.bwd_sec.n_rows > 0 && g.R > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN with a whole row
+  const int r_tail = (L->pattern == SA_STRIDED && L->R > 0) ? N - L->R * L->l : 0;
+  // The natural pass writes the final dQ itself when each query step meets one
+  // of its key tiles; the fp32 accumulator then only carries the earlier
+  // passes' sum (and is neither zeroed nor read when there are none).
+  const bool dq_fin = L->dq_single && dc.bwd_main.n_rows > 0;
+  const bool dq_in = sec || r_tail > 0;
+  // ... and the secondary pass stores its rows instead of adding them when it
+  // meets each one once and no partial row adds to them first.
+  const bool dq_store = sec && L->dq_sec_single && r_tail == 0;
+  const bool zero_dq = !(dq_fin && !dq_in) && !dq_store;
   st = launch(K_BWD_PRE * K_PATTERNS + L->pattern, s, [&] {
     launch_kernel(sa_bwd_pre_kernel<D>, grid_for(rows * (D / 8), 256), 256, 0, s,
                   static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ld_nat, ld_col,
-                  dq_acc, g.BH, N, w.n_pad, g.l, g.R);
+                  zero_dq ? dq_acc : nullptr, g.BH, N, w.n_pad, g.l, g.R);
   });
   if (st) return st;
 
@@ -644,13 +669,14 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.box = make_boxes(g.R, g.c);
   a.bits = nullptr;
   a.blk = 0;
-  const bool sec = dc.bwd_sec.n_rows > 0 && g.R > 0;  // SA_STRIDED, SA_FIXED, SA_COLUMN with a whole row
+  a.dq_out = static_cast<__nv_bfloat16*>(dq);
+  a.dq_in = dq_in ? 1 : 0;
   // SA_COLUMN has no natural view: its column-view pass writes the final dK/dV.
   const bool sec_final = L->pattern == SA_COLUMN;
   a.BH = g.BH;
   const int n_sm = sm_count();
   // Tables whose items average many steps take the LONG shape of the kernel.
-  auto run = [&](int kind, const DevTable& t) -> int {
+  auto run = [&](int kind, const DevTable& t, int dqm) -> int {
     EpiMaps em;
     const int mst = make_epi_maps(&em, dk, dv, dk_part, dv_part, g, a.key_view);
     if (mst) return mst;
@@ -663,20 +689,32 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
       launch_kernel(kernel, grid, threads, smem, s, mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                     mv.col, mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v, em.part_k, em.part_v, a);
     };
+    // the kernel variant of a shape: (FINAL_T, BLK) x DqMode
+    auto pick = [&](auto shape) {
+      constexpr bool L = decltype(shape)::value;
+      using CF = BwdCfg<D, L>;
+      if (final_t) {
+        if (dqm == kDqStore) go(sa_bwd_kernel<D, L, true, false, kDqStore>, CF::THREADS, CF::SMEM);
+        else go(sa_bwd_kernel<D, L, true, false, kDqReduce>, CF::THREADS, CF::SMEM);
+      } else if (blk) {
+        if (dqm == kDqFinal) go(sa_bwd_kernel<D, L, false, true, kDqFinal>, CF::THREADS, CF::SMEM);
+        else go(sa_bwd_kernel<D, L, false, true, kDqReduce>, CF::THREADS, CF::SMEM);
+      } else if (dqm == kDqFinal) {
+        go(sa_bwd_kernel<D, L, false, false, kDqFinal>, CF::THREADS, CF::SMEM);
+      } else if (dqm == kDqStore) {
+        go(sa_bwd_kernel<D, L, false, false, kDqStore>, CF::THREADS, CF::SMEM);
+      } else {
+        go(sa_bwd_kernel<D, L, false, false, kDqReduce>, CF::THREADS, CF::SMEM);
+      }
+    };
     return launch(kind, s, [&] {
       if constexpr (D <= 64) {
         if (long_items) {
-          using CL = BwdCfg<D, true>;
-          if (final_t) go(sa_bwd_kernel<D, true, true>, CL::THREADS, CL::SMEM);
-          else if (blk) go(sa_bwd_kernel<D, true, false, true>, CL::THREADS, CL::SMEM);
-          else go(sa_bwd_kernel<D, true, false>, CL::THREADS, CL::SMEM);
+          pick(std::true_type{});
           return;
         }
       }
-      using CS = BwdCfg<D, false>;
-      if (final_t) go(sa_bwd_kernel<D, false, true>, CS::THREADS, CS::SMEM);
-      else if (blk) go(sa_bwd_kernel<D, false, false, true>, CS::THREADS, CS::SMEM);
-      else go(sa_bwd_kernel<D, false, false>, CS::THREADS, CS::SMEM);
+      pick(std::false_type{});
     });
   };
   if (sec) {
@@ -685,9 +723,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_sec.n_rows;
     a.key_view = (L->pattern == SA_FIXED) ? SRC_S : SRC_T;
     a.add_part = 0;
-    if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec))) return st;
+    if ((st = run(K_BWD_SEC * K_PATTERNS + L->pattern, dc.bwd_sec, dq_store ? kDqStore : kDqReduce))) return st;
   }
-  const int r_tail = (L->pattern == SA_STRIDED && L->R > 0) ? N - L->R * L->l : 0;
   if (r_tail > 0) {  // the partial last row's column part (after the column view's pass)
     const long long warps = static_cast<long long>(g.BH) * r_tail;
     st = launch(K_BWD_TAIL * K_PATTERNS + L->pattern, s, [&] {
@@ -707,8 +744,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.n_slots = dc.bwd_main.n_rows;
     a.key_view = SRC_N;
     a.add_part = (sec && !sec_final) ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
-    if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main))) return st;
+    if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main, dq_fin ? kDqFinal : kDqReduce))) return st;
   }
+  if (dq_fin) return SA_OK;
   const long long n8 = rows * D / 8;
   return launch(K_BWD_FINAL * K_PATTERNS + L->pattern, s, [&] {
     launch_kernel(sa_bwd_final_kernel, grid_for(n8, 256), 256, 0, s, static_cast<const float*>(dq_acc),

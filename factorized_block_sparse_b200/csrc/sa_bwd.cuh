@@ -17,7 +17,10 @@
 //                                   smem or, in the LONG shape, in TMEM)
 //   dV += P^T dO, dK += dS^T Q     (TMEM accumulators of the item)
 //   dQ = dS K for the 128 queries of the global step pair (g even, g odd),
-//   restricted to the item's own steps, then reduced into an fp32 workspace.
+//   restricted to the item's own steps, then reduced into an fp32 workspace
+//   (where each query step meets one key tile of the pass: stored into it by
+//   the first pass, or added to the earlier passes' sum and stored as the
+//   final bf16 rows by the natural pass).
 // K/V are double-buffered so the next item's tiles load during this one, and
 // the dV/dK epilogue of an item runs in the dQ warps while the next item's
 // steps proceed.
@@ -64,7 +67,19 @@ struct BwdArgs {
   BoxSet box;        // column / summary TMA boxes per tile height
   const uint32_t* bits;  // sub-block bits per entry (caller block masks with blocks below a tile)
   int blk;               // their block size (16, 32 or 64), else 0
+  // kDqFinal passes (below): the final bf16 dQ rows, and whether earlier
+  // passes left an fp32 sum in the accumulator to add.
+  __nv_bfloat16* dq_out;
+  int dq_in;
 };
+
+// How a pass hands over its dQ rows (a template argument, so that each form
+// is its own instantiation):
+//   kDqReduce: reduced into the fp32 accumulator;
+//   kDqStore:  stored into it (the first pass, which meets every row once);
+//   kDqFinal:  added to the earlier passes' sum and stored as final bf16 rows
+//              (the natural pass, which meets every row once and is the last).
+enum DqMode : int { kDqReduce = 0, kDqStore = 1, kDqFinal = 2 };
 
 // Two shapes of the same kernel.  LONG is for tables whose items run many
 // steps (D <= 64): P^T is written into TMEM over the second half of its
@@ -239,7 +254,8 @@ __device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size
 // column view of SA_COLUMN, which has no natural view).
 // BLK: a caller block mask whose blocks are smaller than a tile (the
 // entries' sub-block bits are applied on PARTIAL steps).
-template <int D, bool LONG, bool FINAL_T, bool BLK = false>
+// DQM: the DqMode of the pass.
+template <int D, bool LONG, bool FINAL_T, bool BLK = false, int DQM = kDqReduce>
 __global__ void __launch_bounds__(480, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mdo_nat, const __grid_constant__ CUtensorMap mdo_col,
@@ -689,14 +705,75 @@ __global__ void __launch_bounds__(480, 1)
         const int g = gs + jj;
         if (!((g & 1) || jj == it.n - 1)) continue;
         const int qb = qi % C::DQBUF;
-        ok = ok && mbar_wait(bar_dq_full + qb, (qi / C::DQBUF) & 1, abort_flag);
-        tc_fence_after();
+        if constexpr (DQM != kDqFinal) {
+          ok = ok && mbar_wait(bar_dq_full + qb, (qi / C::DQBUF) & 1, abort_flag);
+          tc_fence_after();
+        }
         // rows 0..63 belong to global step 2*(g/2), rows 64..127 to the next one
         const int gstep = (g & ~1) + (row >> 6);
         const int js = gstep - gs;
         const bool svalid = js >= 0 && js <= jj;  // the step (and so this warp's 32 rows) is this item's
         const int xw = svalid ? (a.ent[it.e0 + js] >> 3) * C::TQ + (row & 32) : 0;  // warp's first view row
-        if constexpr (C::DQ_TMA) {
+        if constexpr (C::DQ_TMA && DQM == kDqFinal) {
+          // The natural pass is the last to reach these rows: dQ = (earlier
+          // sum) + s dS K, rounded to bf16 and stored by the lanes (one row
+          // each, 16-byte chunks).  The earlier sum is requested into the
+          // staging buffer before the product is waited for.
+          uint8_t* stg = smem + C::OFF_DQS + quarter * C::DQS_WARP_BYTES;
+          const bool fin_in = svalid && a.dq_in;
+          if (fin_in) {
+            fence_proxy_async_smem();  // earlier reads of the staging come before the load
+            __syncwarp();
+            if (lane == 0) {
+              bulk_wait_read_all();  // earlier stores and reduces have read the staging
+              mbar_arrive_expect_tx(bar_epi + quarter, 32 * D * 4);
+#pragma unroll
+              for (int bx = 0; bx < D / 32; ++bx)
+                tma_load_3d(stg + bx * 4096, &mdq_nat, bar_epi + quarter, bx * 32, xw, it.bh);
+            }
+          }
+          ok = ok && mbar_wait(bar_dq_full + qb, (qi / C::DQBUF) & 1, abort_flag);
+          tc_fence_after();
+          float gq[D];
+#pragma unroll
+          for (int i = 0; i < D / 16; ++i) tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, gq + i * 16);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar_dq_free + qb);  // the TMEM buffer is free; the rows are in registers
+          if (fin_in) {
+            if (ok) ok = mbar_wait(bar_epi + quarter, epi_n & 1, abort_flag);
+            else mbar_wait_drain(bar_epi + quarter, epi_n & 1);  // the load lands before the kernel ends
+            ++epi_n;
+          }
+          const int x = xw + lane;
+          if (svalid && x < a.N) {
+            uint4* dst = reinterpret_cast<uint4*>(a.dq_out + (static_cast<size_t>(it.bh) * a.N + x) * D);
+#pragma unroll
+            for (int bx = 0; bx < D / 32; ++bx)
+#pragma unroll
+              for (int c8 = 0; c8 < 4; ++c8) {
+                float v8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v8[u] = gq[bx * 32 + c8 * 8 + u] * a.scale;
+                if (fin_in) {
+                  const float4 t0 = *reinterpret_cast<const float4*>(stg + bx * 4096 + sw128_offset(lane, 2 * c8));
+                  const float4 t1 = *reinterpret_cast<const float4*>(stg + bx * 4096 + sw128_offset(lane, 2 * c8 + 1));
+                  v8[0] += t0.x;
+                  v8[1] += t0.y;
+                  v8[2] += t0.z;
+                  v8[3] += t0.w;
+                  v8[4] += t1.x;
+                  v8[5] += t1.y;
+                  v8[6] += t1.z;
+                  v8[7] += t1.w;
+                }
+                dst[bx * 4 + c8] = make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]),
+                                              pack_bf16(v8[4], v8[5]), pack_bf16(v8[6], v8[7]));
+              }
+          }
+          fence_proxy_async_smem();  // these reads come before the staging's next async write
+          __syncwarp();
+        } else if constexpr (C::DQ_TMA) {
           float gq[D];
 #pragma unroll
           for (int i = 0; i < D / 16; ++i) tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, gq + i * 16);
@@ -723,16 +800,24 @@ __global__ void __launch_bounds__(480, 1)
                   const int rb = a.box.b[0].rb_t;
                   for (int s0 = 0; s0 < 32; s0 += rb) {
                     const int t = xw + s0;
-                    tma_reduce_add_4d(&mdq_col, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
+                    if constexpr (DQM == kDqStore)
+                      tma_store_4d(&mdq_col, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
+                    else
+                      tma_reduce_add_4d(&mdq_col, stg + bx * 4096 + s0 * 128, bx * 32, t / a.R, t % a.R, it.bh);
                   }
                 } else {
-                  tma_reduce_add_3d(&mdq_nat, stg + bx * 4096, bx * 32, xw, it.bh);
+                  if constexpr (DQM == kDqStore) tma_store_3d(&mdq_nat, stg + bx * 4096, bx * 32, xw, it.bh);
+                  else tma_reduce_add_3d(&mdq_nat, stg + bx * 4096, bx * 32, xw, it.bh);
                 }
               }
               bulk_commit_group();
             }
           }
         } else {
+          if constexpr (DQM == kDqFinal) {
+            ok = ok && mbar_wait(bar_dq_full + qb, (qi / C::DQBUF) & 1, abort_flag);
+            tc_fence_after();
+          }
           const int x = xw + (row & 31);
           const bool qvalid = svalid && x < a.N;
           const int qn = (q_src == SRC_T) ? (x % a.R) * a.l + x / a.R : x;
@@ -743,10 +828,36 @@ __global__ void __launch_bounds__(480, 1)
             tmem_ld16(tmem + lane_base + C::COL_DQ + qb * D + i * 16, gq);
             tmem_wait_ld();
             if (qvalid) {
+              if constexpr (DQM == kDqFinal) {  // final dQ row (as in the staged form above)
+                float v16[16];
 #pragma unroll
-              for (int u = 0; u < 16; u += 4)
-                red_add_v4(dstp + i * 16 + u, gq[u] * a.scale, gq[u + 1] * a.scale, gq[u + 2] * a.scale,
-                           gq[u + 3] * a.scale);
+                for (int u = 0; u < 16; ++u) v16[u] = gq[u] * a.scale;
+                if (a.dq_in) {
+#pragma unroll
+                  for (int u = 0; u < 16; u += 4) {
+                    const float4 t = *reinterpret_cast<const float4*>(dstp + i * 16 + u);
+                    v16[u] += t.x;
+                    v16[u + 1] += t.y;
+                    v16[u + 2] += t.z;
+                    v16[u + 3] += t.w;
+                  }
+                }
+                uint4* dst = reinterpret_cast<uint4*>(a.dq_out + (static_cast<size_t>(it.bh) * a.N + qn) * D + i * 16);
+#pragma unroll
+                for (int u = 0; u < 16; u += 8)
+                  dst[u / 8] = make_uint4(pack_bf16(v16[u], v16[u + 1]), pack_bf16(v16[u + 2], v16[u + 3]),
+                                          pack_bf16(v16[u + 4], v16[u + 5]), pack_bf16(v16[u + 6], v16[u + 7]));
+              } else if constexpr (DQM == kDqStore) {
+#pragma unroll
+                for (int u = 0; u < 16; u += 4)
+                  *reinterpret_cast<float4*>(dstp + i * 16 + u) =
+                      make_float4(gq[u] * a.scale, gq[u + 1] * a.scale, gq[u + 2] * a.scale, gq[u + 3] * a.scale);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 16; u += 4)
+                  red_add_v4(dstp + i * 16 + u, gq[u] * a.scale, gq[u + 1] * a.scale, gq[u + 2] * a.scale,
+                             gq[u + 3] * a.scale);
+              }
             }
           }
           tc_fence_before();
@@ -922,7 +1033,7 @@ __global__ void __launch_bounds__(480, 1)
 //   (in [64-step][2][64] blocks) to the natural-order array and, for the
 //   strided pattern, at the row's column-major position
 //   t = (i mod l) * R + i / l; pads positions [N, n_pad) of both with
-//   (-inf, 0); zeroes the fp32 dQ accumulator.
+//   (-inf, 0); zeroes the fp32 dQ accumulator (null: no pass adds into it).
 template <int D>
 __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dO,
@@ -974,9 +1085,11 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
           ld_col[o + (t / 64) * 128 + 64 + (t % 64)] = -acc;
         }
       }
-      float4* z = reinterpret_cast<float4*>(dq_acc + r * D + sub * 8);
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (dq_acc) {
+        float4* z = reinterpret_cast<float4*>(dq_acc + r * D + sub * 8);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
   }
   const int pad = n_pad - N;

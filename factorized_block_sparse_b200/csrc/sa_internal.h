@@ -75,6 +75,12 @@ struct sa_layout {
   sa::TileTable fwd_col;   // column-order query tiles: T-view keys (strided)
   sa::TileTable bwd_main;  // natural key tiles: N-view query tiles
   sa::TileTable bwd_sec;   // T-order (strided) or summary-order (fixed) key tiles
+  // Every 64-query step of the natural view meets exactly one key tile, so
+  // the backward's natural pass completes each dQ row with one product.
+  bool dq_single = false;
+  // The same for the secondary view's key tiles over the query steps of its
+  // whole rows (the column view with R dividing 64).
+  bool dq_sec_single = false;
   mutable std::mutex mu;
   mutable std::vector<sa::DeviceCopy> dev;
 };

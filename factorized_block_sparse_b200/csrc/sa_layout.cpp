@@ -209,6 +209,22 @@ int view_keys(const sa_layout* L, int view) {
 
 namespace {
 
+// Whether every 64-query step of [0, N) is the entry of exactly one key tile
+// of a backward table (the fixed pattern's own-block view with l = 128, the
+// block-diagonal views, the column view when R divides 64): the pass over
+// that table then meets each dQ row once.
+bool one_key_tile_per_step(const TileTable& t, int N) {
+  const int steps = (N + kBwdTQ - 1) / kBwdTQ;
+  if (t.n_rows == 0 || static_cast<long long>(t.ent.size()) != steps) return false;
+  std::vector<uint8_t> seen(steps, 0);
+  for (const int32_t e : t.ent) {
+    const int x = e >> 3;
+    if (x < 0 || x >= steps || seen[x]) return false;
+    seen[x] = 1;
+  }
+  return true;
+}
+
 // Kernel tile tables from the public tables in L->view / L->viewT.
 void build_kernel_tables(sa_layout* L) {
   const long long N = L->N;
@@ -273,6 +289,7 @@ void build_kernel_tables(sa_layout* L) {
   } else {
     finish_table(L->bwd_main, {});
   }
+  L->dq_single = one_key_tile_per_step(L->bwd_main, L->N);
   // Backward, secondary view key tiles (T order or summary order).
   if (L->has[SA_VIEW_COLUMN] || L->has[SA_VIEW_SUMMARY]) {
     const int v = L->has[SA_VIEW_COLUMN] ? SA_VIEW_COLUMN : SA_VIEW_SUMMARY;
@@ -283,6 +300,7 @@ void build_kernel_tables(sa_layout* L) {
     for (size_t r = 0; r < kt.size(); ++r)
       for (auto& e : kt[r].ent) rows[r].push_back(pack_entry(e.first, src, e.second));
     finish_table(L->bwd_sec, rows);
+    L->dq_sec_single = one_key_tile_per_step(L->bwd_sec, static_cast<int>(v == SA_VIEW_COLUMN ? Ng : N));
   } else {
     finish_table(L->bwd_sec, {});
   }

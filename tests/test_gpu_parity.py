@@ -67,6 +67,10 @@ SMALL = [
     ("strided", 1, 1, 200, 64, 256, 0, 8),      # N < l: no whole row, no column part
     ("fixed", 1, 1, 200, 64, 256, 64, 8),       # N < l: one partial block, no summary view
     ("strided", 1, 1, 3000, 64, 192, 0, 8),     # R = 15 + 120, the natural view in the LONG shape
+    # one key tile per query step in the natural view with no earlier pass:
+    # the natural pass writes the final dQ alone (D = 128, ragged)
+    ("block", 1, 1, 1088, 128, 128, 0, 64),
+    ("block", 2, 1, 1000, 32, 64, 0, 8),
 ]
 
 
@@ -240,6 +244,45 @@ def test_parity_block_mask(cuda_device, B, H, N, D, b, seed):
     for name in ("o", "lse", "dq", "dk", "dv"):
         assert np.isfinite(got[name]).all(), name
         assert_close(f"blocks N={N} D={D} {name}", got[name], ref[name])
+
+
+@pytest.mark.parametrize("B,H,N,D,b", [(1, 2, 1024, 64, 64), (1, 1, 1024, 128, 32), (2, 1, 960, 32, 16)])
+def test_parity_block_diagonal_mask(cuda_device, B, H, N, D, b):
+    """A caller's mask of the diagonal blocks only (blocks below a tile): each
+    64-query step meets one key tile, the case where the natural pass writes
+    the final dQ itself."""
+    from factorized_block_sparse_b200 import sparse_attn as sa
+    from oracle import patterns
+
+    rp, ci = _random_blocks(N // b, 0, p=0.0)
+    lay = sa.Layout.from_blocks(N, b, rp, ci)
+    x, got, _ = run_library("blocks", B, H, N, D, 1, 0, b, layout=lay)
+    ref = oracle_full(x, patterns.BlockMask(N, b, rp, ci), 1, 0)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert np.isfinite(got[name]).all(), name
+        assert_close(f"diagonal blocks N={N} D={D} b={b} {name}", got[name], ref[name])
+
+
+@pytest.mark.parametrize("mode,N,l,c,finalise", [
+    ("fixed", 2048, 128, 32, 0),   # own block = one 128-key tile per 64-query step
+    ("block", 960, 64, 0, 0),
+    ("fixed", 2048, 256, 32, 1),   # a step of the second half of a block meets two key tiles
+    ("strided", 2048, 64, 0, 1),
+    ("column", 2048, 64, 0, 1),    # no natural view
+])
+def test_final_dq_pass(cuda_device, mode, N, l, c, finalise):
+    """The separate dQ finalise runs only where the natural view's pass cannot
+    complete each dQ row with one product."""
+    from factorized_block_sparse_b200 import sparse_attn as sa
+
+    sa.timing_reset()
+    sa.timing_enable(True)
+    try:
+        run_library(mode, 1, 1, N, 64, l, c, 64)
+    finally:
+        sa.timing_enable(False)
+    assert sa.kernel_times()[f"sa_bwd_finalize_dq.{mode}"][1] == finalise
+    sa.timing_reset()
 
 
 def test_block_mask_of_all_lower_blocks_equals_all(cuda_device):
