@@ -611,41 +611,74 @@ def measure_configs(sa, names, pk, dev, stream, flush, steps=10, warmup=3):
 
 
 def measure_e2e(sa, state, stream, steps, step_flops, world, dev):
+    """The step through the public API from pinned host buffers: every step
+    copies its inputs (q, k, v, dO) host->device and its results (o, lse, dq,
+    dk, dv) device->host.  Steps are pipelined over two device buffer sets and
+    three streams (host->device copies, compute, device->host copies), so one
+    step's copies in each direction overlap the neighbouring steps' compute
+    and opposite copies, as a training loop feeding the op from the host would
+    run; the value is the time from the first copy to the last one over the
+    steps."""
     import torch
 
-    host = []
     h2d = d2h = 0
+    hin = []
     for s in state:
-        hin = {t: s["x"][t].pin_memory() for t in ("q", "k", "v", "dO")}
-        hout = {t: torch.empty(s[t].shape, dtype=s[t].dtype, pin_memory=True) for t in ("o", "lse", "dq", "dk", "dv")}
-        h2d += sum(t.numel() * t.element_size() for t in hin.values())
-        d2h += sum(t.numel() * t.element_size() for t in hout.values())
-        host.append((hin, hout))
-    sptr = stream.cuda_stream
+        t_in = {t: s["x"][t].pin_memory() for t in ("q", "k", "v", "dO")}
+        h2d += sum(t.numel() * t.element_size() for t in t_in.values())
+        hin.append(t_in)
+    # two device sets (set 0 is the bench's own tensors) and a pinned output set per device set
+    sets = [state, [dict(s, **{t: torch.empty_like(s[t]) for t in ("q", "k", "v", "dO", "o", "lse", "dq", "dk", "dv")},
+                         ws=torch.empty_like(s["ws"])) for s in state]]
+    hout = [[{t: torch.empty(s[t].shape, dtype=s[t].dtype, pin_memory=True) for t in ("o", "lse", "dq", "dk", "dv")}
+             for s in state] for _ in range(2)]
+    d2h = sum(t.numel() * t.element_size() for h in hout[0] for t in h.values())
+    s_in, s_out, s_c = torch.cuda.Stream(dev), torch.cuda.Stream(dev), stream
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    cptr = s_c.cuda_stream
 
-    def one():
-        for s, (hin, hout) in zip(state, host):
-            for t in ("q", "k", "v", "dO"):
-                s[t].copy_(hin[t], non_blocking=True)
-            sa.sparse_attn_fwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["lay"], sptr)
-            sa.sparse_attn_bwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["dO"], s["dq"], s["dk"], s["dv"],
-                               s["lay"], s["ws"], sptr)
-            for t in ("o", "lse", "dq", "dk", "dv"):
-                hout[t].copy_(s[t], non_blocking=True)
+    def one(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_c[b])  # step i-2 has consumed this set's inputs
+            for d, h in zip(sets[b], hin):
+                for t in ("q", "k", "v", "dO"):
+                    d[t].copy_(h[t], non_blocking=True)
+            ev_in[b].record(s_in)
+        s_c.wait_event(ev_in[b])
+        if i >= 2:
+            s_c.wait_event(ev_out[b])  # step i-2's results have left this set
+        for d in sets[b]:
+            sa.sparse_attn_fwd(d["q"], d["k"], d["v"], d["o"], d["lse"], d["lay"], cptr)
+            sa.sparse_attn_bwd(d["q"], d["k"], d["v"], d["o"], d["lse"], d["dO"], d["dq"], d["dk"], d["dv"],
+                               d["lay"], d["ws"], cptr)
+        ev_c[b].record(s_c)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_c[b])
+            for d, h in zip(sets[b], hout[b]):
+                for t in ("o", "lse", "dq", "dk", "dv"):
+                    h[t].copy_(d[t], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(3):
-        one()
+    for i in range(3):
+        one(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(steps):
+        one(i)
+    s_out.wait_event(ev_c[(steps - 1) % 2])
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
     return {"value": round(world * step_flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": "two device buffer sets; host->device copies, compute and device->host copies on "
+                         "three streams"}
 
 
 def read_traffic(kernel):
