@@ -211,8 +211,9 @@ size_t sparse_attn_bwd_workspace_size(int B, int H, int N, int D, const sa_layou
  * workspace: caller-owned device memory of at least
  * sparse_attn_bwd_workspace_size() bytes, 256-byte aligned; its contents on
  * entry do not matter and on exit are unspecified.  dq accumulates in
- * float32 by bulk reduce-adds in arrival order, so its last bits may vary
- * from run to run; dk and dv are deterministic.
+ * float32 by bulk reduce-adds in arrival order where several key tiles of a
+ * pass meet a query row, so its last bits may vary from run to run; dk and
+ * dv are deterministic.
  * Errors: as sparse_attn_fwd, plus SA_ERR_WORKSPACE.
  */
 int sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -261,7 +262,8 @@ int sparse_attn_bwd_ex(const void* q, const void* k, const void* v, const void* 
  *    before any stream capture;
  *  - every call on a device shares the one array, which keeps whatever the
  *    last call left in it.  The kernels set everything they read from it
- *    (the dQ accumulator is cleared by the preprocess kernel), so no clearing
+ *    (the dQ accumulator is cleared by the preprocess kernel or wholly
+ *    overwritten by the first pass that meets it), so no clearing
  *    is needed between calls, but calls whose GPU work overlaps (different
  *    streams, or different host threads) race on the array and give wrong
  *    results: order them on one stream or with events.
