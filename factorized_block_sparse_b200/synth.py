@@ -62,3 +62,30 @@ def inputs(B, H, N, D, seed_offset=0):
 def to_f64(t):
     """bfloat16 (or any) CPU tensor -> float64 NumPy array, exactly."""
     return t.detach().to("cpu").double().numpy()
+
+
+# Inputs of the Sparse Transformer block around the op (model width C = H * D,
+# hidden width 4C).  Projections are drawn N(0, 1) and scaled by 1/sqrt(fan
+# in), then rounded to bfloat16; the layer-norm gains are 1 + 0.1 N(0, 1) and
+# the biases 0.1 N(0, 1) in float32 (so the affine part is exercised).
+BLOCK_WEIGHTS = (("w_qkv", 1, 3), ("w_o", 1, 1), ("w_1", 1, 4), ("w_2", 4, 1))  # name, rows / C, cols / C
+
+
+def block_inputs(B, N, C, seed_offset=0):
+    """x and the upstream gradient dy as CPU bfloat16 ``[B, N, C]`` tensors."""
+    return {"x": normal_bf16((B, N, C), 10 + seed_offset), "dy": normal_bf16((B, N, C), 11 + seed_offset)}
+
+
+def block_params(C, seed=20):
+    """The block's parameters as CPU tensors: bfloat16 projections (``[in, out]``
+    row-major) and float32 layer-norm gains and biases."""
+    import torch
+
+    p = {}
+    for i, (name, r, c) in enumerate(BLOCK_WEIGHTS):
+        w = normal_f32((r * C, c * C), seed + i) / np.float32(np.sqrt(r * C))
+        p[name] = torch.from_numpy(w).to(torch.bfloat16)
+    for i, name in enumerate(("ln1", "ln2")):
+        p[name + "_g"] = torch.from_numpy(1.0 + 0.1 * normal_f32((C,), seed + 10 + 2 * i))
+        p[name + "_b"] = torch.from_numpy(0.1 * normal_f32((C,), seed + 11 + 2 * i))
+    return p
