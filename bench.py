@@ -375,6 +375,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--configs", type=int, default=1, help="1: also time every other named configuration")
     ap.add_argument("--streams", type=int, default=2, help="streams the step's independent workloads use")
+    ap.add_argument("--block", type=int, default=1, help="1: also time the Sparse Transformer block around the op")
     args = ap.parse_args()
     names = STEPS[args.workload]
     if args.warmup < 3:
@@ -509,6 +510,11 @@ def main():
     if args.configs and world == 1:
         configs = measure_configs(sa, [n for n in CONFIGS if n not in names], pk, dev, stream, flush)
 
+    # the Sparse Transformer block around the op (extra key)
+    block = None
+    if args.block and world == 1:
+        block = measure_block(sa, pk, dev, stream, flush)
+
     # end to end through the C ABI with pinned host buffers
     e2e = None
     if args.e2e_steps > 0:
@@ -534,6 +540,7 @@ def main():
                                 "step's workloads on their own streams"},
         "workloads": workload_lines(state, ktimes, pk),
         "configs": configs,
+        "block": block,
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
@@ -607,6 +614,70 @@ def measure_configs(sa, names, pk, dev, stream, flush, steps=10, warmup=3):
         del q, k, v, dO, o, lse, dq, dk, dv, ws
         lay.close()
         torch.cuda.empty_cache()
+    return out
+
+
+def block_flops(w, counts, C):
+    """FLOPs of one forward + backward of the block (the backward recomputes
+    the forward but for y): projections 2 M K Nn each, 24 M C^2 in the
+    forward and 16 + 48 M C^2 in the backward; the attention's nonzero-block
+    FLOPs forward, again in the backward's recomputation, and backward."""
+    M = w["B"] * w["N"]
+    fa, ba = flops(w, counts)
+    return (24 + 64) * M * C * C + 2 * fa + ba, (24 + 64) * M * C * C
+
+
+def measure_block(sa, pk, dev, stream, flush, steps=10, warmup=3):
+    """forward + backward of the Sparse Transformer block at the text-fixed
+    shape (B=2, N=12288, H=8, D=64: C=512, the fixed pattern), CUDA events
+    around each step, L2 flushed before it; random-init parameters."""
+    import torch
+
+    from factorized_block_sparse_b200 import sparse_block as sb
+
+    w = synth.WORKLOADS["text-fixed"]
+    B, N, H, D = w["B"], w["N"], w["H"], w["D"]
+    C = H * D
+    counts, lay = block_counts(w, sa)
+    fl, fl_gemm = block_flops(w, counts, C)
+    xin = synth.block_inputs(B, N, C)
+    x, dy = xin["x"].to(dev), xin["dy"].to(dev)
+    p = {k: v.to(dev) for k, v in synth.block_params(C).items()}
+    ws = sb.workspace(B, N, H, D, lay, dev)
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    g = {n: torch.empty(p[n].shape, dtype=torch.float32, device=dev) for n in sb.PARAMS}
+    sptr = stream.cuda_stream
+
+    def one():
+        sb.sparse_block_fwd(x, p, y, H, lay, ws, sptr)
+        sb.sparse_block_bwd(x, dy, p, dx, g, H, lay, ws, sptr)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        one()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    st = sa.sparse_attn_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the block: {sa.strerror(st)}")
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    achieved = fl / (ms * 1e-3) / 1e12
+    out = {"workload": f"one block, fixed pattern, B={B}, N={N}, H={H}, D={D} (C={C}, hidden {4 * C}), l={w['l']}, "
+                       f"c={w['c']}, block={w['block']}; bf16 activations, cuBLAS projections",
+           "ms_per_step": round(ms, 4), "tflops": round(achieved, 2), "unit": "TFLOP/s",
+           "flops_per_step": {"total": fl, "projections": fl_gemm},
+           "tokens_per_s": round(B * N / (ms * 1e-3), 1),
+           "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16"],
+                        "frac": round(achieved / pk["bf16"], 4)}}
+    del x, dy, p, ws, y, dx, g
+    lay.close()
+    torch.cuda.empty_cache()
     return out
 
 

@@ -32,6 +32,7 @@ def nvcc_path():
 def command(out=LIB, extra=()):
     return [nvcc_path(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
             "-lineinfo", "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static",
+            "-Xlinker", "-soname=" + os.path.basename(out),
             "-I", os.path.join(ROOT, "include"), "-o", out, *extra, *SOURCES]
 
 
@@ -64,7 +65,37 @@ def build_test_lib(force=False, verbose=False):
     return TEST_LIB
 
 
+# The Sparse Transformer block around the op: its own library, linked against
+# libsparse_attn.so (found next to it) and cuBLAS (the projections).
+BLOCK_LIB = os.path.join(HERE, "libsparse_block.so")
+BLOCK_SOURCES = [os.path.join(HERE, "csrc", "sb_block.cu")]
+BLOCK_HEADERS = [os.path.join(ROOT, "include", "sparse_block.h"), os.path.join(ROOT, "include", "sparse_attn.h")]
+
+
+def cuda_lib_dir():
+    return os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64")
+
+
+def build_block_lib(force=False, verbose=False):
+    """Compile libsparse_block.so (after libsparse_attn.so) if out of date; return its path."""
+    build()
+    if not force and os.path.exists(BLOCK_LIB):
+        t = os.path.getmtime(BLOCK_LIB)
+        if all(os.path.getmtime(p) <= t for p in BLOCK_SOURCES + BLOCK_HEADERS + [LIB]):
+            return BLOCK_LIB
+    cmd = [nvcc_path(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+           "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static", "-Xlinker", "-soname=libsparse_block.so",
+           "-I", os.path.join(ROOT, "include"), "-o", BLOCK_LIB, *BLOCK_SOURCES,
+           "-L", HERE, "-lsparse_attn", "-L", cuda_lib_dir(), "-lcublas",
+           "-Xlinker", "-rpath,$ORIGIN", "-Xlinker", "-rpath," + cuda_lib_dir()]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    return BLOCK_LIB
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
           extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
     build_test_lib(force="--force" in sys.argv, verbose=True)
+    build_block_lib(force="--force" in sys.argv, verbose=True)

@@ -1,0 +1,466 @@
+// The Sparse Transformer block around the attention op: layer norms, the
+// GELU feed-forward, the residual stream and the head layout in CUDA kernels
+// of this file, the projections as cuBLAS GEMMs (bf16 in, fp32 accumulation)
+// and the attention through libsparse_attn's C ABI.
+//
+// The block ("[논문 리뷰] Generating Long Sequences with Sparse Transformers",
+// "제안 방법", third and fourth items; pcnews translation, "Глубокое
+// внимание"): pre-activation residual sub-blocks with layer normalisation,
+// recomputed in the backward pass from the block input.  Formulas and
+// readings: include/sparse_block.h.
+//
+// Data layout: activations [M = B*N rows][C = H*D] bf16 row-major; the
+// attention's q, k, v, o in its own [B, H, N, D] layout (head h = columns
+// h*D .. h*D+D-1 of a C-wide row), converted by to_heads / from_heads.
+#include <cublas_v2.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sparse_block.h"
+
+namespace sb {
+
+constexpr float kEps = 1e-5f;
+constexpr int kMaxC = 6144;  // model width limit (2 C floats of shared memory per layer-norm block)
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) v += __shfl_xor_sync(0xffffffffu, v, w);
+  return v;
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* f) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float* f) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+// Mean and 1/sqrt(var + eps) of a C-wide bf16 row, one warp (two passes
+// over the row: the deviations are summed about the mean).
+__device__ __forceinline__ void row_stats(const __nv_bfloat16* xr, int C, int lane, float& mean, float& rstd) {
+  float s = 0.f;
+  for (int i = lane * 8; i < C; i += 256) {
+    float f[8];
+    load8(xr + i, f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s += f[u];
+  }
+  mean = warp_sum(s) / C;
+  float v = 0.f;
+  for (int i = lane * 8; i < C; i += 256) {
+    float f[8];
+    load8(xr + i, f);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v += (f[u] - mean) * (f[u] - mean);
+  }
+  rstd = rsqrtf(warp_sum(v) / C + kEps);
+}
+
+// y = (x - mean) * rstd * g + b per row; one warp per row.
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
+                                                     const float* __restrict__ b, __nv_bfloat16* __restrict__ y,
+                                                     long long M, int C) {
+  const int lane = threadIdx.x & 31;
+  const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r = w0; r < M; r += nw) {
+    const __nv_bfloat16* xr = x + r * C;
+    float mean, rstd;
+    row_stats(xr, C, lane, mean, rstd);
+    for (int i = lane * 8; i < C; i += 256) {
+      float f[8];
+      load8(xr + i, f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] = (f[u] - mean) * rstd * g[i + u] + b[i + u];
+      store8(y + r * C + i, f);
+    }
+  }
+}
+
+// Layer-norm backward with the residual added:
+//   dx = resid + rstd (dxh - mean(dxh) - xh mean(dxh xh)),  dxh = dy g,
+//   dg += sum_rows dy xh,  db += sum_rows dy  (float32, zeroed by the caller).
+// One warp per row; the block sums its rows' dg/db in shared memory and
+// adds them to global memory once.
+__global__ void __launch_bounds__(256) ln_bwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
+                                                     const __nv_bfloat16* __restrict__ dy,
+                                                     const __nv_bfloat16* __restrict__ resid,
+                                                     __nv_bfloat16* __restrict__ dx, float* __restrict__ dg,
+                                                     float* __restrict__ db, long long M, int C) {
+  extern __shared__ float acc[];  // [2][C]
+  for (int i = threadIdx.x; i < 2 * C; i += blockDim.x) acc[i] = 0.f;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long r = w0; r < M; r += nw) {
+    const __nv_bfloat16* xr = x + r * C;
+    const __nv_bfloat16* dr = dy + r * C;
+    float mean, rstd;
+    row_stats(xr, C, lane, mean, rstd);
+    float s1 = 0.f, s2 = 0.f;
+    for (int i = lane * 8; i < C; i += 256) {
+      float f[8], d[8];
+      load8(xr + i, f);
+      load8(dr + i, d);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float xh = (f[u] - mean) * rstd;
+        const float dxh = d[u] * g[i + u];
+        s1 += dxh;
+        s2 += dxh * xh;
+        atomicAdd(&acc[i + u], d[u] * xh);
+        atomicAdd(&acc[C + i + u], d[u]);
+      }
+    }
+    s1 = warp_sum(s1) / C;
+    s2 = warp_sum(s2) / C;
+    for (int i = lane * 8; i < C; i += 256) {
+      float f[8], d[8], o[8];
+      load8(xr + i, f);
+      load8(dr + i, d);
+      load8(resid + r * C + i, o);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float xh = (f[u] - mean) * rstd;
+        o[u] += rstd * (d[u] * g[i + u] - s1 - xh * s2);
+      }
+      store8(dx + r * C + i, o);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    atomicAdd(&dg[i], acc[i]);
+    atomicAdd(&db[i], acc[C + i]);
+  }
+}
+
+// gelu(u) = u Phi(u) = u (1 + erf(u / sqrt 2)) / 2, 8 elements a thread.
+__global__ void __launch_bounds__(256) gelu_kernel(const __nv_bfloat16* __restrict__ u, __nv_bfloat16* __restrict__ out,
+                                                   long long n8) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float f[8];
+    load8(u + i * 8, f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) f[k] = 0.5f * f[k] * (1.f + erff(f[k] * 0.70710678118654752f));
+    store8(out + i * 8, f);
+  }
+}
+
+// du = dg (Phi(u) + u phi(u)), phi the standard normal density.
+__global__ void __launch_bounds__(256) gelu_bwd_kernel(const __nv_bfloat16* __restrict__ u,
+                                                       const __nv_bfloat16* __restrict__ dg,
+                                                       __nv_bfloat16* __restrict__ du, long long n8) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float f[8], d[8];
+    load8(u + i * 8, f);
+    load8(dg + i * 8, d);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float phi = 0.3989422804014327f * expf(-0.5f * f[k] * f[k]);
+      d[k] *= 0.5f * (1.f + erff(f[k] * 0.70710678118654752f)) + f[k] * phi;
+    }
+    store8(du + i * 8, d);
+  }
+}
+
+// [M][S*C] rows <-> S tensors [B, H, N, D]: 16 bytes (8 of D) a thread.
+template <bool TO_HEADS>
+__global__ void __launch_bounds__(256) heads_kernel(__nv_bfloat16* __restrict__ rows, __nv_bfloat16* __restrict__ h0,
+                                                    __nv_bfloat16* __restrict__ h1, __nv_bfloat16* __restrict__ h2,
+                                                    int B, int N, int H, int D, int S) {
+  const int C = H * D;
+  const long long per_row = static_cast<long long>(S) * C / 8;
+  const long long n = static_cast<long long>(B) * N * per_row;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = i / per_row;
+    const int col = static_cast<int>(i - row * per_row) * 8;
+    const int s = col / C, c = col - s * C;
+    const int h = c / D, d = c - h * D;
+    const long long b = row / N, t = row - b * N;
+    __nv_bfloat16* hs = s == 0 ? h0 : (s == 1 ? h1 : h2);
+    uint4* hp = reinterpret_cast<uint4*>(hs + ((b * H + h) * N + t) * D + d);
+    uint4* rp = reinterpret_cast<uint4*>(rows + row * S * C + col);
+    if (TO_HEADS) *hp = *rp;
+    else *rp = *hp;
+  }
+}
+
+// ------------------------------------------------------------------ host side
+int grid_for(long long items, int per_block) {
+  long long b = (items + per_block - 1) / per_block;
+  if (b < 1) b = 1;
+  if (b > 148 * 8) b = 148 * 8;
+  return static_cast<int>(b);
+}
+
+int last_launch() { return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+// One cuBLAS handle per device, created on first use.
+cublasHandle_t handle_for_current_device() {
+  static std::mutex mu;
+  static cublasHandle_t handles[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!handles[dev] && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
+  return handles[dev];
+}
+
+struct Gemm {
+  cublasHandle_t h;
+  // Row-major Out[M][Nn] = A[M][K] W[K][Nn] + beta Out (bf16 out).
+  int mm(const void* A, const void* W, void* Out, int M, int K, int Nn, float beta) const {
+    const float one = 1.f;
+    return cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_N, Nn, M, K, &one, W, CUDA_R_16BF, Nn, A, CUDA_R_16BF, K, &beta,
+                        Out, CUDA_R_16BF, Nn, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS
+               ? SA_OK
+               : SA_ERR_CUDA;
+  }
+  // Row-major Out[M][K] = dOut[M][Nn] W[K][Nn]^T (bf16 out).
+  int mm_nt(const void* dOut, const void* W, void* Out, int M, int K, int Nn) const {
+    const float one = 1.f, zero = 0.f;
+    return cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, K, M, Nn, &one, W, CUDA_R_16BF, Nn, dOut, CUDA_R_16BF, Nn,
+                        &zero, Out, CUDA_R_16BF, K, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS
+               ? SA_OK
+               : SA_ERR_CUDA;
+  }
+  // Row-major dW[K][Nn] = A[M][K]^T dOut[M][Nn] (float32 out).
+  int mm_tn(const void* A, const void* dOut, float* dW, int M, int K, int Nn) const {
+    const float one = 1.f, zero = 0.f;
+    return cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_T, Nn, K, M, &one, dOut, CUDA_R_16BF, Nn, A, CUDA_R_16BF, K,
+                        &zero, dW, CUDA_R_32F, Nn, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS
+               ? SA_OK
+               : SA_ERR_CUDA;
+  }
+};
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Workspace regions (bytes from the start), in units of M*C bf16 elements.
+struct Ws {
+  size_t a, qkv, q, k, v, o, lse, o2, h, f, u, g;               // forward (and recomputation)
+  size_t dg, du, df, dh, do2, dO, dq, dk, dv, dqkv, da, attn;  // backward
+  size_t attn_bytes, total;
+};
+
+Ws layout_ws(int B, int N, int H, int D, const sa_layout* L) {
+  const size_t mc = static_cast<size_t>(B) * N * H * D * 2;  // bytes of one [M][C] bf16 tensor
+  Ws w{};
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = at;
+    at += align256(bytes);
+    return r;
+  };
+  w.a = take(mc);
+  w.qkv = take(3 * mc);
+  w.q = take(mc);
+  w.k = take(mc);
+  w.v = take(mc);
+  w.o = take(mc);
+  w.lse = take(static_cast<size_t>(B) * H * N * 4);
+  w.o2 = take(mc);
+  w.h = take(mc);
+  w.f = take(mc);
+  w.u = take(4 * mc);
+  w.g = take(4 * mc);
+  w.dg = take(4 * mc);
+  w.du = take(4 * mc);
+  w.df = take(mc);
+  w.dh = take(mc);
+  w.do2 = take(mc);
+  w.dO = take(mc);
+  w.dq = take(mc);
+  w.dk = take(mc);
+  w.dv = take(mc);
+  w.dqkv = take(3 * mc);
+  w.da = take(mc);
+  w.attn_bytes = sparse_attn_bwd_workspace_size(B, H, N, D, L);
+  w.attn = take(w.attn_bytes);
+  w.total = at;
+  return w;
+}
+
+int check_args(int B, int N, int H, int D, const sa_layout* L, void* ws, size_t ws_bytes) {
+  if (B < 1 || N < 1 || H < 1 || !L) return SA_ERR_INVALID_ARG;
+  if (D != 32 && D != 64 && D != 128) return SA_ERR_UNSUPPORTED;
+  if (H * D > kMaxC) return SA_ERR_UNSUPPORTED;  // the layer-norm backward's shared sums
+  const Ws w = layout_ws(B, N, H, D, L);
+  if (w.attn_bytes == 0) return SA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SA_ERR_WORKSPACE;
+  return SA_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// The forward chain into the workspace: a, q, k, v, o, lse, o2, h, f, u, g
+// (and y = h + g W2 when y is given).
+int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, int B, int N, int H, int D,
+                  const sa_layout* L, void* ws, cudaStream_t s, const Gemm& G) {
+  const Ws w = layout_ws(B, N, H, D, L);
+  const long long M = static_cast<long long>(B) * N;
+  const int C = H * D;
+  auto* a = at<__nv_bfloat16>(ws, w.a);
+  auto* qkv = at<__nv_bfloat16>(ws, w.qkv);
+  auto* q = at<__nv_bfloat16>(ws, w.q);
+  auto* k = at<__nv_bfloat16>(ws, w.k);
+  auto* v = at<__nv_bfloat16>(ws, w.v);
+  auto* o = at<__nv_bfloat16>(ws, w.o);
+  auto* lse = at<float>(ws, w.lse);
+  auto* o2 = at<__nv_bfloat16>(ws, w.o2);
+  auto* h = at<__nv_bfloat16>(ws, w.h);
+  auto* f = at<__nv_bfloat16>(ws, w.f);
+  auto* u = at<__nv_bfloat16>(ws, w.u);
+  auto* g = at<__nv_bfloat16>(ws, w.g);
+  int st;
+  ln_fwd_kernel<<<grid_for(M * 32, 256), 256, 0, s>>>(x, p->ln1_g, p->ln1_b, a, M, C);
+  if ((st = last_launch())) return st;
+  if ((st = G.mm(a, p->w_qkv, qkv, static_cast<int>(M), C, 3 * C, 0.f))) return st;
+  heads_kernel<true><<<grid_for(M * 3 * C / 8, 256), 256, 0, s>>>(qkv, q, k, v, B, N, H, D, 3);
+  if ((st = last_launch())) return st;
+  if ((st = sparse_attn_fwd(q, k, v, o, lse, B, H, N, D, L, s))) return st;
+  heads_kernel<false><<<grid_for(M * C / 8, 256), 256, 0, s>>>(o2, o, nullptr, nullptr, B, N, H, D, 1);
+  if ((st = last_launch())) return st;
+  if (cudaMemcpyAsync(h, x, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
+  if ((st = G.mm(o2, p->w_o, h, static_cast<int>(M), C, C, 1.f))) return st;
+  ln_fwd_kernel<<<grid_for(M * 32, 256), 256, 0, s>>>(h, p->ln2_g, p->ln2_b, f, M, C);
+  if ((st = last_launch())) return st;
+  if ((st = G.mm(f, p->w_1, u, static_cast<int>(M), C, 4 * C, 0.f))) return st;
+  gelu_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, M * 4 * C / 8);
+  if ((st = last_launch())) return st;
+  if (y) {
+    if (cudaMemcpyAsync(y, h, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
+    if ((st = G.mm(g, p->w_2, y, static_cast<int>(M), 4 * C, C, 1.f))) return st;
+  }
+  return SA_OK;
+}
+
+bool params_ok(const sb_params* p) {
+  return p && p->ln1_g && p->ln1_b && p->w_qkv && p->w_o && p->ln2_g && p->ln2_b && p->w_1 && p->w_2;
+}
+
+}  // namespace sb
+
+using namespace sb;
+
+extern "C" {
+
+size_t sparse_block_workspace_size(int B, int N, int H, int D, const sa_layout* layout) {
+  if (B < 1 || N < 1 || H < 1 || !layout || (D != 32 && D != 64 && D != 128) || H * D > kMaxC) return 0;
+  const Ws w = layout_ws(B, N, H, D, layout);
+  return w.attn_bytes ? w.total : 0;
+}
+
+int sparse_block_fwd(const void* x, const sb_params* p, void* y, int B, int N, int H, int D,
+                     const sa_layout* layout, void* workspace, size_t ws_bytes, void* stream) {
+  if (!x || !y || x == y || !params_ok(p)) return SA_ERR_INVALID_ARG;
+  int st = check_args(B, N, H, D, layout, workspace, ws_bytes);
+  if (st) return st;
+  Gemm G{handle_for_current_device()};
+  if (!G.h) return SA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cublasSetStream(G.h, s) != CUBLAS_STATUS_SUCCESS) return SA_ERR_CUDA;
+  return forward_chain(static_cast<const __nv_bfloat16*>(x), p, static_cast<__nv_bfloat16*>(y), B, N, H, D, layout,
+                       workspace, s, G);
+}
+
+int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx, const sb_grads* gr, int B, int N,
+                     int H, int D, const sa_layout* layout, void* workspace, size_t ws_bytes, void* stream) {
+  if (!x || !dy || !dx || !params_ok(p) || !gr || !gr->ln1_g || !gr->ln1_b || !gr->w_qkv || !gr->w_o ||
+      !gr->ln2_g || !gr->ln2_b || !gr->w_1 || !gr->w_2)
+    return SA_ERR_INVALID_ARG;
+  int st = check_args(B, N, H, D, layout, workspace, ws_bytes);
+  if (st) return st;
+  Gemm G{handle_for_current_device()};
+  if (!G.h) return SA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cublasSetStream(G.h, s) != CUBLAS_STATUS_SUCCESS) return SA_ERR_CUDA;
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* dyb = static_cast<const __nv_bfloat16*>(dy);
+  // the recomputation: every activation again from x
+  if ((st = forward_chain(xb, p, nullptr, B, N, H, D, layout, workspace, s, G))) return st;
+  const Ws w = layout_ws(B, N, H, D, layout);
+  const long long M = static_cast<long long>(B) * N;
+  const int C = H * D, Mi = static_cast<int>(M);
+  void* ws = workspace;
+  auto* a = at<__nv_bfloat16>(ws, w.a);
+  auto* q = at<__nv_bfloat16>(ws, w.q);
+  auto* k = at<__nv_bfloat16>(ws, w.k);
+  auto* v = at<__nv_bfloat16>(ws, w.v);
+  auto* o = at<__nv_bfloat16>(ws, w.o);
+  auto* lse = at<float>(ws, w.lse);
+  auto* o2 = at<__nv_bfloat16>(ws, w.o2);
+  auto* h = at<__nv_bfloat16>(ws, w.h);
+  auto* f = at<__nv_bfloat16>(ws, w.f);
+  auto* u = at<__nv_bfloat16>(ws, w.u);
+  auto* g = at<__nv_bfloat16>(ws, w.g);
+  auto* dg = at<__nv_bfloat16>(ws, w.dg);
+  auto* du = at<__nv_bfloat16>(ws, w.du);
+  auto* df = at<__nv_bfloat16>(ws, w.df);
+  auto* dh = at<__nv_bfloat16>(ws, w.dh);
+  auto* do2 = at<__nv_bfloat16>(ws, w.do2);
+  auto* dO = at<__nv_bfloat16>(ws, w.dO);
+  auto* dq = at<__nv_bfloat16>(ws, w.dq);
+  auto* dk = at<__nv_bfloat16>(ws, w.dk);
+  auto* dv = at<__nv_bfloat16>(ws, w.dv);
+  auto* dqkv = at<__nv_bfloat16>(ws, w.dqkv);
+  auto* da = at<__nv_bfloat16>(ws, w.da);
+  const int ln_grid = grid_for(M * 32, 256);
+  const size_t ln_smem = 2 * C * sizeof(float);
+  // feed-forward: y = h + gelu(f W1) W2
+  if ((st = G.mm_tn(g, dyb, gr->w_2, Mi, 4 * C, C))) return st;
+  if ((st = G.mm_nt(dyb, p->w_2, dg, Mi, 4 * C, C))) return st;
+  gelu_bwd_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, dg, du, M * 4 * C / 8);
+  if ((st = last_launch())) return st;
+  if ((st = G.mm_tn(f, du, gr->w_1, Mi, C, 4 * C))) return st;
+  if ((st = G.mm_nt(du, p->w_1, df, Mi, C, 4 * C))) return st;
+  if (cudaMemsetAsync(gr->ln2_g, 0, C * sizeof(float), s) != cudaSuccess ||
+      cudaMemsetAsync(gr->ln2_b, 0, C * sizeof(float), s) != cudaSuccess)
+    return SA_ERR_CUDA;
+  ln_bwd_kernel<<<ln_grid, 256, ln_smem, s>>>(h, p->ln2_g, df, dyb, dh, gr->ln2_g, gr->ln2_b, M, C);
+  if ((st = last_launch())) return st;
+  // attention: h = x + o Wo
+  if ((st = G.mm_tn(o2, dh, gr->w_o, Mi, C, C))) return st;
+  if ((st = G.mm_nt(dh, p->w_o, do2, Mi, C, C))) return st;
+  heads_kernel<true><<<grid_for(M * C / 8, 256), 256, 0, s>>>(do2, dO, nullptr, nullptr, B, N, H, D, 1);
+  if ((st = last_launch())) return st;
+  if ((st = sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, D, layout, at<void>(ws, w.attn), w.attn_bytes,
+                            s)))
+    return st;
+  heads_kernel<false><<<grid_for(M * 3 * C / 8, 256), 256, 0, s>>>(dqkv, dq, dk, dv, B, N, H, D, 3);
+  if ((st = last_launch())) return st;
+  if ((st = G.mm_tn(a, dqkv, gr->w_qkv, Mi, C, 3 * C))) return st;
+  if ((st = G.mm_nt(dqkv, p->w_qkv, da, Mi, C, 3 * C))) return st;
+  if (cudaMemsetAsync(gr->ln1_g, 0, C * sizeof(float), s) != cudaSuccess ||
+      cudaMemsetAsync(gr->ln1_b, 0, C * sizeof(float), s) != cudaSuccess)
+    return SA_ERR_CUDA;
+  ln_bwd_kernel<<<ln_grid, 256, ln_smem, s>>>(xb, p->ln1_g, da, dh, static_cast<__nv_bfloat16*>(dx), gr->ln1_g,
+                                               gr->ln1_b, M, C);
+  return last_launch();
+}
+
+}  // extern "C"
