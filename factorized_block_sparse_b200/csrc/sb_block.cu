@@ -16,6 +16,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -25,7 +26,7 @@
 namespace sb {
 
 constexpr float kEps = 1e-5f;
-constexpr int kMaxC = 6144;  // model width limit (2 C floats of shared memory per layer-norm block)
+constexpr int kMaxC = 6144;  // model width limit (the layer-norm backward's 4 warps x 2 C float sums, 192 KiB)
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -52,103 +53,219 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float* f) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
-// Mean and 1/sqrt(var + eps) of a C-wide bf16 row, one warp (two passes
-// over the row: the deviations are summed about the mean).
-__device__ __forceinline__ void row_stats(const __nv_bfloat16* xr, int C, int lane, float& mean, float& rstd) {
-  float s = 0.f;
-  for (int i = lane * 8; i < C; i += 256) {
-    float f[8];
-    load8(xr + i, f);
+// A C-wide bf16 row as seen by one lane: chunks of 8 consecutive channels at
+// lane*8 + 256 j.  NCH > 0: the row is held in registers (C <= 256 NCH);
+// NCH == 0: any C, the row is read again for each pass.
+template <int NCH>
+struct Row {
+  float v[NCH > 0 ? NCH * 8 : 1];
+};
+
+template <int NCH>
+__device__ __forceinline__ void row_load(Row<NCH>& r, const __nv_bfloat16* p, int C, int lane) {
+  if constexpr (NCH > 0) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) s += f[u];
+    for (int j = 0; j < NCH; ++j) {
+      const int i = lane * 8 + 256 * j;
+      if (i < C) load8(p + i, r.v + 8 * j);
+      else
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r.v[8 * j + u] = 0.f;
+    }
+  }
+}
+
+// Mean and 1/sqrt(var + eps) of the row (the deviations summed about the mean).
+template <int NCH>
+__device__ __forceinline__ void row_stats(const Row<NCH>& r, const __nv_bfloat16* xr, int C, int lane, float& mean,
+                                          float& rstd) {
+  float s = 0.f;
+  if constexpr (NCH > 0) {
+#pragma unroll
+    for (int k = 0; k < NCH * 8; ++k) s += r.v[k];
+  } else {
+    for (int i = lane * 8; i < C; i += 256) {
+      float f[8];
+      load8(xr + i, f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s += f[u];
+    }
   }
   mean = warp_sum(s) / C;
   float v = 0.f;
-  for (int i = lane * 8; i < C; i += 256) {
-    float f[8];
-    load8(xr + i, f);
+  if constexpr (NCH > 0) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v += (f[u] - mean) * (f[u] - mean);
+    for (int j = 0; j < NCH; ++j)
+      if (lane * 8 + 256 * j < C)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v += (r.v[8 * j + u] - mean) * (r.v[8 * j + u] - mean);
+  } else {
+    for (int i = lane * 8; i < C; i += 256) {
+      float f[8];
+      load8(xr + i, f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v += (f[u] - mean) * (f[u] - mean);
+    }
   }
   rstd = rsqrtf(warp_sum(v) / C + kEps);
 }
 
+// body(i, j, f) for each of the lane's chunks of the row (first channel i,
+// chunk j, the 8 values f), from registers (unrolled) or read again.
+template <int NCH, typename Body>
+__device__ __forceinline__ void for_chunks(const Row<NCH>& r, const __nv_bfloat16* p, int C, int lane, Body body) {
+  if constexpr (NCH > 0) {
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      const int i = lane * 8 + 256 * j;
+      if (i < C) body(i, j, r.v + 8 * j);
+    }
+  } else {
+    for (int i = lane * 8; i < C; i += 256) {
+      float f[8];
+      load8(p + i, f);
+      body(i, 0, f);
+    }
+  }
+}
+
+// The lane's channels of a float32 per-channel parameter, into registers.
+template <int NCH>
+__device__ __forceinline__ void row_load_f32(Row<NCH>& r, const float* p, int C, int lane) {
+  if constexpr (NCH > 0) {
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      const int i = lane * 8 + 256 * j;
+#pragma unroll
+      for (int u = 0; u < 8; u += 4) {
+        const float4 t = i < C ? *reinterpret_cast<const float4*>(p + i + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        r.v[8 * j + u] = t.x;
+        r.v[8 * j + u + 1] = t.y;
+        r.v[8 * j + u + 2] = t.z;
+        r.v[8 * j + u + 3] = t.w;
+      }
+    }
+  }
+}
+
+// Channel i + u (chunk j) of a per-channel parameter: from registers, or memory.
+template <int NCH>
+__device__ __forceinline__ float param(const Row<NCH>& r, const float* p, int i, int j, int u) {
+  if constexpr (NCH > 0) return r.v[8 * j + u];
+  else return p[i + u];
+}
+
 // y = (x - mean) * rstd * g + b per row; one warp per row.
+template <int NCH>
 __global__ void __launch_bounds__(256) ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
                                                      const float* __restrict__ b, __nv_bfloat16* __restrict__ y,
                                                      long long M, int C) {
   const int lane = threadIdx.x & 31;
   const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  // a lane owns the same channels in every row: their gains and biases stay in registers
+  Row<NCH> gv, bv;
+  row_load_f32(gv, g, C, lane);
+  row_load_f32(bv, b, C, lane);
   for (long long r = w0; r < M; r += nw) {
     const __nv_bfloat16* xr = x + r * C;
+    Row<NCH> row;
+    row_load(row, xr, C, lane);
     float mean, rstd;
-    row_stats(xr, C, lane, mean, rstd);
-    for (int i = lane * 8; i < C; i += 256) {
-      float f[8];
-      load8(xr + i, f);
+    row_stats(row, xr, C, lane, mean, rstd);
+    for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
+      float o[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) f[u] = (f[u] - mean) * rstd * g[i + u] + b[i + u];
-      store8(y + r * C + i, f);
-    }
+      for (int u = 0; u < 8; ++u)
+        o[u] = (f[u] - mean) * rstd * param(gv, g, i, j, u) + param(bv, b, i, j, u);
+      store8(y + r * C + i, o);
+    });
   }
 }
 
 // Layer-norm backward with the residual added:
 //   dx = resid + rstd (dxh - mean(dxh) - xh mean(dxh xh)),  dxh = dy g,
 //   dg += sum_rows dy xh,  db += sum_rows dy  (float32, zeroed by the caller).
-// One warp per row; the block sums its rows' dg/db in shared memory and
-// adds them to global memory once.
-__global__ void __launch_bounds__(256) ln_bwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
+// One warp per row.  A lane owns the same channels in every row it visits, so
+// each warp sums dg/db into its own shared-memory slice with plain adds; the
+// block adds its warps' slices to global memory once.
+template <int NCH>
+__global__ void __launch_bounds__(128) ln_bwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
                                                      const __nv_bfloat16* __restrict__ dy,
                                                      const __nv_bfloat16* __restrict__ resid,
                                                      __nv_bfloat16* __restrict__ dx, float* __restrict__ dg,
                                                      float* __restrict__ db, long long M, int C) {
-  extern __shared__ float acc[];  // [2][C]
-  for (int i = threadIdx.x; i < 2 * C; i += blockDim.x) acc[i] = 0.f;
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
+  extern __shared__ float acc[];  // [warps][2][C]
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  float* mine = acc + wid * 2 * C;
+  for (int i = lane; i < 2 * C; i += 32) mine[i] = 0.f;
+  __syncwarp();
+  // the lane's gains in registers; its dg/db sums in registers too when the
+  // row is short (NCH <= 2), else in the warp's shared slice
+  constexpr bool REG_SUMS = NCH > 0 && NCH <= 2;
+  Row<NCH> gv;
+  row_load_f32(gv, g, C, lane);
+  Row<REG_SUMS ? NCH : 0> sg{}, sb{};
   const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   for (long long r = w0; r < M; r += nw) {
     const __nv_bfloat16* xr = x + r * C;
     const __nv_bfloat16* dr = dy + r * C;
+    Row<NCH> row;
+    row_load(row, xr, C, lane);
     float mean, rstd;
-    row_stats(xr, C, lane, mean, rstd);
+    row_stats(row, xr, C, lane, mean, rstd);
     float s1 = 0.f, s2 = 0.f;
-    for (int i = lane * 8; i < C; i += 256) {
-      float f[8], d[8];
-      load8(xr + i, f);
+    for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
+      float d[8];
       load8(dr + i, d);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const float xh = (f[u] - mean) * rstd;
-        const float dxh = d[u] * g[i + u];
+        const float dxh = d[u] * param(gv, g, i, j, u);
         s1 += dxh;
         s2 += dxh * xh;
-        atomicAdd(&acc[i + u], d[u] * xh);
-        atomicAdd(&acc[C + i + u], d[u]);
+        if constexpr (REG_SUMS) {
+          sg.v[8 * j + u] += d[u] * xh;
+          sb.v[8 * j + u] += d[u];
+        } else {
+          mine[i + u] += d[u] * xh;
+          mine[C + i + u] += d[u];
+        }
       }
-    }
+    });
     s1 = warp_sum(s1) / C;
     s2 = warp_sum(s2) / C;
-    for (int i = lane * 8; i < C; i += 256) {
-      float f[8], d[8], o[8];
-      load8(xr + i, f);
+    for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
+      float d[8], o[8];
       load8(dr + i, d);
       load8(resid + r * C + i, o);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const float xh = (f[u] - mean) * rstd;
-        o[u] += rstd * (d[u] * g[i + u] - s1 - xh * s2);
+        o[u] += rstd * (d[u] * param(gv, g, i, j, u) - s1 - xh * s2);
       }
       store8(dx + r * C + i, o);
+    });
+  }
+  if constexpr (REG_SUMS) {
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      const int i = lane * 8 + 256 * j;
+      if (i < C)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          mine[i + u] = sg.v[8 * j + u];
+          mine[C + i + u] = sb.v[8 * j + u];
+        }
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < C; i += blockDim.x) {
-    atomicAdd(&dg[i], acc[i]);
-    atomicAdd(&db[i], acc[C + i]);
+  const int nwb = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < 2 * C; i += blockDim.x) {
+    float t = 0.f;
+    for (int w = 0; w < nwb; ++w) t += acc[w * 2 * C + i];
+    atomicAdd(i < C ? &dg[i] : &db[i - C], t);
   }
 }
 
@@ -215,6 +332,37 @@ int grid_for(long long items, int per_block) {
 }
 
 int last_launch() { return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+// Layer-norm launches: the row in registers up to C = 1024, read again per
+// pass above that.
+int ln_fwd(const __nv_bfloat16* x, const float* g, const float* b, __nv_bfloat16* y, long long M, int C,
+           cudaStream_t s) {
+  const int grid = grid_for(M * 32, 256);
+  if (C <= 256) ln_fwd_kernel<1><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
+  else if (C <= 512) ln_fwd_kernel<2><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
+  else if (C <= 1024) ln_fwd_kernel<4><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
+  else ln_fwd_kernel<0><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
+  return last_launch();
+}
+
+int ln_bwd(const __nv_bfloat16* x, const float* g, const __nv_bfloat16* dy, const __nv_bfloat16* resid,
+           __nv_bfloat16* dx, float* dg, float* db, long long M, int C, cudaStream_t s) {
+  constexpr int kThreads = 128;  // 4 warps, each with its own dg/db slice
+  const size_t smem = 4 * 2 * static_cast<size_t>(C) * sizeof(float);
+  const int grid = static_cast<int>(std::min<long long>((M + 3) / 4, 148 * 4));
+  auto go = [&](auto kernel) -> int {
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+      return SA_ERR_CUDA;
+    kernel<<<grid, kThreads, smem, s>>>(x, g, dy, resid, dx, dg, db, M, C);
+    return last_launch();
+  };
+  if (C <= 256) return go(ln_bwd_kernel<1>);
+  if (C <= 512) return go(ln_bwd_kernel<2>);
+  if (C <= 1024) return go(ln_bwd_kernel<4>);
+  return go(ln_bwd_kernel<0>);
+}
 
 // One cuBLAS handle per device, created on first use.
 cublasHandle_t handle_for_current_device() {
@@ -337,8 +485,7 @@ int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, 
   auto* u = at<__nv_bfloat16>(ws, w.u);
   auto* g = at<__nv_bfloat16>(ws, w.g);
   int st;
-  ln_fwd_kernel<<<grid_for(M * 32, 256), 256, 0, s>>>(x, p->ln1_g, p->ln1_b, a, M, C);
-  if ((st = last_launch())) return st;
+  if ((st = ln_fwd(x, p->ln1_g, p->ln1_b, a, M, C, s))) return st;
   if ((st = G.mm(a, p->w_qkv, qkv, static_cast<int>(M), C, 3 * C, 0.f))) return st;
   heads_kernel<true><<<grid_for(M * 3 * C / 8, 256), 256, 0, s>>>(qkv, q, k, v, B, N, H, D, 3);
   if ((st = last_launch())) return st;
@@ -347,8 +494,7 @@ int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, 
   if ((st = last_launch())) return st;
   if (cudaMemcpyAsync(h, x, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
   if ((st = G.mm(o2, p->w_o, h, static_cast<int>(M), C, C, 1.f))) return st;
-  ln_fwd_kernel<<<grid_for(M * 32, 256), 256, 0, s>>>(h, p->ln2_g, p->ln2_b, f, M, C);
-  if ((st = last_launch())) return st;
+  if ((st = ln_fwd(h, p->ln2_g, p->ln2_b, f, M, C, s))) return st;
   if ((st = G.mm(f, p->w_1, u, static_cast<int>(M), C, 4 * C, 0.f))) return st;
   gelu_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, M * 4 * C / 8);
   if ((st = last_launch())) return st;
@@ -429,8 +575,6 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   auto* dv = at<__nv_bfloat16>(ws, w.dv);
   auto* dqkv = at<__nv_bfloat16>(ws, w.dqkv);
   auto* da = at<__nv_bfloat16>(ws, w.da);
-  const int ln_grid = grid_for(M * 32, 256);
-  const size_t ln_smem = 2 * C * sizeof(float);
   // feed-forward: y = h + gelu(f W1) W2
   if ((st = G.mm_tn(g, dyb, gr->w_2, Mi, 4 * C, C))) return st;
   if ((st = G.mm_nt(dyb, p->w_2, dg, Mi, 4 * C, C))) return st;
@@ -441,8 +585,7 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   if (cudaMemsetAsync(gr->ln2_g, 0, C * sizeof(float), s) != cudaSuccess ||
       cudaMemsetAsync(gr->ln2_b, 0, C * sizeof(float), s) != cudaSuccess)
     return SA_ERR_CUDA;
-  ln_bwd_kernel<<<ln_grid, 256, ln_smem, s>>>(h, p->ln2_g, df, dyb, dh, gr->ln2_g, gr->ln2_b, M, C);
-  if ((st = last_launch())) return st;
+  if ((st = ln_bwd(h, p->ln2_g, df, dyb, dh, gr->ln2_g, gr->ln2_b, M, C, s))) return st;
   // attention: h = x + o Wo
   if ((st = G.mm_tn(o2, dh, gr->w_o, Mi, C, C))) return st;
   if ((st = G.mm_nt(dh, p->w_o, do2, Mi, C, C))) return st;
@@ -458,9 +601,7 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   if (cudaMemsetAsync(gr->ln1_g, 0, C * sizeof(float), s) != cudaSuccess ||
       cudaMemsetAsync(gr->ln1_b, 0, C * sizeof(float), s) != cudaSuccess)
     return SA_ERR_CUDA;
-  ln_bwd_kernel<<<ln_grid, 256, ln_smem, s>>>(xb, p->ln1_g, da, dh, static_cast<__nv_bfloat16*>(dx), gr->ln1_g,
-                                               gr->ln1_b, M, C);
-  return last_launch();
+  return ln_bwd(xb, p->ln1_g, da, dh, static_cast<__nv_bfloat16*>(dx), gr->ln1_g, gr->ln1_b, M, C, s);
 }
 
 }  // extern "C"
