@@ -772,6 +772,8 @@ def source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "factorized_block_sparse_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
+        if not fn.startswith("sa_"):  # the attention library's sources (not the block around it)
+            continue
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]
