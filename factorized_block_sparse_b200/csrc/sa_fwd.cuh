@@ -424,18 +424,28 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
           tmem_wait_st();
         }
         const float neg = (m_used == -INFINITY) ? 0.f : -m_used;
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // partial row sums
+        uint64_t rs2[4] = {0, 0, 0, 0};  // partial row sums, fp32 pairs
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), ng2 = f2_pack(neg, neg);
         uint32_t pk[C::TK / 2];
 #pragma unroll
         for (int ch = 0; ch < C::TK / 8; ++ch) {
           float p[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            p[u] = ex2(fmaf(s[ch * 8 + u], a.scale_log2, neg));
-            rs8[u] += p[u];
+          for (int u = 0; u < 8; u += 2) {
+            const float2 t = f2_unpack(f2_fma(f2_pack(s[ch * 8 + u], s[ch * 8 + u + 1]), sc2, ng2));
+            p[u] = ex2(t.x);
+            p[u + 1] = ex2(t.y);
+            rs2[u / 2] = f2_add(rs2[u / 2], f2_pack(p[u], p[u + 1]));
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) pk[ch * 4 + u] = pack_bf16(p[2 * u], p[2 * u + 1]);
+        }
+        float rs8[8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 t = f2_unpack(rs2[u]);
+          rs8[2 * u] = t.x;
+          rs8[2 * u + 1] = t.y;
         }
         // P over the first TK/2 columns of its own S buffer (the S values are in registers)
         tmem_st32(tmem + lane_base + sb * C::TK, pk);
