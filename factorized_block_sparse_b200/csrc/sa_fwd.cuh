@@ -35,6 +35,12 @@
 
 namespace sa {
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 struct FwdArgs {
   const int32_t* row_ptr;
   const int32_t* ent;
@@ -391,16 +397,14 @@ __global__ void __launch_bounds__(224, (D <= 64) ? 2 : 1)
             mask_interval64(s, lo - k0, hi - k0, -INFINITY);
           }
         }
-        // row max as a tree (short dependency chains)
-        float mx8[8];
+        // row max as a tree of three-input maxima (short dependency chains)
+        float m21[21];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = s[u];
+        for (int u = 0; u < 21; ++u) m21[u] = max3f(s[3 * u], s[3 * u + 1], s[3 * u + 2]);
+        float m7[7];
 #pragma unroll
-        for (int i = 8; i < C::TK; i += 8)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], s[i + u]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int u = 0; u < 7; ++u) m7[u] = max3f(m21[3 * u], m21[3 * u + 1], m21[3 * u + 2]);
+        const float mx = max3f(max3f(m7[0], m7[1], m7[2]), max3f(m7[3], m7[4], m7[5]), fmaxf(m7[6], s[63]));
         const float m_tile = mx * a.scale_log2;
         float factor = 1.f;
         if (m_tile > m_used + 8.f) {
