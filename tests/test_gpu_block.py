@@ -65,6 +65,13 @@ def _run(mode, B, N, H, D, l, c, block, device):
     ("strided", 2, 256, 4, 32, 16, 0, 16),    # tiny-like pattern, C = 128
     ("all", 1, 256, 2, 128, 1, 0, 64),        # D = 128, C = 256
     ("strided", 1, 384, 3, 64, 48, 0, 16),    # C = 192 (not a multiple of 256), R = 8
+    # the layer norms' widths: rows in registers with per-lane dg/db sums (C = 512),
+    # rows in registers with shared sums (C = 1024), rows read per pass (C = 1536),
+    # and shared sums above the default 48 KiB of dynamic shared memory (C = 2048)
+    ("fixed", 1, 256, 8, 64, 128, 32, 64),
+    ("local", 1, 256, 8, 128, 64, 0, 64),
+    ("all", 1, 128, 12, 128, 1, 0, 64),
+    ("all", 1, 128, 16, 128, 1, 0, 64),
 ])
 def test_block_parity(cuda_device, mode, B, N, H, D, l, c, block):
     got, ref = _run(mode, B, N, H, D, l, c, block, cuda_device)
