@@ -269,57 +269,64 @@ __global__ void __launch_bounds__(128) ln_bwd_kernel(const __nv_bfloat16* __rest
   }
 }
 
-// gelu(u) = u Phi(u) = u (1 + erf(u / sqrt 2)) / 2, 8 elements a thread.
+// gelu(u) = u Phi(u) = u (1 + erf(u / sqrt 2)) / 2, 8 elements a thread;
+// with GRAD also its derivative Phi(u) + u phi(u) (phi the standard normal
+// density), for the backward pass's recomputation.
+template <bool GRAD>
 __global__ void __launch_bounds__(256) gelu_kernel(const __nv_bfloat16* __restrict__ u, __nv_bfloat16* __restrict__ out,
-                                                   long long n8) {
+                                                   __nv_bfloat16* __restrict__ grad, long long n8) {
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    float f[8];
+    float f[8], o[8], gd[8];
     load8(u + i * 8, f);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) f[k] = 0.5f * f[k] * (1.f + erff(f[k] * 0.70710678118654752f));
-    store8(out + i * 8, f);
-  }
-}
-
-// du = dg (Phi(u) + u phi(u)), phi the standard normal density.
-__global__ void __launch_bounds__(256) gelu_bwd_kernel(const __nv_bfloat16* __restrict__ u,
-                                                       const __nv_bfloat16* __restrict__ dg,
-                                                       __nv_bfloat16* __restrict__ du, long long n8) {
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    float f[8], d[8];
-    load8(u + i * 8, f);
-    load8(dg + i * 8, d);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float phi = 0.3989422804014327f * expf(-0.5f * f[k] * f[k]);
-      d[k] *= 0.5f * (1.f + erff(f[k] * 0.70710678118654752f)) + f[k] * phi;
+      const float cdf = 0.5f * (1.f + erff(f[k] * 0.70710678118654752f));
+      o[k] = f[k] * cdf;
+      if (GRAD) gd[k] = cdf + f[k] * 0.3989422804014327f * expf(-0.5f * f[k] * f[k]);
     }
-    store8(du + i * 8, d);
+    store8(out + i * 8, o);
+    if (GRAD) store8(grad + i * 8, gd);
   }
 }
 
-// [M][S*C] rows <-> S tensors [B, H, N, D]: 16 bytes (8 of D) a thread.
+// a *= b elementwise (bf16, 8 elements a thread): du = dg gelu'(u).
+__global__ void __launch_bounds__(256) mul_kernel(__nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                                                  long long n8) {
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float x[8], y[8];
+    load8(a + i * 8, x);
+    load8(b + i * 8, y);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] *= y[k];
+    store8(a + i * 8, x);
+  }
+}
+
+// [M][S*C] rows <-> S tensors [B, H, N, D], 16 bytes (8 of D) a thread: a
+// thread keeps its place in the row (tensor s, head h, d) for every row the
+// block visits.
 template <bool TO_HEADS>
 __global__ void __launch_bounds__(256) heads_kernel(__nv_bfloat16* __restrict__ rows, __nv_bfloat16* __restrict__ h0,
                                                     __nv_bfloat16* __restrict__ h1, __nv_bfloat16* __restrict__ h2,
                                                     int B, int N, int H, int D, int S) {
   const int C = H * D;
-  const long long per_row = static_cast<long long>(S) * C / 8;
-  const long long n = static_cast<long long>(B) * N * per_row;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = i / per_row;
-    const int col = static_cast<int>(i - row * per_row) * 8;
+  const int per_row = S * C / 8;
+  const long long M = static_cast<long long>(B) * N;
+  for (int v = threadIdx.x; v < per_row; v += blockDim.x) {
+    const int col = v * 8;
     const int s = col / C, c = col - s * C;
     const int h = c / D, d = c - h * D;
-    const long long b = row / N, t = row - b * N;
     __nv_bfloat16* hs = s == 0 ? h0 : (s == 1 ? h1 : h2);
-    uint4* hp = reinterpret_cast<uint4*>(hs + ((b * H + h) * N + t) * D + d);
-    uint4* rp = reinterpret_cast<uint4*>(rows + row * S * C + col);
-    if (TO_HEADS) *hp = *rp;
-    else *rp = *hp;
+    hs += static_cast<long long>(h) * N * D + d;
+    for (long long row = blockIdx.x; row < M; row += gridDim.x) {
+      const long long b = row / N, t = row - b * N;
+      uint4* hp = reinterpret_cast<uint4*>(hs + (b * H * N + t) * D);
+      uint4* rp = reinterpret_cast<uint4*>(rows + row * S * C + col);
+      if (TO_HEADS) *hp = *rp;
+      else *rp = *hp;
+    }
   }
 }
 
@@ -332,6 +339,10 @@ int grid_for(long long items, int per_block) {
 }
 
 int last_launch() { return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+// heads_kernel: a block per row (grid-stride), a thread per 16 bytes of it.
+int heads_grid(long long M) { return static_cast<int>(std::min<long long>(M, 148 * 16)); }
+int heads_block(int width) { return std::min(256, std::max(32, (width / 8 + 31) / 32 * 32)); }
 
 // Layer-norm launches: the row in registers up to C = 1024, read again per
 // pass above that.
@@ -466,9 +477,9 @@ T* at(void* ws, size_t off) {
 }
 
 // The forward chain into the workspace: a, q, k, v, o, lse, o2, h, f, u, g
-// (and y = h + g W2 when y is given).
+// (and y = h + g W2 when y is given; gelu'(u) into gelu_grad when given).
 int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, int B, int N, int H, int D,
-                  const sa_layout* L, void* ws, cudaStream_t s, const Gemm& G) {
+                  const sa_layout* L, void* ws, cudaStream_t s, const Gemm& G, __nv_bfloat16* gelu_grad = nullptr) {
   const Ws w = layout_ws(B, N, H, D, L);
   const long long M = static_cast<long long>(B) * N;
   const int C = H * D;
@@ -487,16 +498,17 @@ int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, 
   int st;
   if ((st = ln_fwd(x, p->ln1_g, p->ln1_b, a, M, C, s))) return st;
   if ((st = G.mm(a, p->w_qkv, qkv, static_cast<int>(M), C, 3 * C, 0.f))) return st;
-  heads_kernel<true><<<grid_for(M * 3 * C / 8, 256), 256, 0, s>>>(qkv, q, k, v, B, N, H, D, 3);
+  heads_kernel<true><<<heads_grid(M), heads_block(3 * C), 0, s>>>(qkv, q, k, v, B, N, H, D, 3);
   if ((st = last_launch())) return st;
   if ((st = sparse_attn_fwd(q, k, v, o, lse, B, H, N, D, L, s))) return st;
-  heads_kernel<false><<<grid_for(M * C / 8, 256), 256, 0, s>>>(o2, o, nullptr, nullptr, B, N, H, D, 1);
+  heads_kernel<false><<<heads_grid(M), heads_block(C), 0, s>>>(o2, o, nullptr, nullptr, B, N, H, D, 1);
   if ((st = last_launch())) return st;
   if (cudaMemcpyAsync(h, x, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
   if ((st = G.mm(o2, p->w_o, h, static_cast<int>(M), C, C, 1.f))) return st;
   if ((st = ln_fwd(h, p->ln2_g, p->ln2_b, f, M, C, s))) return st;
   if ((st = G.mm(f, p->w_1, u, static_cast<int>(M), C, 4 * C, 0.f))) return st;
-  gelu_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, M * 4 * C / 8);
+  if (gelu_grad) gelu_kernel<true><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, gelu_grad, M * 4 * C / 8);
+  else gelu_kernel<false><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, nullptr, M * 4 * C / 8);
   if ((st = last_launch())) return st;
   if (y) {
     if (cudaMemcpyAsync(y, h, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
@@ -548,8 +560,9 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
   const auto* dyb = static_cast<const __nv_bfloat16*>(dy);
   // the recomputation: every activation again from x
-  if ((st = forward_chain(xb, p, nullptr, B, N, H, D, layout, workspace, s, G))) return st;
   const Ws w = layout_ws(B, N, H, D, layout);
+  if ((st = forward_chain(xb, p, nullptr, B, N, H, D, layout, workspace, s, G, at<__nv_bfloat16>(workspace, w.du))))
+    return st;
   const long long M = static_cast<long long>(B) * N;
   const int C = H * D, Mi = static_cast<int>(M);
   void* ws = workspace;
@@ -562,7 +575,6 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   auto* o2 = at<__nv_bfloat16>(ws, w.o2);
   auto* h = at<__nv_bfloat16>(ws, w.h);
   auto* f = at<__nv_bfloat16>(ws, w.f);
-  auto* u = at<__nv_bfloat16>(ws, w.u);
   auto* g = at<__nv_bfloat16>(ws, w.g);
   auto* dg = at<__nv_bfloat16>(ws, w.dg);
   auto* du = at<__nv_bfloat16>(ws, w.du);
@@ -578,7 +590,7 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   // feed-forward: y = h + gelu(f W1) W2
   if ((st = G.mm_tn(g, dyb, gr->w_2, Mi, 4 * C, C))) return st;
   if ((st = G.mm_nt(dyb, p->w_2, dg, Mi, 4 * C, C))) return st;
-  gelu_bwd_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, dg, du, M * 4 * C / 8);
+  mul_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(du, dg, M * 4 * C / 8);  // du held gelu'(u)
   if ((st = last_launch())) return st;
   if ((st = G.mm_tn(f, du, gr->w_1, Mi, C, 4 * C))) return st;
   if ((st = G.mm_nt(du, p->w_1, df, Mi, C, 4 * C))) return st;
@@ -589,12 +601,12 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   // attention: h = x + o Wo
   if ((st = G.mm_tn(o2, dh, gr->w_o, Mi, C, C))) return st;
   if ((st = G.mm_nt(dh, p->w_o, do2, Mi, C, C))) return st;
-  heads_kernel<true><<<grid_for(M * C / 8, 256), 256, 0, s>>>(do2, dO, nullptr, nullptr, B, N, H, D, 1);
+  heads_kernel<true><<<heads_grid(M), heads_block(C), 0, s>>>(do2, dO, nullptr, nullptr, B, N, H, D, 1);
   if ((st = last_launch())) return st;
   if ((st = sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, D, layout, at<void>(ws, w.attn), w.attn_bytes,
                             s)))
     return st;
-  heads_kernel<false><<<grid_for(M * 3 * C / 8, 256), 256, 0, s>>>(dqkv, dq, dk, dv, B, N, H, D, 3);
+  heads_kernel<false><<<heads_grid(M), heads_block(3 * C), 0, s>>>(dqkv, dq, dk, dv, B, N, H, D, 3);
   if ((st = last_launch())) return st;
   if ((st = G.mm_tn(a, dqkv, gr->w_qkv, Mi, C, 3 * C))) return st;
   if ((st = G.mm_nt(dqkv, p->w_qkv, da, Mi, C, 3 * C))) return st;

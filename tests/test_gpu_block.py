@@ -5,8 +5,8 @@ Tolerance.  The block's activations are bf16: on the way to y about ten
 intermediates are rounded to bf16 (a, q/k/v, the attention output, h, f, u,
 gelu(u), y and the attention's own rounding), each by at most 2^-9 of its
 magnitude, and the gradients pass through about twice as many (the
-recomputed forward, then dg, du, df, dh, do, the attention backward, dqkv,
-da, dx); the GEMMs accumulate in float32.  Hence the bounds: relative L2
+recomputed forward, then dg, gelu'(u), du, df, dh, do, the attention
+backward, dqkv, da, dx); the GEMMs accumulate in float32.  Hence the bounds: relative L2
 error at most 1e-2 (about sqrt(20) * 2^-9 with room), and every element
 within 5e-2 of the largest magnitude of its reference (about 20 * 2^-9),
 for y, dx and each parameter gradient.
