@@ -29,10 +29,13 @@ namespace sa {
 namespace {
 
 // ------------------------------------------------------------ instrumentation
-enum Kind { K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_FINAL, K_FWD_TAIL, K_BWD_TAIL, K_KERNELS };
+enum Kind {
+  K_FWD_COL = 0, K_FWD_MAIN, K_BWD_PRE, K_BWD_SEC, K_BWD_MAIN, K_BWD_FINAL, K_FWD_TAIL, K_BWD_TAIL, K_BWD_SUMFIN,
+  K_KERNELS
+};
 const char* const kKernelNames[K_KERNELS] = {"sa_fwd_column_view",  "sa_fwd_natural_view", "sa_bwd_preprocess",
                                              "sa_bwd_secondary_view", "sa_bwd_natural_view", "sa_bwd_finalize_dq",
-                                             "sa_fwd_partial_row",  "sa_bwd_partial_row"};
+                                             "sa_fwd_partial_row",  "sa_bwd_partial_row",  "sa_bwd_finalize_summary_dkv"};
 constexpr int K_PATTERNS = 7;
 const char* const kPatternNames[K_PATTERNS] = {"all", "local", "strided", "fixed", "column", "block", "blocks"};
 // Instrumentation kinds: one per (kernel, pattern), kind = kernel * K_PATTERNS + pattern.
@@ -619,6 +622,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   if ((st = set_bwd_smem<D, false>())) return st;
   if constexpr (D <= 64) {
     if ((st = set_bwd_smem<D, true>())) return st;
+    // the fixed pattern's natural pass with the summary keys' rows reduced into the partials
+    if ((st = set_smem(sa_bwd_kernel<D, false, false, false, kDqReduce, true>, BwdCfg<D, false>::SMEM))) return st;
+    if ((st = set_smem(sa_bwd_kernel<D, false, false, false, kDqFinal, true>, BwdCfg<D, false>::SMEM))) return st;
   }
   const WsLayout w = ws_layout(B, H, N, D, L);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -676,6 +682,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
   a.BH = g.BH;
   const int n_sm = sm_count();
   // Tables whose items average many steps take the LONG shape of the kernel.
+  bool summary_reduced = false;  // the natural pass reduced the summary keys' rows into the partials
   auto run = [&](int kind, const DevTable& t, int dqm) -> int {
     EpiMaps em;
     const int mst = make_epi_maps(&em, dk, dv, dk_part, dv_part, g, a.key_view);
@@ -685,6 +692,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     const bool long_items = D <= 64 && t.nnz >= kBwdLongSteps * static_cast<long long>(t.n_rows);
     const bool final_t = sec_final && a.key_view == SRC_T;
     const bool blk = a.blk > 0;  // caller block mask with blocks below a tile (natural view only)
+    const bool sum_red = D <= 64 && !long_items && a.add_part == 2 && !blk && dqm != kDqStore;
     auto go = [&](auto kernel, int threads, int smem) {
       launch_kernel(kernel, grid, threads, smem, s, mq.nat, mq.col, mdo.nat, mdo.col, mk.nat, mk.col, mk.sum, mv.nat,
                     mv.col, mv.sum, mdq_nat, mdq_col, em.out_k, em.out_v, em.part_k, em.part_v, a);
@@ -707,8 +715,15 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
         go(sa_bwd_kernel<D, L, false, false, kDqReduce>, CF::THREADS, CF::SMEM);
       }
     };
+    if (sum_red) summary_reduced = true;
     return launch(kind, s, [&] {
       if constexpr (D <= 64) {
+        if (sum_red) {
+          using CS = BwdCfg<D, false>;
+          if (dqm == kDqFinal) go(sa_bwd_kernel<D, false, false, false, kDqFinal, true>, CS::THREADS, CS::SMEM);
+          else go(sa_bwd_kernel<D, false, false, false, kDqReduce, true>, CS::THREADS, CS::SMEM);
+          return;
+        }
         if (long_items) {
           pick(std::true_type{});
           return;
@@ -745,6 +760,15 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const f
     a.key_view = SRC_N;
     a.add_part = (sec && !sec_final) ? (L->pattern == SA_STRIDED ? 1 : 2) : 0;
     if ((st = run(K_BWD_MAIN * K_PATTERNS + L->pattern, dc.bwd_main, dq_fin ? kDqFinal : kDqReduce))) return st;
+  }
+  if (summary_reduced && g.R > 0) {  // the summary keys' dK, dV: their fp32 sums rounded to bf16
+    const long long n = static_cast<long long>(g.BH) * g.R * g.c * (D / 8);
+    st = launch(K_BWD_SUMFIN * K_PATTERNS + L->pattern, s, [&] {
+      launch_kernel(sa_bwd_summary_final_kernel<D>, grid_for(n, 256), 256, 0, s, static_cast<const float*>(dk_part),
+                    static_cast<const float*>(dv_part), static_cast<__nv_bfloat16*>(dk),
+                    static_cast<__nv_bfloat16*>(dv), g.BH, N, g.l, g.c, g.R);
+    });
+    if (st) return st;
   }
   if (dq_fin) return SA_OK;
   const long long n8 = rows * D / 8;

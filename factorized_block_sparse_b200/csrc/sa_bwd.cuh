@@ -255,7 +255,11 @@ __device__ __forceinline__ void store_grad_row(const BwdArgs& a, int which, size
 // BLK: a caller block mask whose blocks are smaller than a tile (the
 // entries' sub-block bits are applied on PARTIAL steps).
 // DQM: the DqMode of the pass.
-template <int D, bool LONG, bool FINAL_T, bool BLK = false, int DQM = kDqReduce>
+// SUM_RED: the natural pass of the fixed pattern adds its dK/dV rows of the
+// summary keys to the summary view's fp32 partials by TMA reduce-add (and a
+// later launch rounds them to bf16) instead of loading the partials and
+// storing the sum itself.
+template <int D, bool LONG, bool FINAL_T, bool BLK = false, int DQM = kDqReduce, bool SUM_RED = false>
 __global__ void __launch_bounds__(480, 1)
     sa_bwd_kernel(const __grid_constant__ CUtensorMap mq_nat, const __grid_constant__ CUtensorMap mq_col,
                   const __grid_constant__ CUtensorMap mdo_nat, const __grid_constant__ CUtensorMap mdo_col,
@@ -883,6 +887,58 @@ __global__ void __launch_bounds__(480, 1)
         if (nat_out && a.add_part == 1) row_add = kr.kvalid && kr.knat < a.R * a.l;  // keys of whole rows
         else if (nat_out && a.add_part == 2) row_add = kr.kvalid && (kr.knat % a.l) >= (a.l - a.c) && kr.knat < a.R * a.l;
         const bool warp_add = __any_sync(0xffffffffu, row_add);
+        if (SUM_RED && warp_add) {
+          // Rows of summary keys: their fp32 rows go to the partials by TMA
+          // reduce-add (the other rows of the warp are added there too, at
+          // positions nothing reads); the warp's rows of other keys are
+          // stored as final bf16 rows directly.
+          const size_t roff = (static_cast<size_t>(it.bh) * a.N + (kr.kvalid ? kr.knat : 0)) * D;
+#pragma unroll 1
+          for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+            if (lane == 0) bulk_wait_read_all();  // earlier stores and reduces have read the staging
+            __syncwarp();
+            const uint32_t col = (which ? C::COL_DK : C::COL_DV) + (ne % C::DKVB) * 2 * D;
+            const float mul = which ? a.scale : 1.f;
+#pragma unroll
+            for (int h = 0; h < D / 32; ++h) {
+              float gv[32];
+              if (it.n > 0) {
+                tmem_ld16(tmem + lane_base + col + h * 32, gv);
+                tmem_ld16(tmem + lane_base + col + h * 32 + 16, gv + 16);
+                tmem_wait_ld();
+                if (which == 1 && h == D / 32 - 1) {
+                  tc_fence_before();
+                  mbar_arrive(bar_dkv_free + ne % C::DKVB);  // both accumulators have been read
+                }
+              } else {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) gv[u] = 0.f;
+              }
+#pragma unroll
+              for (int u = 0; u < 32; ++u) gv[u] *= mul;
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<float4*>(stg + h * 4096 + sw128_offset(lane, ch)) =
+                    make_float4(gv[ch * 4], gv[ch * 4 + 1], gv[ch * 4 + 2], gv[ch * 4 + 3]);
+              if (!row_add && kr.kvalid) {
+                uint4* dstp = reinterpret_cast<uint4*>((which ? a.dk : a.dv) + roff + h * 32);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                  dstp[c4] = make_uint4(pack_bf16(gv[8 * c4], gv[8 * c4 + 1]), pack_bf16(gv[8 * c4 + 2], gv[8 * c4 + 3]),
+                                        pack_bf16(gv[8 * c4 + 4], gv[8 * c4 + 5]),
+                                        pack_bf16(gv[8 * c4 + 6], gv[8 * c4 + 7]));
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+#pragma unroll
+              for (int bx = 0; bx < D / 32; ++bx)
+                tma_reduce_add_3d(which ? &mdk_part : &mdv_part, stg + bx * 4096, bx * 32, y0, it.bh);
+              bulk_commit_group();
+            }
+          }
+        } else {
 #pragma unroll 1
         for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
           if (lane == 0) bulk_wait_read_all();  // earlier stores and reduces have read the staging
@@ -981,6 +1037,7 @@ __global__ void __launch_bounds__(480, 1)
             }
             bulk_commit_group();
           }
+        }
         }
         if (it.n > 0) ++ne;
       } else {
@@ -1108,6 +1165,37 @@ __global__ void __launch_bounds__(256) sa_bwd_pre_kernel(const __nv_bfloat16* __
       const long long o = bh * n_pad * 2 + (i / 64) * 128 + (i % 64);
       ld_col[o] = -INFINITY;
       ld_col[o + 64] = 0.f;
+    }
+  }
+}
+
+// dK, dV (bf16) of the fixed pattern's summary keys = their fp32 partials
+// (summary view + the natural view's reduce-adds): positions p with
+// p mod l >= l - c of the R whole blocks, 8 channels a thread.
+template <int D>
+__global__ void __launch_bounds__(256) sa_bwd_summary_final_kernel(const float* __restrict__ dk_part,
+                                                                   const float* __restrict__ dv_part,
+                                                                   __nv_bfloat16* __restrict__ dk,
+                                                                   __nv_bfloat16* __restrict__ dv, int BH, int N,
+                                                                   int l, int c, int R) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int V = D / 8;  // 8-channel vectors per row
+  const long long n = static_cast<long long>(BH) * R * c * V;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long key = i / V;
+    const int v = static_cast<int>(i - key * V);
+    const long long bh = key / (static_cast<long long>(R) * c);
+    const int sk = static_cast<int>(key - bh * R * c);  // summary key of the head
+    const int p = (sk / c) * l + (l - c) + sk % c;
+    const size_t off = (static_cast<size_t>(bh) * N + p) * D + v * 8;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const float4* src = reinterpret_cast<const float4*>((which ? dk_part : dv_part) + off);
+      const float4 a0 = src[0], a1 = src[1];
+      *reinterpret_cast<uint4*>((which ? dk : dv) + off) =
+          make_uint4(pack_bf16(a0.x, a0.y), pack_bf16(a0.z, a0.w), pack_bf16(a1.x, a1.y), pack_bf16(a1.z, a1.w));
     }
   }
 }

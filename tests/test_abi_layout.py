@@ -99,7 +99,7 @@ def test_argument_errors(sa):
         assert sa.lib.sparse_attn_bwd(*([fake] * 9), 1, 1, N, 32, odd.handle, fake, 1 << 30, None) \
             == sa.SA_ERR_UNSUPPORTED, mode
     assert sa.strerror(sa.SA_ERR_TIMEOUT) == "device-side wait timed out"
-    assert sa.lib.sparse_attn_kernel_kinds() == 56  # 8 kernels x 7 patterns
+    assert sa.lib.sparse_attn_kernel_kinds() == 63  # 9 kernels x 7 patterns
 
 
 def _compare(sa, mode, N, l, c, b, rows=None):

@@ -263,16 +263,18 @@ def test_parity_block_diagonal_mask(cuda_device, B, H, N, D, b):
         assert_close(f"diagonal blocks N={N} D={D} b={b} {name}", got[name], ref[name])
 
 
-@pytest.mark.parametrize("mode,N,l,c,finalise", [
-    ("fixed", 2048, 128, 32, 0),   # own block = one 128-key tile per 64-query step
-    ("block", 960, 64, 0, 0),
-    ("fixed", 2048, 256, 32, 1),   # a step of the second half of a block meets two key tiles
-    ("strided", 2048, 64, 0, 1),
-    ("column", 2048, 64, 0, 1),    # no natural view
+@pytest.mark.parametrize("mode,N,l,c,finalise,summary", [
+    ("fixed", 2048, 128, 32, 0, 1),   # own block = one 128-key tile per 64-query step
+    ("block", 960, 64, 0, 0, 0),
+    ("fixed", 2048, 256, 32, 1, 0),   # a step of the second half of a block meets two key tiles;
+                                      # its natural items run the LONG shape, which adds the partials itself
+    ("strided", 2048, 64, 0, 1, 0),
+    ("column", 2048, 64, 0, 1, 0),    # no natural view
 ])
-def test_final_dq_pass(cuda_device, mode, N, l, c, finalise):
+def test_final_dq_pass(cuda_device, mode, N, l, c, finalise, summary):
     """The separate dQ finalise runs only where the natural view's pass cannot
-    complete each dQ row with one product."""
+    complete each dQ row with one product; the summary keys' dK/dV finalise
+    only where the natural pass reduced their rows into the partials."""
     from factorized_block_sparse_b200 import sparse_attn as sa
 
     sa.timing_reset()
@@ -281,7 +283,9 @@ def test_final_dq_pass(cuda_device, mode, N, l, c, finalise):
         run_library(mode, 1, 1, N, 64, l, c, 64)
     finally:
         sa.timing_enable(False)
-    assert sa.kernel_times()[f"sa_bwd_finalize_dq.{mode}"][1] == finalise
+    kt = sa.kernel_times()
+    assert kt[f"sa_bwd_finalize_dq.{mode}"][1] == finalise
+    assert kt[f"sa_bwd_finalize_summary_dkv.{mode}"][1] == summary
     sa.timing_reset()
 
 
