@@ -266,8 +266,9 @@ def test_parity_block_diagonal_mask(cuda_device, B, H, N, D, b):
 @pytest.mark.parametrize("mode,N,l,c,finalise,summary", [
     ("fixed", 2048, 128, 32, 0, 1),   # own block = one 128-key tile per 64-query step
     ("block", 960, 64, 0, 0, 0),
-    ("fixed", 2048, 256, 32, 1, 0),   # a step of the second half of a block meets two key tiles;
-                                      # its natural items run the LONG shape, which adds the partials itself
+    ("fixed", 2048, 256, 32, 1, 1),   # a step of the second half of a block meets two key tiles
+    ("fixed", 2048, 512, 32, 1, 0),   # natural items of 5 steps on average: the LONG shape, which adds
+                                      # the summary partials itself
     ("strided", 2048, 64, 0, 1, 0),
     ("column", 2048, 64, 0, 1, 0),    # no natural view
 ])
