@@ -71,6 +71,9 @@ SMALL = [
     # the natural pass writes the final dQ alone (D = 128, ragged)
     ("block", 1, 1, 1088, 128, 128, 0, 64),
     ("block", 2, 1, 1000, 32, 64, 0, 8),
+    # fixed with l = 512: natural items of 5 steps on average take the LONG shape, whose epilogue
+    # loads the summary partials and adds them itself (the SHORT shape reduces into them instead)
+    ("fixed", 1, 1, 2048, 64, 512, 64, 64),
 ]
 
 
