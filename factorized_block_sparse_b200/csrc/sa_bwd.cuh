@@ -21,9 +21,13 @@
 //   (where each query step meets one key tile of the pass: stored into it by
 //   the first pass, or added to the earlier passes' sum and stored as the
 //   final bf16 rows by the natural pass).
-// K/V are double-buffered so the next item's tiles load during this one, and
-// the dV/dK epilogue of an item runs in the dQ warps while the next item's
-// steps proceed.
+// In the SHORT shape K/V and dV/dK are double-buffered so the next item's
+// tiles load and accumulate during this one; the dV/dK epilogue of an item
+// runs in the dQ warps while the next item's steps proceed.  A secondary
+// (column or summary) view's pass writes its dK/dV as fp32 partials at the
+// keys' natural positions; the natural pass then adds them to its own rows
+// and writes bf16 (or, SUM_RED, reduce-adds its rows into the partials and a
+// small launch rounds them).
 // Roles (480 threads): warp 0 producer (TMA for K, V, Q, dO; bulk copy of
 // the packed lse/Delta), warp 1 TMEM allocation and lane 0 issue of ST/dPT,
 // warps 2..9 elementwise (two groups of four taking alternate global steps,
