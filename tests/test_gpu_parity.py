@@ -74,6 +74,9 @@ SMALL = [
     # fixed with l = 512: natural items of 5 steps on average take the LONG shape, whose epilogue
     # loads the summary partials and adds them itself (the SHORT shape reduces into them instead)
     ("fixed", 1, 1, 2048, 64, 512, 64, 64),
+    # summary rows of up to 127 steps (LONG items of many steps), and a ragged last block at D = 32
+    ("fixed", 1, 1, 8192, 64, 64, 16, 64),
+    ("fixed", 2, 1, 8100, 32, 64, 16, 4),       # ragged last block, D = 32
 ]
 
 
