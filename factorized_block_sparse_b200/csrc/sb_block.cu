@@ -375,6 +375,10 @@ int ln_bwd(const __nv_bfloat16* x, const float* g, const __nv_bfloat16* dy, cons
   return go(ln_bwd_kernel<0>);
 }
 
+// Serialises the host side of the block calls: the per-device cuBLAS handle
+// is bound to the caller's stream for the duration of one call's enqueue.
+std::mutex g_call_mu;
+
 // One cuBLAS handle per device, created on first use.
 cublasHandle_t handle_for_current_device() {
   static std::mutex mu;
@@ -538,6 +542,7 @@ int sparse_block_fwd(const void* x, const sb_params* p, void* y, int B, int N, i
   if (!x || !y || x == y || !params_ok(p)) return SA_ERR_INVALID_ARG;
   int st = check_args(B, N, H, D, layout, workspace, ws_bytes);
   if (st) return st;
+  std::lock_guard<std::mutex> lock(g_call_mu);
   Gemm G{handle_for_current_device()};
   if (!G.h) return SA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -553,6 +558,7 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
     return SA_ERR_INVALID_ARG;
   int st = check_args(B, N, H, D, layout, workspace, ws_bytes);
   if (st) return st;
+  std::lock_guard<std::mutex> lock(g_call_mu);
   Gemm G{handle_for_current_device()};
   if (!G.h) return SA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

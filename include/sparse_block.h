@@ -25,7 +25,9 @@
  * by the weight's rows); layer-norm parameters and all parameter gradients
  * float32.  Every call is asynchronous on `stream` (a cudaStream_t, or NULL
  * for the legacy default stream) and returns an sa_status of sparse_attn.h;
- * argument errors are returned before any device work.
+ * argument errors are returned before any device work.  Calls from several
+ * host threads are safe (their enqueues are serialised); calls whose GPU work
+ * overlaps must not share a workspace.
  */
 #ifndef SPARSE_BLOCK_H
 #define SPARSE_BLOCK_H
