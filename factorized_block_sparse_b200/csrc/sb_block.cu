@@ -183,12 +183,41 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const __nv_bfloat16* __rest
   }
 }
 
+// A lane's chunks of a bf16 row kept as raw 16-byte words (half the
+// registers of floats), zero beyond C.
+template <int NCH>
+struct Raw {
+  uint4 v[NCH > 0 ? NCH : 1];
+};
+
+template <int NCH>
+__device__ __forceinline__ void raw_load(Raw<NCH>& r, const __nv_bfloat16* p, int C, int lane) {
+#pragma unroll
+  for (int j = 0; j < NCH; ++j) {
+    const int i = lane * 8 + 256 * j;
+    r.v[j] = i < C ? *reinterpret_cast<const uint4*>(p + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
 // Layer-norm backward with the residual added:
 //   dx = resid + rstd (dxh - mean(dxh) - xh mean(dxh xh)),  dxh = dy g,
 //   dg += sum_rows dy xh,  db += sum_rows dy  (float32, zeroed by the caller).
 // One warp per row.  A lane owns the same channels in every row it visits, so
 // each warp sums dg/db into its own shared-memory slice with plain adds; the
-// block adds its warps' slices to global memory once.
+// block adds its warps' slices to global memory once.  For short rows
+// (NCH <= 2) a warp requests the x, dy and residual rows of its next row
+// before it works on the current one (kept as raw bf16 words), so that the
+// loads of a row overlap the arithmetic of the one before.
 template <int NCH>
 __global__ void __launch_bounds__(128) ln_bwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
                                                      const __nv_bfloat16* __restrict__ dy,
@@ -208,45 +237,111 @@ __global__ void __launch_bounds__(128) ln_bwd_kernel(const __nv_bfloat16* __rest
   Row<REG_SUMS ? NCH : 0> sg{}, sb{};
   const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long r = w0; r < M; r += nw) {
-    const __nv_bfloat16* xr = x + r * C;
-    const __nv_bfloat16* dr = dy + r * C;
-    Row<NCH> row;
-    row_load(row, xr, C, lane);
-    float mean, rstd;
-    row_stats(row, xr, C, lane, mean, rstd);
-    float s1 = 0.f, s2 = 0.f;
-    for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
-      float d[8];
-      load8(dr + i, d);
+  if constexpr (NCH > 0 && NCH <= 2) {
+    Raw<NCH> xa, da, ra;
+    auto load3 = [&](long long r, Raw<NCH>& xr, Raw<NCH>& dr, Raw<NCH>& rr) {
+      raw_load(xr, x + r * C, C, lane);
+      raw_load(dr, dy + r * C, C, lane);
+      raw_load(rr, resid + r * C, C, lane);
+    };
+    if (w0 < M) load3(w0, xa, da, ra);
+    for (long long r = w0; r < M; r += nw) {
+      Raw<NCH> xn, dn, rn;  // the next row of this warp, requested before this one is worked on
+      if (r + nw < M) load3(r + nw, xn, dn, rn);
+      float xs[NCH * 8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float xh = (f[u] - mean) * rstd;
-        const float dxh = d[u] * param(gv, g, i, j, u);
-        s1 += dxh;
-        s2 += dxh * xh;
-        if constexpr (REG_SUMS) {
-          sg.v[8 * j + u] += d[u] * xh;
-          sb.v[8 * j + u] += d[u];
-        } else {
+      for (int jc = 0; jc < NCH; ++jc) unpack8(xa.v[jc], xs + 8 * jc);
+      float sum = 0.f;
+#pragma unroll
+      for (int k = 0; k < NCH * 8; ++k) sum += xs[k];
+      const float mean = warp_sum(sum) / C;
+      float var = 0.f;
+#pragma unroll
+      for (int jc = 0; jc < NCH; ++jc)
+        if (lane * 8 + 256 * jc < C)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) var += (xs[8 * jc + u] - mean) * (xs[8 * jc + u] - mean);
+      const float rstd = rsqrtf(warp_sum(var) / C + kEps);
+      float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+      for (int jc = 0; jc < NCH; ++jc) {
+        const int i = lane * 8 + 256 * jc;
+        if (i >= C) continue;
+        float d[8];
+        unpack8(da.v[jc], d);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int k = 8 * jc + u;
+          const float xh = (xs[k] - mean) * rstd;
+          const float dxh = d[u] * gv.v[k];
+          s1 += dxh;
+          s2 += dxh * xh;
+          if constexpr (REG_SUMS) {
+            sg.v[k] += d[u] * xh;
+            sb.v[k] += d[u];
+          } else {
+            mine[i + u] += d[u] * xh;
+            mine[C + i + u] += d[u];
+          }
+        }
+      }
+      s1 = warp_sum(s1) / C;
+      s2 = warp_sum(s2) / C;
+#pragma unroll
+      for (int jc = 0; jc < NCH; ++jc) {
+        const int i = lane * 8 + 256 * jc;
+        if (i >= C) continue;
+        float d[8], o[8];
+        unpack8(da.v[jc], d);
+        unpack8(ra.v[jc], o);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int k = 8 * jc + u;
+          const float xh = (xs[k] - mean) * rstd;
+          o[u] += rstd * (d[u] * gv.v[k] - s1 - xh * s2);
+        }
+        store8(dx + r * C + i, o);
+      }
+      xa = xn;
+      da = dn;
+      ra = rn;
+    }
+  } else {
+    for (long long r = w0; r < M; r += nw) {
+      const __nv_bfloat16* xr = x + r * C;
+      const __nv_bfloat16* dr = dy + r * C;
+      Row<NCH> row;
+      row_load(row, xr, C, lane);
+      float mean, rstd;
+      row_stats(row, xr, C, lane, mean, rstd);
+      float s1 = 0.f, s2 = 0.f;
+      for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
+        float d[8];
+        load8(dr + i, d);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float xh = (f[u] - mean) * rstd;
+          const float dxh = d[u] * param(gv, g, i, j, u);
+          s1 += dxh;
+          s2 += dxh * xh;
           mine[i + u] += d[u] * xh;
           mine[C + i + u] += d[u];
         }
-      }
-    });
-    s1 = warp_sum(s1) / C;
-    s2 = warp_sum(s2) / C;
-    for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
-      float d[8], o[8];
-      load8(dr + i, d);
-      load8(resid + r * C + i, o);
+      });
+      s1 = warp_sum(s1) / C;
+      s2 = warp_sum(s2) / C;
+      for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
+        float d[8], o[8];
+        load8(dr + i, d);
+        load8(resid + r * C + i, o);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float xh = (f[u] - mean) * rstd;
-        o[u] += rstd * (d[u] * param(gv, g, i, j, u) - s1 - xh * s2);
-      }
-      store8(dx + r * C + i, o);
-    });
+        for (int u = 0; u < 8; ++u) {
+          const float xh = (f[u] - mean) * rstd;
+          o[u] += rstd * (d[u] * param(gv, g, i, j, u) - s1 - xh * s2);
+        }
+        store8(dx + r * C + i, o);
+      });
+    }
   }
   if constexpr (REG_SUMS) {
 #pragma unroll
@@ -360,12 +455,19 @@ int ln_bwd(const __nv_bfloat16* x, const float* g, const __nv_bfloat16* dy, cons
            __nv_bfloat16* dx, float* dg, float* db, long long M, int C, cudaStream_t s) {
   constexpr int kThreads = 128;  // 4 warps, each with its own dg/db slice
   const size_t smem = 4 * 2 * static_cast<size_t>(C) * sizeof(float);
-  const int grid = static_cast<int>(std::min<long long>((M + 3) / 4, 148 * 4));
   auto go = [&](auto kernel) -> int {
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
             cudaSuccess)
       return SA_ERR_CUDA;
+    // one wave of resident blocks (at most 4 a SM: each adds 2 C sums to dg/db)
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem) != cudaSuccess)
+      return SA_ERR_CUDA;
+    per_sm = std::max(1, std::min(per_sm, 4));
+    const int grid = static_cast<int>(std::min<long long>((M + 3) / 4, static_cast<long long>(sms) * per_sm));
     kernel<<<grid, kThreads, smem, s>>>(x, g, dy, resid, dx, dg, db, M, C);
     return last_launch();
   };
