@@ -583,7 +583,8 @@ T* at(void* ws, size_t off) {
 }
 
 // The forward chain into the workspace: a, q, k, v, o, lse, o2, h, f, u, g
-// (and y = h + g W2 when y is given; gelu'(u) into gelu_grad when given).
+// (when y is given, h is built in y and y = h + g W2 follows; gelu'(u) into
+// gelu_grad when given).
 int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, int B, int N, int H, int D,
                   const sa_layout* L, void* ws, cudaStream_t s, const Gemm& G, __nv_bfloat16* gelu_grad = nullptr) {
   const Ws w = layout_ws(B, N, H, D, L);
@@ -609,17 +610,17 @@ int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, 
   if ((st = sparse_attn_fwd(q, k, v, o, lse, B, H, N, D, L, s))) return st;
   heads_kernel<false><<<heads_grid(M), heads_block(C), 0, s>>>(o2, o, nullptr, nullptr, B, N, H, D, 1);
   if ((st = last_launch())) return st;
-  if (cudaMemcpyAsync(h, x, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
-  if ((st = G.mm(o2, p->w_o, h, static_cast<int>(M), C, C, 1.f))) return st;
-  if ((st = ln_fwd(h, p->ln2_g, p->ln2_b, f, M, C, s))) return st;
+  // h = x + o Wo; the forward proper builds h in y itself (y = h + ff then
+  // needs no copy of h), the recomputation in the workspace
+  __nv_bfloat16* hb = y ? y : h;
+  if (cudaMemcpyAsync(hb, x, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
+  if ((st = G.mm(o2, p->w_o, hb, static_cast<int>(M), C, C, 1.f))) return st;
+  if ((st = ln_fwd(hb, p->ln2_g, p->ln2_b, f, M, C, s))) return st;
   if ((st = G.mm(f, p->w_1, u, static_cast<int>(M), C, 4 * C, 0.f))) return st;
   if (gelu_grad) gelu_kernel<true><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, gelu_grad, M * 4 * C / 8);
   else gelu_kernel<false><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, nullptr, M * 4 * C / 8);
   if ((st = last_launch())) return st;
-  if (y) {
-    if (cudaMemcpyAsync(y, h, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
-    if ((st = G.mm(g, p->w_2, y, static_cast<int>(M), 4 * C, C, 1.f))) return st;
-  }
+  if (y && (st = G.mm(g, p->w_2, y, static_cast<int>(M), 4 * C, C, 1.f))) return st;
   return SA_OK;
 }
 

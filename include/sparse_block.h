@@ -73,7 +73,10 @@ size_t sparse_block_workspace_size(int B, int N, int H, int D, const sa_layout* 
 
 /*
  * sparse_block_fwd - y = block(x).  x, y: bf16 [B, N, H*D] (y must not
- * alias x).  D in {32, 64, 128}; layout as for sparse_attn_fwd (its N).
+ * alias x, and must not overlap x or the workspace: the residual stream
+ * h = x + attn(LN1(x)) is built in y before y = h + ff(LN2(h)), so after an
+ * error y holds unspecified values).  D in {32, 64, 128}; layout as for
+ * sparse_attn_fwd (its N).
  * workspace: at least sparse_block_workspace_size() bytes, 256-byte
  * aligned, contents on entry irrelevant, on exit unspecified.
  * Errors: SA_ERR_INVALID_ARG (null pointer, non-positive size, y == x),
