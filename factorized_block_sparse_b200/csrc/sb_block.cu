@@ -155,34 +155,6 @@ __device__ __forceinline__ float param(const Row<NCH>& r, const float* p, int i,
   else return p[i + u];
 }
 
-// y = (x - mean) * rstd * g + b per row; one warp per row.
-template <int NCH>
-__global__ void __launch_bounds__(256) ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
-                                                     const float* __restrict__ b, __nv_bfloat16* __restrict__ y,
-                                                     long long M, int C) {
-  const int lane = threadIdx.x & 31;
-  const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  // a lane owns the same channels in every row: their gains and biases stay in registers
-  Row<NCH> gv, bv;
-  row_load_f32(gv, g, C, lane);
-  row_load_f32(bv, b, C, lane);
-  for (long long r = w0; r < M; r += nw) {
-    const __nv_bfloat16* xr = x + r * C;
-    Row<NCH> row;
-    row_load(row, xr, C, lane);
-    float mean, rstd;
-    row_stats(row, xr, C, lane, mean, rstd);
-    for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
-      float o[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        o[u] = (f[u] - mean) * rstd * param(gv, g, i, j, u) + param(bv, b, i, j, u);
-      store8(y + r * C + i, o);
-    });
-  }
-}
-
 // A lane's chunks of a bf16 row kept as raw 16-byte words (half the
 // registers of floats), zero beyond C.
 template <int NCH>
@@ -206,6 +178,55 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* f) {
     const float2 t = __bfloat1622float2(h[i]);
     f[2 * i] = t.x;
     f[2 * i + 1] = t.y;
+  }
+}
+
+// y = (x - mean) * rstd * g + b per row; one warp per row.
+template <int NCH>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
+                                                     const float* __restrict__ b, __nv_bfloat16* __restrict__ y,
+                                                     long long M, int C) {
+  const int lane = threadIdx.x & 31;
+  const long long w0 = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  // a lane owns the same channels in every row: their gains and biases stay in registers
+  Row<NCH> gv, bv;
+  row_load_f32(gv, g, C, lane);
+  row_load_f32(bv, b, C, lane);
+  if constexpr (NCH > 0 && NCH <= 2) {
+    // short rows: the warp requests its next row before it works on this one
+    Raw<NCH> xa, xn;
+    if (w0 < M) raw_load(xa, x + w0 * C, C, lane);
+    for (long long r = w0; r < M; r += nw) {
+      if (r + nw < M) raw_load(xn, x + (r + nw) * C, C, lane);
+      Row<NCH> row;
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) unpack8(xa.v[j], row.v + 8 * j);
+      float mean, rstd;
+      row_stats(row, x + r * C, C, lane, mean, rstd);
+      for_chunks(row, x + r * C, C, lane, [&](int i, int j, const float* f) {
+        float o[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) o[u] = (f[u] - mean) * rstd * gv.v[8 * j + u] + bv.v[8 * j + u];
+        store8(y + r * C + i, o);
+      });
+      xa = xn;
+    }
+  } else {
+    for (long long r = w0; r < M; r += nw) {
+      const __nv_bfloat16* xr = x + r * C;
+      Row<NCH> row;
+      row_load(row, xr, C, lane);
+      float mean, rstd;
+      row_stats(row, xr, C, lane, mean, rstd);
+      for_chunks(row, xr, C, lane, [&](int i, int j, const float* f) {
+        float o[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          o[u] = (f[u] - mean) * rstd * param(gv, g, i, j, u) + param(bv, b, i, j, u);
+        store8(y + r * C + i, o);
+      });
+    }
   }
 }
 
@@ -440,15 +461,26 @@ int heads_grid(long long M) { return static_cast<int>(std::min<long long>(M, 148
 int heads_block(int width) { return std::min(256, std::max(32, (width / 8 + 31) / 32 * 32)); }
 
 // Layer-norm launches: the row in registers up to C = 1024, read again per
-// pass above that.
+// pass above that; for C <= 512 each warp requests its next row ahead.
 int ln_fwd(const __nv_bfloat16* x, const float* g, const float* b, __nv_bfloat16* y, long long M, int C,
            cudaStream_t s) {
-  const int grid = grid_for(M * 32, 256);
-  if (C <= 256) ln_fwd_kernel<1><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
-  else if (C <= 512) ln_fwd_kernel<2><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
-  else if (C <= 1024) ln_fwd_kernel<4><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
-  else ln_fwd_kernel<0><<<grid, 256, 0, s>>>(x, g, b, y, M, C);
-  return last_launch();
+  auto go = [&](auto kernel, bool one_wave) -> int {
+    int grid = grid_for(M * 32, 256);
+    if (one_wave) {  // rows requested ahead: one wave of resident blocks, each warp several rows
+      int dev = 0, sms = 0, per_sm = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess)
+        return SA_ERR_CUDA;
+      grid = static_cast<int>(std::min<long long>(grid, static_cast<long long>(sms) * std::max(per_sm, 1)));
+    }
+    kernel<<<grid, 256, 0, s>>>(x, g, b, y, M, C);
+    return last_launch();
+  };
+  if (C <= 256) return go(ln_fwd_kernel<1>, true);
+  if (C <= 512) return go(ln_fwd_kernel<2>, true);
+  if (C <= 1024) return go(ln_fwd_kernel<4>, false);
+  return go(ln_fwd_kernel<0>, false);
 }
 
 int ln_bwd(const __nv_bfloat16* x, const float* g, const __nv_bfloat16* dy, const __nv_bfloat16* resid,
