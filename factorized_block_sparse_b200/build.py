@@ -86,7 +86,7 @@ def build_block_lib(force=False, verbose=False):
     cmd = [nvcc_path(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
            "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static", "-Xlinker", "-soname=libsparse_block.so",
            "-I", os.path.join(ROOT, "include"), "-o", BLOCK_LIB, *BLOCK_SOURCES,
-           "-L", HERE, "-lsparse_attn", "-L", cuda_lib_dir(), "-lcublas",
+           "-L", HERE, "-lsparse_attn", "-L", cuda_lib_dir(), "-lcublas", "-lcublasLt",
            "-Xlinker", "-rpath,$ORIGIN", "-Xlinker", "-rpath," + cuda_lib_dir()]
     if verbose:
         print(" ".join(cmd), flush=True)

@@ -1,7 +1,8 @@
 // The Sparse Transformer block around the attention op: layer norms, the
 // GELU feed-forward, the residual stream and the head layout in CUDA kernels
-// of this file, the projections as cuBLAS GEMMs (bf16 in, fp32 accumulation)
-// and the attention through libsparse_attn's C ABI.
+// of this file, the projections as cuBLAS GEMMs (bf16 in, fp32 accumulation;
+// cuBLASLt where the residual input and the output differ) and the attention
+// through libsparse_attn's C ABI.
 //
 // The block ("[논문 리뷰] Generating Long Sequences with Sparse Transformers",
 // "제안 방법", third and fourth items; pcnews translation, "Глубокое
@@ -12,6 +13,7 @@
 // Data layout: activations [M = B*N rows][C = H*D] bf16 row-major; the
 // attention's q, k, v, o in its own [B, H, N, D] layout (head h = columns
 // h*D .. h*D+D-1 of a C-wide row), converted by to_heads / from_heads.
+#include <cublasLt.h>
 #include <cublas_v2.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -524,6 +526,48 @@ cublasHandle_t handle_for_current_device() {
   return handles[dev];
 }
 
+cublasLtHandle_t lt_handle_for_current_device() {
+  static std::mutex mu;
+  static cublasLtHandle_t handles[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!handles[dev] && cublasLtCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
+  return handles[dev];
+}
+
+// Row-major Out[M][Nn] = A[M][K] W[K][Nn] + R[M][Nn], all bf16, float32
+// accumulation; R and Out distinct buffers (cuBLASLt, no workspace).
+int mm_residual(cublasLtHandle_t lt, const void* A, const void* W, const void* R, void* Out, int M, int K, int Nn,
+                cudaStream_t s) {
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  int st = SA_ERR_CUDA;
+  const float one = 1.f;
+  size_t ws = 0;
+  cublasLtMatmulHeuristicResult_t res{};
+  int n_res = 0;
+  if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) == CUBLAS_STATUS_SUCCESS &&
+      cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, Nn, K, Nn) == CUBLAS_STATUS_SUCCESS &&
+      cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, K, M, K) == CUBLAS_STATUS_SUCCESS &&
+      cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, Nn, M, Nn) == CUBLAS_STATUS_SUCCESS &&
+      cublasLtMatmulPreferenceCreate(&pref) == CUBLAS_STATUS_SUCCESS &&
+      cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws, sizeof(ws)) ==
+          CUBLAS_STATUS_SUCCESS &&
+      cublasLtMatmulAlgoGetHeuristic(lt, op, la, lb, lc, lc, pref, 1, &res, &n_res) == CUBLAS_STATUS_SUCCESS &&
+      n_res > 0 &&
+      cublasLtMatmul(lt, op, &one, W, la, A, lb, &one, R, lc, Out, lc, &res.algo, nullptr, 0, s) ==
+          CUBLAS_STATUS_SUCCESS)
+    st = SA_OK;
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return st;
+}
+
 struct Gemm {
   cublasHandle_t h;
   // Row-major Out[M][Nn] = A[M][K] W[K][Nn] + beta Out (bf16 out).
@@ -642,11 +686,15 @@ int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, 
   if ((st = sparse_attn_fwd(q, k, v, o, lse, B, H, N, D, L, s))) return st;
   heads_kernel<false><<<heads_grid(M), heads_block(C), 0, s>>>(o2, o, nullptr, nullptr, B, N, H, D, 1);
   if ((st = last_launch())) return st;
-  // h = x + o Wo; the forward proper builds h in y itself (y = h + ff then
-  // needs no copy of h), the recomputation in the workspace
+  // h = x + o Wo, the residual added by the GEMM itself (cuBLASLt reads x
+  // and writes h, so no copy of x); the forward proper builds h in y itself
+  // (y = h + ff then needs no copy of h), the recomputation in the workspace
   __nv_bfloat16* hb = y ? y : h;
-  if (cudaMemcpyAsync(hb, x, M * C * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return SA_ERR_CUDA;
-  if ((st = G.mm(o2, p->w_o, hb, static_cast<int>(M), C, C, 1.f))) return st;
+  {
+    cublasLtHandle_t lt = lt_handle_for_current_device();
+    if (!lt) return SA_ERR_CUDA;
+    if ((st = mm_residual(lt, o2, p->w_o, x, hb, static_cast<int>(M), C, C, s))) return st;
+  }
   if ((st = ln_fwd(hb, p->ln2_g, p->ln2_b, f, M, C, s))) return st;
   if ((st = G.mm(f, p->w_1, u, static_cast<int>(M), C, 4 * C, 0.f))) return st;
   if (gelu_grad) gelu_kernel<true><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, gelu_grad, M * 4 * C / 8);
