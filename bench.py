@@ -142,6 +142,8 @@ def kernel_units(w, counts):
         f"sa_bwd_preprocess.{m}": ("hbm", rows * (2 * D * 2 + 4)),
         f"sa_bwd_finalize_dq.{m}": ("hbm", rows * D * (4 + 2)),
     }
+    if m == "fixed" and w.get("c"):  # the summary keys' dK, dV: two fp32 rows read, two bf16 rows written
+        out[f"sa_bwd_finalize_summary_dkv.{m}"] = ("hbm", w["B"] * w["H"] * (w["N"] // w["l"]) * w["c"] * D * 12)
     if "N" in counts:
         out[f"sa_fwd_natural_view.{m}"] = ("tensor", 4 * per * fwd_main)
         out[f"sa_bwd_natural_view.{m}"] = ("tensor", 10 * per * counts["N"])
@@ -488,7 +490,7 @@ def main():
     # dominant kernel of the timed region
     dom, dom_ms = None, -1.0
     for name, (ms, cnt) in ktimes.items():
-        if cnt and ms > dom_ms:
+        if cnt and name in units and ms > dom_ms:
             dom, dom_ms = name, ms
     cnt = ktimes[dom][1]
     bound, per_launch = units.get(dom, ("tensor", None))
