@@ -1,7 +1,7 @@
 /*
  * sparse_block.h - C ABI of the Sparse Transformer block around the
  * factorized sparse attention op (libsparse_block.so, which calls
- * libsparse_attn.so for the attention and cuBLAS for the projections).
+ * libsparse_attn.so for the attention and cuBLAS and cuBLASLt for the projections).
  *
  * The block ("[논문 리뷰] Generating Long Sequences with Sparse Transformers",
  * "제안 방법", third and fourth items; the pcnews translation "Генеративное
@@ -82,7 +82,7 @@ size_t sparse_block_workspace_size(int B, int N, int H, int D, const sa_layout* 
  * Errors: SA_ERR_INVALID_ARG (null pointer, non-positive size, y == x),
  * SA_ERR_WORKSPACE (workspace null or too small), SA_ERR_UNSUPPORTED (D not
  * in {32, 64, 128}, or H*D above 6144), the errors of sparse_attn_fwd,
- * SA_ERR_CUDA when a cuBLAS call or a launch fails.
+ * SA_ERR_CUDA when a cuBLAS or cuBLASLt call or a launch fails.
  */
 int sparse_block_fwd(const void* x, const sb_params* p, void* y, int B, int N, int H, int D,
                      const sa_layout* layout, void* workspace, size_t ws_bytes, void* stream);
