@@ -671,7 +671,7 @@ def measure_block(sa, pk, dev, stream, flush, steps=10, warmup=3):
     ms = sum(a.elapsed_time(b) for a, b in evs) / steps
     achieved = fl / (ms * 1e-3) / 1e12
     out = {"workload": f"one block, fixed pattern, B={B}, N={N}, H={H}, D={D} (C={C}, hidden {4 * C}), l={w['l']}, "
-                       f"c={w['c']}, block={w['block']}; bf16 activations, cuBLAS projections",
+                       f"c={w['c']}, block={w['block']}; bf16 activations, cuBLAS and cuBLASLt projections",
            "ms_per_step": round(ms, 4), "tflops": round(achieved, 2), "unit": "TFLOP/s",
            "flops_per_step": {"total": fl, "projections": fl_gemm},
            "tokens_per_s": round(B * N / (ms * 1e-3), 1),

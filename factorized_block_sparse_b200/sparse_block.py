@@ -2,8 +2,8 @@
 Transformer block around the attention op.
 
 Argument marshalling only: the block runs in ``libsparse_block.so`` (CUDA
-kernels for the layer norms, GELU and head layout, cuBLAS for the
-projections, ``libsparse_attn.so`` for the attention).  Tensors are
+kernels for the layer norms, GELU and head layout, cuBLAS and cuBLASLt for
+the projections, ``libsparse_attn.so`` for the attention).  Tensors are
 ``torch.Tensor`` objects on a CUDA device: activations bf16 ``[B, N, C]``
 with ``C = H * D``, projection weights bf16 ``[in, out]``, layer-norm
 parameters and parameter gradients float32.  There is no CPU fallback.
