@@ -387,9 +387,27 @@ __global__ void __launch_bounds__(128) ln_bwd_kernel(const __nv_bfloat16* __rest
   }
 }
 
-// gelu(u) = u Phi(u) = u (1 + erf(u / sqrt 2)) / 2, 8 elements a thread;
-// with GRAD also its derivative Phi(u) + u phi(u) (phi the standard normal
-// density), for the backward pass's recomputation.
+// Phi(u) and the standard normal density phi(u) from one exponential, by
+// the rational approximation of the complementary error function in
+// Abramowitz and Stegun, Handbook of Mathematical Functions, eq. 7.1.26
+// (absolute error below 1.5e-7 for z >= 0):
+//   erfc(z) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2),  t = 1 / (1 + p z),
+// with z = |u| / sqrt 2, so that exp(-z^2) = sqrt(2 pi) phi(u) and
+// Phi(-|u|) = erfc(z) / 2.
+__device__ __forceinline__ void normal_cdf_pdf(float u, float& cdf, float& pdf) {
+  const float z = fabsf(u) * 0.70710678118654752f;
+  const float t = __fdividef(1.f, fmaf(0.3275911f, z, 1.f));
+  const float e = __expf(-z * z);
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f), 0.254829592f);
+  const float tail = 0.5f * poly * e;  // Phi(-|u|)
+  cdf = u >= 0.f ? 1.f - tail : tail;
+  pdf = 0.3989422804014327f * e;
+}
+
+// gelu(u) = u Phi(u), 8 elements a thread; with GRAD also its derivative
+// Phi(u) + u phi(u) (phi the standard normal density), for the backward
+// pass's recomputation.
 template <bool GRAD>
 __global__ void __launch_bounds__(256) gelu_kernel(const __nv_bfloat16* __restrict__ u, __nv_bfloat16* __restrict__ out,
                                                    __nv_bfloat16* __restrict__ grad, long long n8) {
@@ -399,9 +417,10 @@ __global__ void __launch_bounds__(256) gelu_kernel(const __nv_bfloat16* __restri
     load8(u + i * 8, f);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float cdf = 0.5f * (1.f + erff(f[k] * 0.70710678118654752f));
+      float cdf, pdf;
+      normal_cdf_pdf(f[k], cdf, pdf);
       o[k] = f[k] * cdf;
-      if (GRAD) gd[k] = cdf + f[k] * 0.3989422804014327f * expf(-0.5f * f[k] * f[k]);
+      if (GRAD) gd[k] = cdf + f[k] * pdf;
     }
     store8(out + i * 8, o);
     if (GRAD) store8(grad + i * 8, gd);
@@ -713,6 +732,21 @@ bool params_ok(const sb_params* p) {
 using namespace sb;
 
 extern "C" {
+
+int sparse_block_gelu(const void* u, void* g, void* dgelu, size_t n, void* stream) {
+  if (!u || !g || n % 8 || ((reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(g) |
+                             reinterpret_cast<uintptr_t>(dgelu)) & 15u))
+    return SA_ERR_INVALID_ARG;
+  if (dgelu && (dgelu == u || dgelu == g)) return SA_ERR_INVALID_ARG;
+  if (n == 0) return SA_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long n8 = static_cast<long long>(n / 8);
+  const auto* ub = static_cast<const __nv_bfloat16*>(u);
+  auto* gb = static_cast<__nv_bfloat16*>(g);
+  if (dgelu) gelu_kernel<true><<<grid_for(n8, 256), 256, 0, s>>>(ub, gb, static_cast<__nv_bfloat16*>(dgelu), n8);
+  else gelu_kernel<false><<<grid_for(n8, 256), 256, 0, s>>>(ub, gb, nullptr, n8);
+  return last_launch();
+}
 
 size_t sparse_block_workspace_size(int B, int N, int H, int D, const sa_layout* layout) {
   if (B < 1 || N < 1 || H < 1 || !layout || (D != 32 && D != 64 && D != 128) || H * D > kMaxC) return 0;

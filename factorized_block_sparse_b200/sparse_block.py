@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsparse_block.so")
 
 PARAMS = ("ln1_g", "ln1_b", "w_qkv", "w_o", "ln2_g", "ln2_b", "w_1", "w_2")
-EXPORTS = ("sparse_block_workspace_size", "sparse_block_fwd", "sparse_block_bwd")
+EXPORTS = ("sparse_block_workspace_size", "sparse_block_fwd", "sparse_block_bwd", "sparse_block_gelu")
 
 
 class _Params(ctypes.Structure):
@@ -39,6 +39,8 @@ def load_library(path=None):
     lib.sparse_block_fwd.restype = I
     lib.sparse_block_bwd.argtypes = [VP, VP, P, VP, P, I, I, I, I, VP, VP, SZ, VP]
     lib.sparse_block_bwd.restype = I
+    lib.sparse_block_gelu.argtypes = [VP, VP, VP, SZ, VP]
+    lib.sparse_block_gelu.restype = I
     return lib
 
 
@@ -101,3 +103,18 @@ def backward(x, dy, params, H, layout, ws=None, stream=None):
     grads = {n: torch.empty(params[n].shape, dtype=torch.float32, device=x.device) for n in PARAMS}
     sparse_block_bwd(x, dy, params, dx, grads, H, layout, ws, stream)
     return dx, grads
+
+
+def sparse_block_gelu(u, g, dgelu=None, stream=None):
+    sa._check(lib.sparse_block_gelu(sa._ptr(u), sa._ptr(g), sa._ptr(dgelu) if dgelu is not None else None,
+                                    u.numel(), sa._stream_ptr(stream)), "sparse_block_gelu")
+
+
+def gelu(u, grad=False, stream=None):
+    """``gelu(u)`` (and ``gelu'(u)`` when ``grad``) of a bf16 tensor with a multiple of 8 elements."""
+    import torch
+
+    g = torch.empty_like(u)
+    d = torch.empty_like(u) if grad else None
+    sparse_block_gelu(u, g, d, stream)
+    return (g, d) if grad else g

@@ -88,6 +88,22 @@ int sparse_block_fwd(const void* x, const sb_params* p, void* y, int B, int N, i
                      const sa_layout* layout, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * sparse_block_gelu - the block's feed-forward activation on its own,
+ * elementwise over n bf16 values: g = gelu(u) = u Phi(u) and, when dgelu is
+ * not null, dgelu = gelu'(u) = Phi(u) + u phi(u) (Phi, phi: the standard
+ * normal distribution and density).  Phi is taken from the rational
+ * approximation of erfc in Abramowitz and Stegun, Handbook of Mathematical
+ * Functions, eq. 7.1.26: absolute error below 7.5e-8 in Phi, so below
+ * |u| 7.5e-8 in gelu (relative error grows only in the far negative tail,
+ * where |gelu(u)| < 1.5e-6), before the bf16 rounding of the result.
+ * u, g, dgelu: device pointers, 16-byte aligned; n a multiple of 8; g may
+ * be u (in place); dgelu must be neither.  Enqueued on stream.
+ * Errors: SA_ERR_INVALID_ARG (u or g null, n not a multiple of 8, a pointer
+ * not 16-byte aligned, dgelu equal to u or g), SA_ERR_CUDA (launch failure).
+ */
+int sparse_block_gelu(const void* u, void* g, void* dgelu, size_t n, void* stream);
+
+/*
  * sparse_block_bwd - given dy (bf16 [B, N, H*D]), the gradients of
  * sum(y * dy): dx (bf16 [B, N, H*D]) and every parameter (g, float32).
  * Only x is read from the forward pass: the whole block is recomputed from

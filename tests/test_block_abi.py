@@ -52,3 +52,19 @@ def test_block_workspace_size(sb):
     assert ws(1, 1024, 64, 128, lay.handle) == 0      # H * D above 6144
     assert ws(0, 1024, 4, 64, lay.handle) == 0
     assert ws(1, 1024, 4, 64, None) == 0
+
+
+def test_gelu_argument_checks(sb):
+    # refused before anything reaches the device (no GPU needed)
+    from factorized_block_sparse_b200 import sparse_attn as sa
+
+    f = sb.lib.sparse_block_gelu
+    a, b, c = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    assert f(None, b, None, 8, None) == sa.SA_ERR_INVALID_ARG           # u null
+    assert f(a, None, None, 8, None) == sa.SA_ERR_INVALID_ARG           # g null
+    assert f(a, b, None, 12, None) == sa.SA_ERR_INVALID_ARG             # n not a multiple of 8
+    assert f(ctypes.c_void_p(0x10008), b, None, 8, None) == sa.SA_ERR_INVALID_ARG  # u not 16-byte aligned
+    assert f(a, b, ctypes.c_void_p(0x30004), 8, None) == sa.SA_ERR_INVALID_ARG     # dgelu not aligned
+    assert f(a, b, a, 8, None) == sa.SA_ERR_INVALID_ARG                 # dgelu is u
+    assert f(a, b, b, 8, None) == sa.SA_ERR_INVALID_ARG                 # dgelu is g
+    assert f(a, b, c, 0, None) == sa.SA_OK                              # nothing to do

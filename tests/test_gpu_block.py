@@ -94,3 +94,34 @@ def test_block_rejects_bad_arguments(cuda_device):
     with pytest.raises(sa.SparseAttnError) as e:
         sb.sparse_block_fwd(x, p, torch.empty_like(x), H, lay, ws[: ws.numel() // 2])
     assert e.value.status == sa.SA_ERR_WORKSPACE
+
+
+def test_gelu_against_fp32_reference(cuda_device):
+    """The block's GELU and its derivative against PyTorch's exact (erf) GELU
+    in float32 and its derivative in float64, on the same bf16 inputs: within
+    half a bf16 spacing of the reference (the output's own rounding) plus
+    1e-6 (the approximation of Phi, below 7.5e-8 absolute, times |u| <= 12)."""
+    from factorized_block_sparse_b200 import sparse_block as sb
+
+    gen = torch.Generator().manual_seed(30)
+    grid = torch.linspace(-12.0, 12.0, 24576)
+    u = torch.cat([grid, 2.0 * torch.randn(40960, generator=gen)]).to(torch.bfloat16)
+    g, d = sb.gelu(u.to(cuda_device), grad=True)
+    g_in_place = u.to(cuda_device)
+    sb.sparse_block_gelu(g_in_place, g_in_place)
+    torch.cuda.synchronize()
+    uf = u.double()
+    ref_g = torch.nn.functional.gelu(u.float()).double()
+    phi = torch.exp(-0.5 * uf * uf) / np.sqrt(2.0 * np.pi)
+    ref_d = 0.5 * (1.0 + torch.erf(uf / np.sqrt(2.0))) + uf * phi
+
+    def half_ulp(x):
+        ax = x.abs().clamp_min(2.0 ** -126)
+        return 2.0 ** (torch.floor(torch.log2(ax)) - 8)
+
+    for name, got, ref in (("gelu", g, ref_g), ("gelu'", d, ref_d), ("gelu in place", g_in_place, ref_g)):
+        got = got.double().cpu()
+        err = (got - ref).abs()
+        bound = half_ulp(ref) + 1e-6
+        assert torch.isfinite(got).all(), name
+        assert (err <= bound).all(), f"{name}: worst excess {(err - bound).max().item():.3e}"
