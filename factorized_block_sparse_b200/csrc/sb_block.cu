@@ -427,17 +427,24 @@ __global__ void __launch_bounds__(256) gelu_kernel(const __nv_bfloat16* __restri
   }
 }
 
-// a *= b elementwise (bf16, 8 elements a thread): du = dg gelu'(u).
-__global__ void __launch_bounds__(256) mul_kernel(__nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
-                                                  long long n8) {
+// du = dg gelu'(u) elementwise (bf16, 8 elements a thread), gelu'(u) computed
+// again from u (one exponential and one reciprocal an element are cheaper than
+// writing gelu'(u) in the recomputation and reading it back here).
+__global__ void __launch_bounds__(256) dgelu_mul_kernel(const __nv_bfloat16* __restrict__ u,
+                                                        const __nv_bfloat16* __restrict__ dg,
+                                                        __nv_bfloat16* __restrict__ du, long long n8) {
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     float x[8], y[8];
-    load8(a + i * 8, x);
-    load8(b + i * 8, y);
+    load8(u + i * 8, x);
+    load8(dg + i * 8, y);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) x[k] *= y[k];
-    store8(a + i * 8, x);
+    for (int k = 0; k < 8; ++k) {
+      float cdf, pdf;
+      normal_cdf_pdf(x[k], cdf, pdf);
+      y[k] *= cdf + x[k] * pdf;
+    }
+    store8(du + i * 8, y);
   }
 }
 
@@ -678,10 +685,9 @@ T* at(void* ws, size_t off) {
 }
 
 // The forward chain into the workspace: a, q, k, v, o, lse, o2, h, f, u, g
-// (when y is given, h is built in y and y = h + g W2 follows; gelu'(u) into
-// gelu_grad when given).
+// (when y is given, h is built in y and y = h + g W2 follows).
 int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, int B, int N, int H, int D,
-                  const sa_layout* L, void* ws, cudaStream_t s, const Gemm& G, __nv_bfloat16* gelu_grad = nullptr) {
+                  const sa_layout* L, void* ws, cudaStream_t s, const Gemm& G) {
   const Ws w = layout_ws(B, N, H, D, L);
   const long long M = static_cast<long long>(B) * N;
   const int C = H * D;
@@ -716,8 +722,7 @@ int forward_chain(const __nv_bfloat16* x, const sb_params* p, __nv_bfloat16* y, 
   }
   if ((st = ln_fwd(hb, p->ln2_g, p->ln2_b, f, M, C, s))) return st;
   if ((st = G.mm(f, p->w_1, u, static_cast<int>(M), C, 4 * C, 0.f))) return st;
-  if (gelu_grad) gelu_kernel<true><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, gelu_grad, M * 4 * C / 8);
-  else gelu_kernel<false><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, nullptr, M * 4 * C / 8);
+  gelu_kernel<false><<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(u, g, nullptr, M * 4 * C / 8);
   if ((st = last_launch())) return st;
   if (y && (st = G.mm(g, p->w_2, y, static_cast<int>(M), 4 * C, C, 1.f))) return st;
   return SA_OK;
@@ -784,7 +789,7 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   const auto* dyb = static_cast<const __nv_bfloat16*>(dy);
   // the recomputation: every activation again from x
   const Ws w = layout_ws(B, N, H, D, layout);
-  if ((st = forward_chain(xb, p, nullptr, B, N, H, D, layout, workspace, s, G, at<__nv_bfloat16>(workspace, w.du))))
+  if ((st = forward_chain(xb, p, nullptr, B, N, H, D, layout, workspace, s, G)))
     return st;
   const long long M = static_cast<long long>(B) * N;
   const int C = H * D, Mi = static_cast<int>(M);
@@ -813,7 +818,7 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   // feed-forward: y = h + gelu(f W1) W2
   if ((st = G.mm_tn(g, dyb, gr->w_2, Mi, 4 * C, C))) return st;
   if ((st = G.mm_nt(dyb, p->w_2, dg, Mi, 4 * C, C))) return st;
-  mul_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(du, dg, M * 4 * C / 8);  // du held gelu'(u)
+  dgelu_mul_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(at<__nv_bfloat16>(ws, w.u), dg, du, M * 4 * C / 8);
   if ((st = last_launch())) return st;
   if ((st = G.mm_tn(f, du, gr->w_1, Mi, C, 4 * C))) return st;
   if ((st = G.mm_nt(du, p->w_1, df, Mi, C, 4 * C))) return st;
