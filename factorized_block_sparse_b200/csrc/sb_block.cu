@@ -594,6 +594,37 @@ int mm_residual(cublasLtHandle_t lt, const void* A, const void* W, const void* R
   return st;
 }
 
+// A second stream per device, with a cuBLAS handle of its own, for the
+// weight gradients of the backward pass: they run beside the chain of data
+// gradients and join it before the call returns.  Created on first use,
+// under the call lock.
+struct Side {
+  cudaStream_t s = nullptr;
+  cublasHandle_t h = nullptr;
+  cudaEvent_t ev[5] = {};
+};
+
+Side* side_for_current_device() {
+  static Side sides[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  Side& sd = sides[dev];
+  if (sd.s) return &sd;
+  Side n;
+  bool ok = cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking) == cudaSuccess &&
+            cublasCreate(&n.h) == CUBLAS_STATUS_SUCCESS && cublasSetStream(n.h, n.s) == CUBLAS_STATUS_SUCCESS;
+  for (auto& e : n.ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    for (auto& e : n.ev)
+      if (e) cudaEventDestroy(e);
+    if (n.h) cublasDestroy(n.h);
+    if (n.s) cudaStreamDestroy(n.s);
+    return nullptr;
+  }
+  sd = n;
+  return &sd;
+}
+
 struct Gemm {
   cublasHandle_t h;
   // Row-major Out[M][Nn] = A[M][K] W[K][Nn] + beta Out (bf16 out).
@@ -815,33 +846,53 @@ int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx
   auto* dv = at<__nv_bfloat16>(ws, w.dv);
   auto* dqkv = at<__nv_bfloat16>(ws, w.dqkv);
   auto* da = at<__nv_bfloat16>(ws, w.da);
-  // feed-forward: y = h + gelu(f W1) W2
-  if ((st = G.mm_tn(g, dyb, gr->w_2, Mi, 4 * C, C))) return st;
-  if ((st = G.mm_nt(dyb, p->w_2, dg, Mi, 4 * C, C))) return st;
-  dgelu_mul_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(at<__nv_bfloat16>(ws, w.u), dg, du, M * 4 * C / 8);
-  if ((st = last_launch())) return st;
-  if ((st = G.mm_tn(f, du, gr->w_1, Mi, C, 4 * C))) return st;
-  if ((st = G.mm_nt(du, p->w_1, df, Mi, C, 4 * C))) return st;
-  if (cudaMemsetAsync(gr->ln2_g, 0, C * sizeof(float), s) != cudaSuccess ||
-      cudaMemsetAsync(gr->ln2_b, 0, C * sizeof(float), s) != cudaSuccess)
-    return SA_ERR_CUDA;
-  if ((st = ln_bwd(h, p->ln2_g, df, dyb, dh, gr->ln2_g, gr->ln2_b, M, C, s))) return st;
-  // attention: h = x + o Wo
-  if ((st = G.mm_tn(o2, dh, gr->w_o, Mi, C, C))) return st;
-  if ((st = G.mm_nt(dh, p->w_o, do2, Mi, C, C))) return st;
-  heads_kernel<true><<<heads_grid(M), heads_block(C), 0, s>>>(do2, dO, nullptr, nullptr, B, N, H, D, 1);
-  if ((st = last_launch())) return st;
-  if ((st = sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, D, layout, at<void>(ws, w.attn), w.attn_bytes,
-                            s)))
-    return st;
-  heads_kernel<false><<<heads_grid(M), heads_block(3 * C), 0, s>>>(dqkv, dq, dk, dv, B, N, H, D, 3);
-  if ((st = last_launch())) return st;
-  if ((st = G.mm_tn(a, dqkv, gr->w_qkv, Mi, C, 3 * C))) return st;
-  if ((st = G.mm_nt(dqkv, p->w_qkv, da, Mi, C, 3 * C))) return st;
-  if (cudaMemsetAsync(gr->ln1_g, 0, C * sizeof(float), s) != cudaSuccess ||
-      cudaMemsetAsync(gr->ln1_b, 0, C * sizeof(float), s) != cudaSuccess)
-    return SA_ERR_CUDA;
-  return ln_bwd(xb, p->ln1_g, da, dh, static_cast<__nv_bfloat16*>(dx), gr->ln1_g, gr->ln1_b, M, C, s);
+  // The weight gradients go to the side stream as soon as their operands
+  // exist (fork k: an event on the caller's stream that the side stream
+  // waits for); the side stream joins the caller's stream at the end, on
+  // every path that forked.
+  Side* sd = side_for_current_device();
+  if (!sd) return SA_ERR_CUDA;
+  const Gemm GS{sd->h};
+  bool forked = false;
+  auto fork = [&](int k) {
+    forked = true;
+    return cudaEventRecord(sd->ev[k], s) == cudaSuccess && cudaStreamWaitEvent(sd->s, sd->ev[k], 0) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+  };
+  auto chain = [&]() -> int {
+    // feed-forward: y = h + gelu(f W1) W2
+    if ((st = fork(0)) || (st = GS.mm_tn(g, dyb, gr->w_2, Mi, 4 * C, C))) return st;
+    if ((st = G.mm_nt(dyb, p->w_2, dg, Mi, 4 * C, C))) return st;
+    dgelu_mul_kernel<<<grid_for(M * 4 * C / 8, 256), 256, 0, s>>>(at<__nv_bfloat16>(ws, w.u), dg, du, M * 4 * C / 8);
+    if ((st = last_launch())) return st;
+    if ((st = fork(1)) || (st = GS.mm_tn(f, du, gr->w_1, Mi, C, 4 * C))) return st;
+    if ((st = G.mm_nt(du, p->w_1, df, Mi, C, 4 * C))) return st;
+    if (cudaMemsetAsync(gr->ln2_g, 0, C * sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(gr->ln2_b, 0, C * sizeof(float), s) != cudaSuccess)
+      return SA_ERR_CUDA;
+    if ((st = ln_bwd(h, p->ln2_g, df, dyb, dh, gr->ln2_g, gr->ln2_b, M, C, s))) return st;
+    // attention: h = x + o Wo
+    if ((st = fork(2)) || (st = GS.mm_tn(o2, dh, gr->w_o, Mi, C, C))) return st;
+    if ((st = G.mm_nt(dh, p->w_o, do2, Mi, C, C))) return st;
+    heads_kernel<true><<<heads_grid(M), heads_block(C), 0, s>>>(do2, dO, nullptr, nullptr, B, N, H, D, 1);
+    if ((st = last_launch())) return st;
+    if ((st = sparse_attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, D, layout, at<void>(ws, w.attn),
+                              w.attn_bytes, s)))
+      return st;
+    heads_kernel<false><<<heads_grid(M), heads_block(3 * C), 0, s>>>(dqkv, dq, dk, dv, B, N, H, D, 3);
+    if ((st = last_launch())) return st;
+    if ((st = fork(3)) || (st = GS.mm_tn(a, dqkv, gr->w_qkv, Mi, C, 3 * C))) return st;
+    if ((st = G.mm_nt(dqkv, p->w_qkv, da, Mi, C, 3 * C))) return st;
+    if (cudaMemsetAsync(gr->ln1_g, 0, C * sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(gr->ln1_b, 0, C * sizeof(float), s) != cudaSuccess)
+      return SA_ERR_CUDA;
+    return ln_bwd(xb, p->ln1_g, da, dh, static_cast<__nv_bfloat16*>(dx), gr->ln1_g, gr->ln1_b, M, C, s);
+  };
+  st = chain();
+  if (forked && (cudaEventRecord(sd->ev[4], sd->s) != cudaSuccess || cudaStreamWaitEvent(s, sd->ev[4], 0) != cudaSuccess))
+    st = st ? st : SA_ERR_CUDA;
+  return st;
 }
 
 }  // extern "C"

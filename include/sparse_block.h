@@ -110,6 +110,12 @@ int sparse_block_gelu(const void* u, void* g, void* dgelu, size_t n, void* strea
  * it first (the recomputation of the pages), then differentiated.  dq of the
  * attention, the projection-weight gradients and the layer-norm parameter
  * gradients are float32 sums whose last bits may vary from run to run.
+ * The projection-weight gradients are computed on a second stream of the
+ * library's own (one a device, with its own cuBLAS handle), forked from
+ * `stream` by events as their operands become ready and joined back into it
+ * before the call returns, so all of the call's work is ordered before what
+ * the caller enqueues on `stream` next (this fork and join can be captured
+ * into a CUDA graph).
  * Errors: as sparse_block_fwd, plus those of sparse_attn_bwd.
  */
 int sparse_block_bwd(const void* x, const void* dy, const sb_params* p, void* dx, const sb_grads* g,
