@@ -72,6 +72,8 @@ def _run(mode, B, N, H, D, l, c, block, device):
     ("local", 1, 256, 8, 128, 64, 0, 64),
     ("all", 1, 128, 12, 128, 1, 0, 64),
     ("all", 1, 128, 16, 128, 1, 0, 64),
+    # ragged: N = 1000 (M = 2000 rows, no multiple of a tile), a partial last row of the strided view
+    ("strided", 2, 1000, 2, 64, 64, 0, 8),
 ])
 def test_block_parity(cuda_device, mode, B, N, H, D, l, c, block):
     got, ref = _run(mode, B, N, H, D, l, c, block, cuda_device)
