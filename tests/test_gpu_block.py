@@ -127,3 +127,44 @@ def test_gelu_against_fp32_reference(cuda_device):
         bound = half_ulp(ref) + 1e-6
         assert torch.isfinite(got).all(), name
         assert (err <= bound).all(), f"{name}: worst excess {(err - bound).max().item():.3e}"
+
+
+def test_block_calls_from_two_threads(cuda_device):
+    """Two host threads, each with its own stream and workspace, run forward +
+    backward of the block at the same time: the results equal those of one
+    thread alone, bit for bit where the block is deterministic (y) and within
+    float32 reduction-order noise for the gradients."""
+    import threading
+
+    from factorized_block_sparse_b200 import sparse_attn as sa
+    from factorized_block_sparse_b200 import sparse_block as sb
+
+    B, N, H, D = 1, 512, 2, 64
+    lay = sa.Layout("fixed", N, 128, 32, 64)
+    lay.upload()
+    p = {k: v.to(cuda_device) for k, v in synth.block_params(H * D).items()}
+    xin = synth.block_inputs(B, N, H * D)
+    x, dy = xin["x"].to(cuda_device), xin["dy"].to(cuda_device)
+
+    def run(stream, out):
+        with torch.cuda.stream(stream):
+            ws = sb.workspace(B, N, H, D, lay, cuda_device)
+            for _ in range(3):
+                y = sb.forward(x, p, H, lay, ws, stream.cuda_stream)
+                dx, g = sb.backward(x, dy, p, H, lay, ws, stream.cuda_stream)
+            stream.synchronize()
+            out.update(y=y.float().cpu(), dx=dx.float().cpu(), w_1=g["w_1"].cpu(), ln1_g=g["ln1_g"].cpu())
+
+    ref = {}
+    run(torch.cuda.Stream(device=cuda_device), ref)
+    outs = [{}, {}]
+    threads = [threading.Thread(target=run, args=(torch.cuda.Stream(device=cuda_device), o)) for o in outs]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert sa.sparse_attn_status() == sa.SA_OK
+    for o in outs:
+        assert torch.equal(o["y"], ref["y"])
+        for name in ("dx", "w_1", "ln1_g"):
+            assert torch.allclose(o[name], ref[name], rtol=1e-2, atol=1e-3 * ref[name].abs().max().item()), name
